@@ -1,0 +1,345 @@
+"""Benchmark of the DuoAttention hybrid-GQA attention path on B200.
+
+Default workload (one GPU): one-token decode, B=32 sequences at context
+32768, 48 query / 8 KV heads, head_dim 128, 2 of 8 KV heads full-context
+(seeded mask), the other 6 streaming heads with 64 sink + 256 recent slots
+and ring pointers at random offsets.  A step is one ``duo_attn_decode`` over
+the whole batch.  Metric: algorithmic HBM bytes per second (K and V rows the
+heads must read, plus q and out), inputs resident in HBM and larger than L2.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+                  [--workload decode_b32|prefill_16k|sliding_32k|stack40]
+
+With N > 1 (torchrun, one process per GPU) every rank decodes its own batch
+of 32 (weak scaling, no data-path collective); the time is the max over ranks.
+``--impl reference`` times the float64 CPU oracle on this host's cores on a
+bounded sample of the same workload, in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kv_cache_reduction_b200 as duo  # noqa: E402
+from kv_cache_reduction_b200 import inputs  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "decode attn HBM GB/s (% of ~8 TB/s); prefill attn TFLOP/s (% bf16 peak)"
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, p in rows:
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        busy = [r[0] for r in rows] or [0.0]
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ workloads
+class DecodeB32:
+    """One-token decode at context 32768 for 32 sequences."""
+
+    def __init__(self, rank: int):
+        w = self.w = inputs.workload("decode_b32")
+        B, n = w.batch, w.seq_len
+        self.params = duo.DuoParams(B, 48, 8, 128, inputs.SINK, inputs.RECENT, 0, 128 ** -0.5,
+                                    w.full_mask, None)
+        seed = w.seed + 7919 * rank
+        self.cache = duo.DuoCache.allocate(self.params, n)
+        for i, t in enumerate((self.cache.full_k, self.cache.full_v, self.cache.strm_k,
+                               self.cache.strm_v)):
+            inputs.randn_bf16_into(t, seed * 10 + i)
+        rng = np.random.default_rng(seed)
+        self.cache.seq_len.fill_(n)
+        self.cache.ring_head.copy_(torch.as_tensor(rng.integers(0, inputs.RECENT, size=B),
+                                                   dtype=torch.int32))
+        self.q = inputs.randn_bf16((B, 48, 128), seed + 5, "cuda")
+        self.out = torch.empty((B, 48, 128), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty((B, 48), dtype=torch.float32, device="cuda")
+        self.ws = duo.workspace_for(self.params, n)
+        # algorithmic bytes: K and V rows each head reads, plus q and out
+        n_full, n_ring = self.params.n_full, self.params.n_ring
+        rows = B * (n_full * n + n_ring * min(n, inputs.SINK + inputs.RECENT))
+        self.bytes = rows * 2 * 128 * 2 + 2 * self.q.numel() * 2
+        self.launches_per_step = 2
+        self.unit = "GB/s"
+
+    def step(self):
+        duo.duo_attn_decode(self.params, self.cache, self.q, self.w.seq_len, self.out, self.lse,
+                            self.ws)
+
+    def e2e_buffers(self):
+        self.h_q = self.q.cpu().pin_memory()
+        self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h_lse = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
+        self.d_q = torch.empty_like(self.q)
+        return self.h_q.numel() * 2, self.h_out.numel() * 2 + self.h_lse.numel() * 4
+
+    def e2e_step(self):
+        self.d_q.copy_(self.h_q, non_blocking=True)
+        duo.duo_attn_decode(self.params, self.cache, self.d_q, self.w.seq_len, self.out, self.lse,
+                            self.ws)
+        self.h_out.copy_(self.out, non_blocking=True)
+        self.h_lse.copy_(self.lse, non_blocking=True)
+
+    def config(self):
+        return {"workload": "decode_b32: one-token decode, B=32, context 32768, 48 Q / 8 KV heads, "
+                            "head_dim 128, 2 of 8 KV heads full, sink 64 + recent 256 ring",
+                "batch_per_gpu": self.w.batch, "context": self.w.seq_len,
+                "full_mask": list(self.w.full_mask),
+                "l2": "inputs larger than L2 (1.1 GB of cache per step)"}
+
+    # -------------------------------------------------- CPU oracle on a bounded sample
+    def oracle_sample(self, budget_s: float = 15.0):
+        import oracle
+        p = self.params
+        olayer = oracle.Layer(p.batch, 48, 8, 128, p.sink, p.recent, 0, p.softmax_scale,
+                              p.full_mask, None)
+        hc = oracle.Cache(olayer, self.w.seq_len)
+        hc.full_k, hc.full_v = inputs.bits(self.cache.full_k), inputs.bits(self.cache.full_v)
+        hc.strm_k, hc.strm_v = inputs.bits(self.cache.strm_k), inputs.bits(self.cache.strm_v)
+        hc.seq_len = self.cache.seq_len.cpu().numpy().astype(np.int32)
+        hc.ring_head = self.cache.ring_head.cpu().numpy().astype(np.int32)
+        qb = inputs.bits(self.q)
+        n = self.w.seq_len
+        units = [(b, g) for b in range(p.batch) for g in range(8)]
+        done_bytes, t_total, used = 0, 0.0, 0
+        for b, g in units:        # whole GQA groups, in order, until the time budget is spent
+            rows = [b * 48 + g * 6 + j for j in range(6)]
+            t0 = time.perf_counter()
+            oracle.attn_decode(olayer, hc, qb, rows=rows)
+            t_total += time.perf_counter() - t0
+            tokens = n if p.full_mask[g] else min(n, p.sink + p.recent)
+            done_bytes += tokens * 512 + 6 * 2 * 256
+            used += 1
+            if t_total >= budget_s:
+                break
+        return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+                "kind": "oracle",
+                "sample": f"{used} of {len(units)} (sequence, KV head) groups of one decode step "
+                          f"(6 query heads each), float64, {t_total:.1f} s"}
+
+
+WORKLOADS = {"decode_b32": DecodeB32}
+
+
+# ------------------------------------------------------------------ timing
+def time_steps(fn, steps, stream, world):
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(stop) / 1e3
+
+
+def run_ours(args, world, rank):
+    wl = WORKLOADS[args.workload](rank)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+    if duo.duo_get_device_status() != duo.DUO_OK:
+        raise RuntimeError("device status error during warm-up")
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t = time_steps(wl.step, args.steps, stream, world)
+    t = max_over_ranks(t, world)
+    clocks = clk.summary()
+    # end to end: host buffers, copies inside the timed region
+    h2d, d2h = wl.e2e_buffers()
+    for _ in range(max(1, args.warmup)):
+        wl.e2e_step()
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(time_steps(wl.e2e_step, args.steps, stream, world), world)
+    if duo.duo_get_device_status() != duo.DUO_OK:
+        raise RuntimeError("device status error during timing")
+    pk, pk_kind = peaks()
+    per_step = t / args.steps
+    value = wl.bytes * world / per_step / 1e9
+    achieved = wl.bytes / per_step / 1e9
+    res = {"metric": METRIC, "value": round(value, 2), "unit": wl.unit, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 4),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded N(0,1) bf16 caches and queries)",
+           "config": {**wl.config(), "parallelism": f"dp{world} (independent batches)"},
+           "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
+                        "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                        "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)",
+                        "kernel": "decode_split + decode_merge (one duo_attn_decode call)"},
+           "e2e": {"value": round(wl.bytes * world / (t_e2e / args.steps) / 1e9, 2),
+                   "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+           "gpu_launches": wl.launches_per_step * args.steps,
+           "clocks": clocks}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = wl.oracle_sample(args.cpu_budget)
+    return res
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle
+    wl = WORKLOADS[args.workload](0)
+    vals = []
+    samples = []
+    per = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        r = wl.oracle_sample(per)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            samples.append(r["sample"])
+    v = statistics.median(vals)
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) bf16 caches and queries)",
+            "config": {**wl.config(), "parallelism": "CPU oracle, rank 0 only"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": samples[0]},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b32")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # the CPU oracle runs on rank 0 only; no process group is needed
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:
+            return
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        res = run_reference(args, world, rank)
+        print(json.dumps(res), flush=True)
+        return
+    world, rank = dist_init()
+    try:
+        res = run_ours(args, world, rank) if args.impl == "ours" else run_reference(args, world, rank)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,168 @@
+/*
+ * duo_attn.h -- C ABI of the B200 (sm_100a) DuoAttention hybrid-GQA
+ * attention library (libduoattn.so).
+ *
+ * What is computed (DuoAttention Laguna Adapter model card, sections Summary
+ * and Why It Works; Laguna sliding-window articles; Laguna-XS-2.1 cookbook,
+ * section 1): each KV head of a layer is
+ *   - a full-context head: the query at position i attends to every key
+ *     j <= i, and the cache keeps every token;
+ *   - a streaming head: the query attends to keys j <= i with j < sink or
+ *     j > i - recent (sink 64, recent 256 on the pages), and the cache keeps
+ *     only those: `sink` fixed slots plus a ring of `recent` slots;
+ *   - on a sliding-window layer (window > 0, 512 on the pages) every head
+ *     attends to keys i - window < j <= i and keeps a ring of `window` slots.
+ * Query head h reads KV head h / (num_q_heads / num_kv_heads).  Scores are
+ * softmax_scale * q.k; an optional per-query-head sink logit (not scaled)
+ * joins the softmax denominator with a zero value vector, and the exported
+ * log-sum-exp (natural log) includes it.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     keeps no pointer after the call returns and allocates no device memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on that stream; a non-negative return only means the work
+ *     was enqueued.
+ *   - bf16 tensors are dense row-major with the shapes given; every tensor
+ *     pointer must be 16-byte aligned.
+ *   - Arguments are checked on the host before anything is launched; a call
+ *     that returns an error has launched nothing and written nothing.
+ *     Conditions that only the device can see (cache capacity overflow, a
+ *     bounded wait that expired) set a device status word that
+ *     duo_get_device_status() returns.
+ *   - Supported geometry: head_dim 128, num_q_heads / num_kv_heads == 6,
+ *     num_kv_heads <= 64, sequence positions below 2^30.
+ */
+#ifndef DUO_ATTN_H
+#define DUO_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DUO_API __attribute__((visibility("default")))
+#else
+#define DUO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return and status codes. */
+#define DUO_OK 0
+#define DUO_ERR_INVALID_ARG (-1) /* NULL / misaligned pointer, bad size or range   */
+#define DUO_ERR_UNSUPPORTED (-2) /* geometry outside what the kernels implement     */
+#define DUO_ERR_CUDA (-3)        /* a CUDA runtime call or a launch failed          */
+#define DUO_ERR_WORKSPACE (-4)   /* decode workspace NULL or smaller than required  */
+#define DUO_ERR_TIMEOUT (-5)     /* device: a bounded wait inside a kernel expired  */
+#define DUO_ERR_CAPACITY (-6)    /* device: an append ran past the full-cache capacity */
+#define DUO_ERR_DEVICE (-7)      /* the current device is not sm_100 (B200)          */
+
+/* One attention layer.
+ *   window > 0 : sliding-window layer; full_mask, sink and recent are ignored.
+ *   window == 0: DuoAttention layer; full_mask[g] == 1 marks KV head g as a
+ *                full-context head, 0 as a streaming head (sink + recent).
+ * full_mask is a HOST array [num_kv_heads]; sink_logit is a DEVICE array
+ * [num_q_heads] of fp32 logits, or NULL for none. */
+typedef struct {
+    int32_t batch;          /* B >= 1                                        */
+    int32_t num_q_heads;    /* Hq (48 on the pages)                          */
+    int32_t num_kv_heads;   /* Hkv (8 on the pages); Hq == 6 * Hkv           */
+    int32_t head_dim;       /* D, must be 128                                */
+    int32_t sink;           /* streaming heads: sink tokens kept (64), >= 0  */
+    int32_t recent;         /* streaming heads: recent tokens kept (256), >= 1 */
+    int32_t window;         /* 0, or the sliding window (512), <= 8192       */
+    float softmax_scale;    /* > 0, usually 1/sqrt(D)                        */
+    const uint8_t *full_mask;  /* host [Hkv]                                 */
+    const float *sink_logit;   /* device [Hq] fp32, or NULL                  */
+} duo_params;
+
+/* A layer's KV cache (all device memory, bf16, caller-owned).
+ * Let n_full = number of full heads (0 on a sliding layer), n_ring =
+ * Hkv - n_full, and ring_slots = sink + recent (Duo layer) or window
+ * (sliding layer).  Head g's slot in either array is its rank among the
+ * heads of its kind (the number of same-kind heads with a lower index).
+ *   full_k, full_v : [B][n_full][capacity][D]  (may be NULL if n_full == 0)
+ *   strm_k, strm_v : [B][n_ring][ring_slots][D] (may be NULL if n_ring == 0)
+ *                    slots 0..sink-1 hold positions 0..sink-1; slots
+ *                    sink..ring_slots-1 form the ring of recent tokens.
+ *   seq_len        : device int32 [B], tokens appended so far.
+ *   ring_head      : device int32 [B], ring slot (0..ring_slots-sink-1,
+ *                    relative to the first ring slot) that the next ring
+ *                    write goes to.  It advances once per appended position
+ *                    >= sink.  Any starting value is allowed.
+ * The valid ring slots are the min(max(seq_len - sink, 0), ring size) slots
+ * written last, i.e. those just before ring_head, cyclically. */
+typedef struct {
+    void *full_k;
+    void *full_v;
+    int64_t capacity;       /* rows per full head, >= the longest sequence  */
+    void *strm_k;
+    void *strm_v;
+    int32_t *seq_len;
+    int32_t *ring_head;
+} duo_cache;
+
+/* Appends n_new tokens to every sequence of the cache.
+ * k, v: device bf16 [B][n_new][Hkv][D] (token-major, as a K/V projection
+ * writes them).  For each sequence b and token t the position is
+ * p = seq_len[b] + t; a full head writes row p of its full cache; a
+ * streaming / sliding head writes slot p if p < sink, else the ring slot the
+ * sequential rule gives, and only tokens that would still be in the ring
+ * after all n_new appends are written (the result equals n_new one-token
+ * appends).  Afterwards seq_len[b] += n_new and ring_head advances.
+ * p >= capacity on a full head sets DUO_ERR_CAPACITY on the device and skips
+ * that write.  Defined by the DuoAttention card, section Summary (sink and
+ * recent sizes) and section Why It Works (what each head keeps). */
+DUO_API int duo_kv_append(const duo_params *params, const duo_cache *cache, const void *k,
+                  const void *v, int32_t n_new, void *stream);
+
+/* Prefill attention over a sequence that starts at position 0 (empty cache).
+ * q: device bf16 [B][L][Hq][D]; k, v: device bf16 [B][L][Hkv][D]; L = seq_len.
+ * out: device bf16 [B][L][Hq][D].  lse: device fp32 [B][Hq][L] (natural-log
+ * log-sum-exp of the row's scores, sink term included) or NULL.
+ * Query i of head h attends to the keys its KV head's rule allows (full:
+ * j <= i; streaming: j < sink or i - recent < j <= i; sliding:
+ * i - window < j <= i).  Computed with tcgen05 tensor cores (bf16 inputs,
+ * fp32 accumulation, probabilities rounded to bf16 before the PV product).
+ * The cache is not touched: call duo_kv_append(n_new = L) to fill it. */
+DUO_API int duo_attn_prefill(const duo_params *params, const void *q, const void *k, const void *v,
+                     int32_t seq_len, void *out, float *lse, void *stream);
+
+/* Bytes of device workspace duo_attn_decode needs for this layer when no
+ * sequence holds more than max_seq_len tokens.  Returns 0 on invalid params. */
+DUO_API size_t duo_decode_workspace_bytes(const duo_params *params, int32_t max_seq_len);
+
+/* One-token decode against the cache: the query of sequence b sits at
+ * position seq_len[b] - 1 (append its K/V first).
+ * q: device bf16 [B][Hq][D]; out: device bf16 [B][Hq][D]; lse: device fp32
+ * [B][Hq] or NULL.  max_seq_len bounds every seq_len[b] (it sizes the split
+ * of long caches into parallel pieces; a sequence longer than it is an error
+ * the device cannot report, so pass a true bound).  workspace: device memory
+ * of at least duo_decode_workspace_bytes(params, max_seq_len) bytes, 256-byte
+ * aligned, contents need not be initialised.  A full head reads its seq_len
+ * rows, a ring head only its valid sink and ring slots (at most
+ * sink + recent or window).  A sequence with seq_len 0 gives out = 0 and
+ * lse = -inf (or the sink logit when one is given). */
+DUO_API int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void *q,
+                    int32_t max_seq_len, void *out, float *lse, void *workspace,
+                    size_t workspace_bytes, void *stream);
+
+/* Reads and clears the device status word of the current device after
+ * synchronising `stream`: DUO_OK, DUO_ERR_TIMEOUT or DUO_ERR_CAPACITY (the
+ * first error any kernel recorded since the last read), or DUO_ERR_CUDA. */
+DUO_API int duo_get_device_status(void *stream);
+
+/* Short English text for a return or status code (static storage). */
+DUO_API const char *duo_status_string(int code);
+
+/* Text of the last host-side error on the calling thread (static storage of
+ * that thread; "" if none). */
+DUO_API const char *duo_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DUO_ATTN_H */

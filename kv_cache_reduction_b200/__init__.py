@@ -1,1 +1,233 @@
-"""B200-native DuoAttention hybrid-GQA attention (placeholder until the binding lands)."""
+"""B200-native (sm_100a) DuoAttention hybrid-GQA attention.
+
+Thin ctypes binding over ``libduoattn.so`` (the C ABI declared in
+``include/duo_attn.h``).  The functions below carry the C names and only
+marshal arguments: torch tensors are passed as device pointers and the
+current CUDA stream as the stream handle.  Every step of the attention runs
+in the library's CUDA kernels; there is no Python or CPU fallback, and a
+missing library raises ``DuoLibraryMissing``.
+
+Layouts (bf16 unless noted):
+  prefill  q [B][L][Hq][D], k/v [B][L][Hkv][D] -> out [B][L][Hq][D], lse fp32 [B][Hq][L]
+  append   k/v [B][n_new][Hkv][D] into the cache
+  decode   q [B][Hq][D] -> out [B][Hq][D], lse fp32 [B][Hq]
+  cache    full_k/v [B][n_full][capacity][D], strm_k/v [B][n_ring][ring_slots][D],
+           seq_len, ring_head int32 [B]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libduoattn.so")
+
+DUO_OK = 0
+DUO_ERR_INVALID_ARG = -1
+DUO_ERR_UNSUPPORTED = -2
+DUO_ERR_CUDA = -3
+DUO_ERR_WORKSPACE = -4
+DUO_ERR_TIMEOUT = -5
+DUO_ERR_CAPACITY = -6
+DUO_ERR_DEVICE = -7
+
+EXPORTED = ("duo_kv_append", "duo_attn_prefill", "duo_decode_workspace_bytes", "duo_attn_decode",
+            "duo_get_device_status", "duo_status_string", "duo_last_error")
+
+
+class DuoLibraryMissing(RuntimeError):
+    pass
+
+
+class DuoError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"{message} (code {code})")
+        self.code = code
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("sink", ctypes.c_int32), ("recent", ctypes.c_int32),
+                ("window", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("full_mask", ctypes.c_void_p), ("sink_logit", ctypes.c_void_p)]
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [("full_k", ctypes.c_void_p), ("full_v", ctypes.c_void_p),
+                ("capacity", ctypes.c_int64), ("strm_k", ctypes.c_void_p),
+                ("strm_v", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
+                ("ring_head", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIBRARY_PATH) -> ctypes.CDLL:
+    """Loads libduoattn.so (raises DuoLibraryMissing if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise DuoLibraryMissing(
+            f"{path} is missing: build it with `python -m kv_cache_reduction_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, C, vp = ctypes.POINTER(_Params), ctypes.POINTER(_Cache), ctypes.c_void_p
+    lib.duo_kv_append.argtypes = [P, C, vp, vp, ctypes.c_int32, vp]
+    lib.duo_kv_append.restype = ctypes.c_int
+    lib.duo_attn_prefill.argtypes = [P, vp, vp, vp, ctypes.c_int32, vp, vp, vp]
+    lib.duo_attn_prefill.restype = ctypes.c_int
+    lib.duo_decode_workspace_bytes.argtypes = [P, ctypes.c_int32]
+    lib.duo_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.duo_attn_decode.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.duo_attn_decode.restype = ctypes.c_int
+    lib.duo_get_device_status.argtypes = [vp]
+    lib.duo_get_device_status.restype = ctypes.c_int
+    lib.duo_status_string.argtypes = [ctypes.c_int]
+    lib.duo_status_string.restype = ctypes.c_char_p
+    lib.duo_last_error.argtypes = []
+    lib.duo_last_error.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+@dataclass
+class DuoParams:
+    """One attention layer (mirrors ``duo_params``).
+
+    ``full_mask`` is a host sequence of 0/1 per KV head (ignored when
+    window > 0); ``sink_logit`` is a device fp32 tensor [Hq] or None.
+    """
+    batch: int
+    num_q_heads: int = 48
+    num_kv_heads: int = 8
+    head_dim: int = 128
+    sink: int = 64
+    recent: int = 256
+    window: int = 0
+    softmax_scale: float = 128 ** -0.5
+    full_mask: Sequence[int] = (0,) * 8
+    sink_logit: Optional[torch.Tensor] = None
+    _mask_buf: ctypes.Array = field(default=None, repr=False, compare=False)
+
+    def as_c(self) -> _Params:
+        self._mask_buf = (ctypes.c_uint8 * max(1, len(self.full_mask)))(*[int(m) for m in self.full_mask])
+        return _Params(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.sink,
+                       self.recent, self.window, float(self.softmax_scale),
+                       ctypes.addressof(self._mask_buf), _ptr(self.sink_logit))
+
+    @property
+    def n_full(self) -> int:
+        return 0 if self.window > 0 else sum(1 for m in self.full_mask if m)
+
+    @property
+    def n_ring(self) -> int:
+        return self.num_kv_heads - self.n_full
+
+    @property
+    def ring_slots(self) -> int:
+        return self.window if self.window > 0 else self.sink + self.recent
+
+
+@dataclass
+class DuoCache:
+    """Device KV cache of one layer (mirrors ``duo_cache``); tensors are caller-owned."""
+    full_k: Optional[torch.Tensor]
+    full_v: Optional[torch.Tensor]
+    capacity: int
+    strm_k: Optional[torch.Tensor]
+    strm_v: Optional[torch.Tensor]
+    seq_len: torch.Tensor
+    ring_head: torch.Tensor
+
+    @staticmethod
+    def allocate(params: DuoParams, capacity: int, device="cuda") -> "DuoCache":
+        B, D = params.batch, params.head_dim
+        kw = dict(dtype=torch.bfloat16, device=device)
+        fk = torch.empty((B, params.n_full, capacity, D), **kw) if params.n_full else None
+        fv = torch.empty_like(fk) if fk is not None else None
+        sk = torch.empty((B, params.n_ring, params.ring_slots, D), **kw) if params.n_ring else None
+        sv = torch.empty_like(sk) if sk is not None else None
+        return DuoCache(fk, fv, capacity, sk, sv,
+                        torch.zeros((B,), dtype=torch.int32, device=device),
+                        torch.zeros((B,), dtype=torch.int32, device=device))
+
+    def as_c(self) -> _Cache:
+        return _Cache(_ptr(self.full_k), _ptr(self.full_v), int(self.capacity), _ptr(self.strm_k),
+                      _ptr(self.strm_v), _ptr(self.seq_len), _ptr(self.ring_head))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(rc: int) -> int:
+    if rc < 0:
+        lib = load_library()
+        raise DuoError(rc, (lib.duo_last_error() or b"").decode() or
+                       lib.duo_status_string(rc).decode())
+    return rc
+
+
+def duo_kv_append(params: DuoParams, cache: DuoCache, k: torch.Tensor, v: torch.Tensor,
+                  n_new: Optional[int] = None, stream=None) -> None:
+    n_new = int(k.shape[1]) if n_new is None else int(n_new)
+    p, c = params.as_c(), cache.as_c()
+    _check(load_library().duo_kv_append(ctypes.byref(p), ctypes.byref(c), _ptr(k), _ptr(v), n_new,
+                                        _stream(stream)))
+
+
+def duo_attn_prefill(params: DuoParams, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                     out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                     seq_len: Optional[int] = None, stream=None) -> None:
+    L = int(q.shape[1]) if seq_len is None else int(seq_len)
+    p = params.as_c()
+    _check(load_library().duo_attn_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), L, _ptr(out),
+                                           _ptr(lse), _stream(stream)))
+
+
+def duo_decode_workspace_bytes(params: DuoParams, max_seq_len: int) -> int:
+    p = params.as_c()
+    return int(load_library().duo_decode_workspace_bytes(ctypes.byref(p), int(max_seq_len)))
+
+
+def duo_attn_decode(params: DuoParams, cache: DuoCache, q: torch.Tensor, max_seq_len: int,
+                    out: torch.Tensor, lse: Optional[torch.Tensor], workspace: torch.Tensor,
+                    stream=None) -> None:
+    p, c = params.as_c(), cache.as_c()
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load_library().duo_attn_decode(ctypes.byref(p), ctypes.byref(c), _ptr(q), int(max_seq_len),
+                                          _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
+                                          _stream(stream)))
+
+
+def duo_get_device_status(stream=None) -> int:
+    return int(load_library().duo_get_device_status(_stream(stream)))
+
+
+def duo_status_string(code: int) -> str:
+    return load_library().duo_status_string(int(code)).decode()
+
+
+def duo_last_error() -> str:
+    return (load_library().duo_last_error() or b"").decode()
+
+
+def workspace_for(params: DuoParams, max_seq_len: int, device="cuda") -> torch.Tensor:
+    """Allocates a decode workspace of the size the library asks for (torch memory)."""
+    n = max(duo_decode_workspace_bytes(params, max_seq_len), 256)
+    return torch.empty((n + 255) // 256 * 256, dtype=torch.uint8, device=device)

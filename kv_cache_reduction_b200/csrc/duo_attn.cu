@@ -1,0 +1,342 @@
+// duo_attn.cu -- the C ABI of libduoattn.so: argument checks, work
+// planning and kernel launches.  Every check runs on the host before the
+// first launch, so a call that returns an error has launched nothing.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/duo_attn.h"
+#include "decode.cuh"
+#include "kv_append.cuh"
+#include "prefill.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+constexpr int kMaxHkv = 64;
+constexpr int kMaxWindow = 8192;
+constexpr int kMaxRing = 8192;
+constexpr int64_t kMaxPos = (int64_t)1 << 30;
+
+struct Layout {
+    bool sliding;
+    int n_full, n_ring;
+    int sink, ring, slots;     // ring cache geometry
+    duo::HeadTable heads;
+    int8_t full_head[64], ring_head_of[64];
+};
+
+int check_device(int *sm_count) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(DUO_ERR_CUDA, "cudaGetDevice failed");
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+        return fail(DUO_ERR_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                    major, minor);
+    if (sm_count) cudaDeviceGetAttribute(sm_count, cudaDevAttrMultiProcessorCount, dev);
+    return DUO_OK;
+}
+
+int check_params(const duo_params *p, Layout *lay) {
+    if (!p) return fail(DUO_ERR_INVALID_ARG, "params is NULL");
+    if (p->batch < 1) return fail(DUO_ERR_INVALID_ARG, "batch must be >= 1 (got %d)", p->batch);
+    if (p->head_dim != duo::kD)
+        return fail(DUO_ERR_UNSUPPORTED, "head_dim must be 128 (got %d)", p->head_dim);
+    if (p->num_kv_heads < 1 || p->num_kv_heads > kMaxHkv)
+        return fail(DUO_ERR_UNSUPPORTED, "num_kv_heads must be in [1, %d]", kMaxHkv);
+    if (p->num_q_heads != duo::kGroup * p->num_kv_heads)
+        return fail(DUO_ERR_UNSUPPORTED, "num_q_heads must be 6 * num_kv_heads (got %d, %d)",
+                    p->num_q_heads, p->num_kv_heads);
+    if (!(p->softmax_scale > 0.f) || !std::isfinite(p->softmax_scale))
+        return fail(DUO_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if (p->window < 0 || p->window > kMaxWindow)
+        return fail(DUO_ERR_INVALID_ARG, "window must be in [0, %d]", kMaxWindow);
+    if (p->sink_logit && !aligned16(p->sink_logit))
+        return fail(DUO_ERR_INVALID_ARG, "sink_logit must be 16-byte aligned");
+    Layout L{};
+    L.sliding = p->window > 0;
+    if (L.sliding) {
+        L.sink = 0;
+        L.ring = p->window;
+    } else {
+        if (!p->full_mask) return fail(DUO_ERR_INVALID_ARG, "full_mask is NULL on a DuoAttention layer");
+        if (p->sink < 0 || p->recent < 1 || (int64_t)p->sink + p->recent > kMaxRing)
+            return fail(DUO_ERR_INVALID_ARG, "need sink >= 0, recent >= 1, sink + recent <= %d",
+                        kMaxRing);
+        L.sink = p->sink;
+        L.ring = p->recent;
+    }
+    L.slots = L.sink + L.ring;
+    for (int g = 0; g < p->num_kv_heads; ++g) {
+        const bool full = !L.sliding && p->full_mask[g] != 0;
+        if (!L.sliding && p->full_mask[g] > 1)
+            return fail(DUO_ERR_INVALID_ARG, "full_mask[%d] must be 0 or 1", g);
+        L.heads.is_full[g] = full ? 1 : 0;
+        if (full) {
+            L.heads.rank[g] = (int8_t)L.n_full;
+            L.full_head[L.n_full++] = (int8_t)g;
+        } else {
+            L.heads.rank[g] = (int8_t)L.n_ring;
+            L.ring_head_of[L.n_ring++] = (int8_t)g;
+        }
+    }
+    *lay = L;
+    return DUO_OK;
+}
+
+int check_cache(const duo_cache *c, const Layout &L) {
+    if (!c) return fail(DUO_ERR_INVALID_ARG, "cache is NULL");
+    if (!c->seq_len || !c->ring_head) return fail(DUO_ERR_INVALID_ARG, "seq_len / ring_head is NULL");
+    if (L.n_full > 0) {
+        if (!c->full_k || !c->full_v) return fail(DUO_ERR_INVALID_ARG, "full_k / full_v is NULL");
+        if (!aligned16(c->full_k) || !aligned16(c->full_v))
+            return fail(DUO_ERR_INVALID_ARG, "full_k / full_v must be 16-byte aligned");
+        if (c->capacity < 1 || c->capacity > kMaxPos)
+            return fail(DUO_ERR_INVALID_ARG, "capacity must be in [1, 2^30]");
+    }
+    if (L.n_ring > 0) {
+        if (!c->strm_k || !c->strm_v) return fail(DUO_ERR_INVALID_ARG, "strm_k / strm_v is NULL");
+        if (!aligned16(c->strm_k) || !aligned16(c->strm_v))
+            return fail(DUO_ERR_INVALID_ARG, "strm_k / strm_v must be 16-byte aligned");
+    }
+    if (((uintptr_t)c->seq_len & 3u) || ((uintptr_t)c->ring_head & 3u))
+        return fail(DUO_ERR_INVALID_ARG, "seq_len / ring_head must be 4-byte aligned");
+    return DUO_OK;
+}
+
+int launch_status(const char *what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DUO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return DUO_OK;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device.
+template <typename Kernel>
+int set_smem_once(Kernel kernel, size_t bytes, const char *name, bool (&done)[64]) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && done[dev]) return DUO_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return fail(DUO_ERR_CUDA, "cudaFuncSetAttribute(%s) failed", name);
+    if (dev >= 0 && dev < 64) done[dev] = true;
+    return DUO_OK;
+}
+
+// ------------------------------------------------------------------ decode plan
+struct DecodePlan {
+    int chunk_full = duo::kDecTile, splits_full = 0;
+    int chunk_ring = duo::kDecTile, splits_ring = 0;
+    int max_splits = 1;
+    int64_t items = 0;
+};
+
+int round_up(int64_t x, int m) { return (int)((x + m - 1) / m * m); }
+
+// Splits long full-head caches so that the grid holds about eight CTAs per
+// SM in total (one CTA is resident per SM), and ring heads into pieces of
+// whole tiles when there are too few of them to fill the GPU.
+DecodePlan plan_decode(const duo_params *p, const Layout &L, int64_t max_n, int sms) {
+    DecodePlan d;
+    const int64_t ring_units = (int64_t)p->batch * L.n_ring;
+    const int64_t full_units = (int64_t)p->batch * L.n_full;
+    const int ring_valid = L.slots;
+    if (ring_units > 0) {
+        int want = (int)std::max<int64_t>(1, (2 * sms + ring_units - 1) / ring_units);
+        if (full_units > 0 && max_n > 4 * ring_valid) want = 1;   // full heads fill the GPU
+        const int max_pieces = (ring_valid + duo::kDecTile - 1) / duo::kDecTile;
+        want = std::min(want, max_pieces);
+        d.chunk_ring = round_up((ring_valid + want - 1) / want, duo::kDecTile);
+        d.splits_ring = (ring_valid + d.chunk_ring - 1) / d.chunk_ring;
+    }
+    if (full_units > 0) {
+        const int64_t n = std::max<int64_t>(max_n, 1);
+        const int64_t budget = std::max<int64_t>(8 * (int64_t)sms - ring_units * d.splits_ring, 4 * sms);
+        int64_t chunk = (full_units * n + budget - 1) / budget;
+        chunk = std::max<int64_t>(round_up(chunk, duo::kDecTile), 256);
+        d.chunk_full = (int)std::min<int64_t>(chunk, round_up(n, duo::kDecTile));
+        d.splits_full = (int)((n + d.chunk_full - 1) / d.chunk_full);
+    }
+    d.max_splits = std::max(1, std::max(d.splits_full, d.splits_ring));
+    d.items = full_units * d.splits_full + ring_units * d.splits_ring;
+    return d;
+}
+
+size_t workspace_bytes(const duo_params *p, const DecodePlan &d) {
+    return (size_t)p->batch * p->num_kv_heads * d.max_splits * duo::kPartFloats * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *duo_last_error(void) { return g_err; }
+
+const char *duo_status_string(int code) {
+    switch (code) {
+    case DUO_OK: return "ok";
+    case DUO_ERR_INVALID_ARG: return "invalid argument";
+    case DUO_ERR_UNSUPPORTED: return "unsupported geometry";
+    case DUO_ERR_CUDA: return "CUDA error";
+    case DUO_ERR_WORKSPACE: return "workspace missing or too small";
+    case DUO_ERR_TIMEOUT: return "a bounded device wait expired";
+    case DUO_ERR_CAPACITY: return "append past the full-cache capacity";
+    case DUO_ERR_DEVICE: return "device is not sm_100";
+    default: return "unknown status";
+    }
+}
+
+int duo_kv_append(const duo_params *params, const duo_cache *cache, const void *k, const void *v,
+                  int32_t n_new, void *stream) {
+    Layout L;
+    int rc = check_params(params, &L);
+    if (rc) return rc;
+    if ((rc = check_cache(cache, L))) return rc;
+    if (n_new < 0 || n_new > kMaxPos) return fail(DUO_ERR_INVALID_ARG, "n_new must be in [0, 2^30]");
+    if (n_new == 0) return DUO_OK;
+    if (!k || !v) return fail(DUO_ERR_INVALID_ARG, "k / v is NULL");
+    if (!aligned16(k) || !aligned16(v)) return fail(DUO_ERR_INVALID_ARG, "k / v must be 16-byte aligned");
+    if ((rc = check_device(nullptr))) return rc;
+    duo::AppendArgs a{};
+    a.k = (const uint4 *)k;
+    a.v = (const uint4 *)v;
+    a.full_k = (uint4 *)cache->full_k;
+    a.full_v = (uint4 *)cache->full_v;
+    a.strm_k = (uint4 *)cache->strm_k;
+    a.strm_v = (uint4 *)cache->strm_v;
+    a.seq_len = cache->seq_len;
+    a.ring_head = cache->ring_head;
+    a.capacity = L.n_full > 0 ? cache->capacity : 0;
+    a.batch = params->batch;
+    a.n_new = n_new;
+    a.hkv = params->num_kv_heads;
+    a.n_full = L.n_full;
+    a.n_ring = L.n_ring;
+    a.sink = L.sink;
+    a.ring = L.ring;
+    a.slots = L.slots;
+    a.heads = L.heads;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t vecs = (int64_t)params->batch * n_new * params->num_kv_heads * duo::kVecPerRow;
+    const int64_t blocks = (vecs + 255) / 256;
+    if (blocks > INT32_MAX) return fail(DUO_ERR_INVALID_ARG, "append too large for one launch");
+    duo::kv_append_scatter<<<(unsigned)blocks, 256, 0, st>>>(a);
+    if ((rc = launch_status("kv_append_scatter"))) return rc;
+    duo::kv_append_commit<<<(params->batch + 127) / 128, 128, 0, st>>>(
+        cache->seq_len, cache->ring_head, params->batch, n_new, L.sink, L.ring);
+    return launch_status("kv_append_commit");
+}
+
+size_t duo_decode_workspace_bytes(const duo_params *params, int32_t max_seq_len) {
+    Layout L;
+    if (check_params(params, &L) || max_seq_len < 0) return 0;
+    int sms = 148;
+    if (check_device(&sms)) sms = 148;
+    return workspace_bytes(params, plan_decode(params, L, max_seq_len, sms));
+}
+
+int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void *q,
+                    int32_t max_seq_len, void *out, float *lse, void *workspace,
+                    size_t workspace_size, void *stream) {
+    Layout L;
+    int rc = check_params(params, &L);
+    if (rc) return rc;
+    if ((rc = check_cache(cache, L))) return rc;
+    if (max_seq_len < 0 || max_seq_len > kMaxPos)
+        return fail(DUO_ERR_INVALID_ARG, "max_seq_len must be in [0, 2^30]");
+    if (L.n_full > 0 && max_seq_len > cache->capacity)
+        return fail(DUO_ERR_INVALID_ARG, "max_seq_len %d exceeds capacity %lld", max_seq_len,
+                    (long long)cache->capacity);
+    if (!q || !out) return fail(DUO_ERR_INVALID_ARG, "q / out is NULL");
+    if (!aligned16(q) || !aligned16(out) || (lse && !aligned16(lse)))
+        return fail(DUO_ERR_INVALID_ARG, "q / out / lse must be 16-byte aligned");
+    int sms = 148;
+    if ((rc = check_device(&sms))) return rc;
+    const DecodePlan d = plan_decode(params, L, max_seq_len, sms);
+    const size_t need = workspace_bytes(params, d);
+    if (!workspace || workspace_size < need || ((uintptr_t)workspace & 255u))
+        return fail(DUO_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
+                    workspace_size);
+    duo::DecodeArgs a{};
+    a.full_k = (const __nv_bfloat16 *)cache->full_k;
+    a.full_v = (const __nv_bfloat16 *)cache->full_v;
+    a.strm_k = (const __nv_bfloat16 *)cache->strm_k;
+    a.strm_v = (const __nv_bfloat16 *)cache->strm_v;
+    a.seq_len = cache->seq_len;
+    a.ring_head = cache->ring_head;
+    a.q = (const __nv_bfloat16 *)q;
+    a.sink_logit = params->sink_logit;
+    a.part = (float *)workspace;
+    a.out = (__nv_bfloat16 *)out;
+    a.lse = lse;
+    a.capacity = L.n_full > 0 ? cache->capacity : 0;
+    a.batch = params->batch;
+    a.hkv = params->num_kv_heads;
+    a.n_full = L.n_full;
+    a.n_ring = L.n_ring;
+    a.sink = L.sink;
+    a.ring = L.ring;
+    a.slots = L.slots;
+    a.chunk_full = d.chunk_full;
+    a.splits_full = d.splits_full;
+    a.chunk_ring = d.chunk_ring;
+    a.splits_ring = d.splits_ring;
+    a.max_splits = d.max_splits;
+    a.scale_log2 = params->softmax_scale * duo::kLog2eF;
+    memcpy(a.full_head, L.full_head, sizeof a.full_head);
+    memcpy(a.ring_head_of, L.ring_head_of, sizeof a.ring_head_of);
+    a.heads = L.heads;
+    cudaStream_t st = (cudaStream_t)stream;
+    static bool smem_set[64] = {};
+    if ((rc = set_smem_once(duo::decode_split, duo::kDecSmem, "decode_split", smem_set))) return rc;
+    if (d.items > 0) {
+        duo::decode_split<<<(unsigned)d.items, duo::kDecThreads, duo::kDecSmem, st>>>(a);
+        if ((rc = launch_status("decode_split"))) return rc;
+    }
+    duo::decode_merge<<<(unsigned)((int64_t)params->batch * params->num_q_heads), duo::kD, 0, st>>>(a);
+    return launch_status("decode_merge");
+}
+
+int duo_attn_prefill(const duo_params *params, const void *q, const void *k, const void *v,
+                     int32_t seq_len, void *out, float *lse, void *stream) {
+    Layout L;
+    int rc = check_params(params, &L);
+    if (rc) return rc;
+    if (seq_len < 0 || seq_len > kMaxPos) return fail(DUO_ERR_INVALID_ARG, "seq_len must be in [0, 2^30]");
+    if (seq_len == 0) return DUO_OK;
+    if (!q || !k || !v || !out) return fail(DUO_ERR_INVALID_ARG, "q / k / v / out is NULL");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned16(lse)))
+        return fail(DUO_ERR_INVALID_ARG, "q / k / v / out / lse must be 16-byte aligned");
+    if ((rc = check_device(nullptr))) return rc;
+    return duo::launch_prefill(params, L.sliding, L.heads.is_full, L.sink, L.ring, q, k, v, seq_len,
+                               out, lse, (cudaStream_t)stream, g_err, sizeof g_err);
+}
+
+int duo_get_device_status(void *stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+        return fail(DUO_ERR_CUDA, "stream synchronize failed: %s", cudaGetErrorString(cudaGetLastError()));
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, duo::g_status, sizeof v) != cudaSuccess)
+        return fail(DUO_ERR_CUDA, "reading the status word failed");
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(duo::g_status, &zero, sizeof zero) != cudaSuccess)
+        return fail(DUO_ERR_CUDA, "clearing the status word failed");
+    return v;
+}
+
+}  // extern "C"

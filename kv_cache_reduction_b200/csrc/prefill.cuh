@@ -1,0 +1,424 @@
+// prefill.cuh -- causal / banded FlashAttention-style prefill on tcgen05.
+//
+// What each query row attends to (DuoAttention Laguna Adapter card, Summary
+// and Why It Works; Laguna sliding-window articles): a full-context KV head
+// every key j <= i; a streaming head the sink j < sink plus the recent keys
+// i - recent < j <= i; a sliding-window layer the keys i - window < j <= i.
+// An optional per-query-head sink logit (Laguna XS 2.1 article, attention
+// sinks) joins the softmax denominator with a zero value vector.
+//
+// One CTA computes a 128-row query tile for two query heads of the same GQA
+// group, so both heads share every K/V tile in shared memory:
+//   warp 0     TMA producer: Q of both heads once, then K and V tiles into
+//              a two-stage ring (128-byte swizzled, no multicast)
+//   warp 1     TMEM allocator and MMA issuer (one thread):
+//              S_h = Q_h K^T  (tcgen05.mma, both operands in shared memory)
+//              O_h += P_h V   (tcgen05.mma, P_h read from tensor memory)
+//   warps 4-7  softmax of head 0, warps 8-11 softmax of head 1: thread r
+//              owns query row r, reads S from TMEM, writes P (bf16) back
+//              over S, rescales O in TMEM only when the running max grew by
+//              more than 2^8, and writes O / l and the log-sum-exp at the end.
+// TMEM: S0 | S1 | O0 | O1, 128 fp32 columns each (512 in total).  Key tiles
+// that no row of the query tile attends to are never loaded.
+#pragma once
+
+#include <cuda.h>
+
+#include "ptx.cuh"
+
+namespace duo {
+
+constexpr int kPfM = 128;                  // query rows per tile
+constexpr int kPfN = 128;                  // keys per tile
+constexpr int kPfThreads = 384;            // 12 warps
+constexpr int kPfStages = 2;
+constexpr uint32_t kTileBytes = kPfM * 128 * 2;      // 128 rows x 128 bf16 = 32 KB
+constexpr uint32_t kHalfTileBytes = kTileBytes / 2;  // one 64-column swizzled box
+constexpr size_t kPfSmem = 2 * kTileBytes + 2 * kPfStages * kTileBytes + 1024;
+
+enum : int { kKindFull = 0, kKindStreaming = 1, kKindSliding = 2 };
+
+struct PrefillArgs {
+    CUtensorMap tm_q;      // [B][L][Hq][128] bf16, box 64 x 1 x 128 x 1
+    CUtensorMap tm_k;      // [B][L][Hkv][128]
+    CUtensorMap tm_v;
+    __nv_bfloat16 *out;    // [B][L][Hq][128]
+    float *lse;            // [B][Hq][L] or null
+    const float *sink_logit;
+    int32_t L, hq, hkv, n_qtiles;
+    int32_t sink, recent, window;
+    float scale_log2;
+    int8_t kind[64];       // per KV head
+};
+
+// Key tiles of query tile t for one head kind: an optional run of sink
+// tiles [0, n_sink_tiles) followed by the band [band_lo, t].
+struct TileList {
+    int n_sink_tiles, band_lo, t;
+    __device__ int count() const { return n_sink_tiles + (t - band_lo + 1); }
+    __device__ int at(int j) const { return j < n_sink_tiles ? j : band_lo + (j - n_sink_tiles); }
+};
+
+__device__ __forceinline__ TileList tile_list(int kind, int t, int sink, int recent, int window) {
+    TileList tl{0, 0, t};
+    if (kind == kKindFull) return tl;
+    const int span = kind == kKindStreaming ? recent : window;
+    const int first = t * kPfM - span + 1;           // lowest key of the band (row t*128)
+    tl.band_lo = first <= 0 ? 0 : first / kPfN;
+    if (kind == kKindStreaming && sink > 0) {
+        const int st = (sink + kPfN - 1) / kPfN;
+        if (st < tl.band_lo) tl.n_sink_tiles = st;
+        else tl.band_lo = 0;                           // sink and band tiles merge
+    }
+    return tl;
+}
+
+__device__ __forceinline__ bool key_attended(int kind, int i, int j, int sink, int recent, int window) {
+    if (j > i) return false;
+    if (kind == kKindFull) return true;
+    if (kind == kKindStreaming) return j < sink || j > i - recent;
+    return j > i - window;
+}
+
+// True when every (row, key) pair of the tile is attended.
+__device__ __forceinline__ bool tile_dense(int kind, int r0, int c0, int sink, int recent, int window) {
+    const int r1 = r0 + kPfM - 1, c1 = c0 + kPfN - 1;
+    if (c1 > r0) return false;                         // crosses the diagonal
+    if (kind == kKindFull) return true;
+    if (kind == kKindStreaming) return c1 < sink || c0 > r1 - recent;
+    return c0 > r1 - window;
+}
+
+__global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_constant__ PrefillArgs a) {
+    extern __shared__ __align__(1024) char psmem_raw[];
+    char *smem = (char *)(((uintptr_t)psmem_raw + 1023) & ~(uintptr_t)1023);
+    char *sQ = smem;                                   // [2 heads][32 KB]
+    char *sK = smem + 2 * kTileBytes;                  // [stages][32 KB]
+    char *sV = sK + kPfStages * kTileBytes;            // [stages][32 KB]
+    __shared__ uint64_t q_full, k_full[kPfStages], v_full[kPfStages], kv_empty[kPfStages];
+    __shared__ uint64_t s_full[2], p_full[2], o_done[2];
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // work tile: x = (b, g, head pair), y = query tile, heaviest tiles first
+    const int pairs = a.hq / 2;
+    const int bgp = blockIdx.x;
+    const int b = bgp / pairs;
+    const int h0 = (bgp % pairs) * 2;
+    const int g = h0 / (a.hq / a.hkv);
+    const int t = a.n_qtiles - 1 - (int)blockIdx.y;
+    const int kind = a.kind[g];
+    const TileList tl = tile_list(kind, t, a.sink, a.recent, a.window);
+    const int n_kv = tl.count();
+
+    if (threadIdx.x == 0) {
+        mbar_init(&q_full, 1);
+        for (int s = 0; s < kPfStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&s_full[h], 1);
+            mbar_init(&p_full[h], 4);
+            mbar_init(&o_done[h], 1);
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncwarp();      // reconverge before the CTA barrier (bar.sync is warp-aligned)
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&a.tm_q);
+            prefetch_tmap(&a.tm_k);
+            prefetch_tmap(&a.tm_v);
+            mbar_expect_tx(&q_full, 2 * kTileBytes);
+            for (int h = 0; h < 2; ++h)
+                for (int half = 0; half < 2; ++half)
+                    tma_load_4d(sQ + h * kTileBytes + half * kHalfTileBytes, &a.tm_q, half * 64,
+                                h0 + h, t * kPfM, b, &q_full);
+            for (int j = 0; j < n_kv; ++j) {
+                const int st = j % kPfStages;
+                if (j >= kPfStages && !mbar_wait(&kv_empty[st], ((j / kPfStages) - 1) & 1)) {
+                    abort_flag = 1;
+                    break;
+                }
+                const int row = tl.at(j) * kPfN;
+                mbar_expect_tx(&k_full[st], kTileBytes);
+                for (int half = 0; half < 2; ++half)
+                    tma_load_4d(sK + st * kTileBytes + half * kHalfTileBytes, &a.tm_k, half * 64, g,
+                                row, b, &k_full[st]);
+                mbar_expect_tx(&v_full[st], kTileBytes);
+                for (int half = 0; half < 2; ++half)
+                    tma_load_4d(sV + st * kTileBytes + half * kHalfTileBytes, &a.tm_v, half * 64, g,
+                                row, b, &v_full[st]);
+            }
+        }
+        __syncwarp();  // lanes 1..31 wait for the producer lane before the CTA barrier
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_qk = idesc_bf16_f32(kPfM, kPfN, 0, 0);
+            const uint32_t id_pv = idesc_bf16_f32(kPfM, 128, 0, 1);
+            const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+            bool ok = mbar_wait(&q_full, 0);
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int st = j % kPfStages;
+                const uint32_t par = (j / kPfStages) & 1;
+                if (!(ok = mbar_wait(&k_full[st], par))) break;
+                tc_fence_after();
+                for (int h = 0; h < 2 && ok; ++h) {
+                    // S_h aliases P_h: the previous P_h V must be done reading it
+                    if (j > 0 && !(ok = mbar_wait(&o_done[h], (j - 1) & 1))) break;
+                    tc_fence_after();
+                    const uint32_t s_tmem = tmem + h * 128;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = (k >> 2) * kHalfTileBytes + (k & 3) * 32;
+                        mma_ss(s_tmem, smem_desc_sw128(q_addr + h * kTileBytes + off, 16, 1024),
+                               smem_desc_sw128(k_addr + st * kTileBytes + off, 16, 1024), id_qk,
+                               k > 0);
+                    }
+                    mma_commit(&s_full[h]);
+                }
+                if (!ok || !(ok = mbar_wait(&v_full[st], par))) break;
+                for (int h = 0; h < 2 && ok; ++h) {
+                    if (!(ok = mbar_wait(&p_full[h], j & 1))) break;
+                    tc_fence_after();
+                    const uint32_t p_tmem = tmem + h * 128;
+                    const uint32_t o_tmem = tmem + 256 + h * 128;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(o_tmem, p_tmem + k * 8,
+                               smem_desc_sw128(v_addr + st * kTileBytes + k * 2048, kHalfTileBytes, 1024),
+                               id_pv, (j > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(&o_done[h]);
+                }
+                mma_commit(&kv_empty[st]);
+            }
+            if (!ok) abort_flag = 1;
+        }
+        __syncwarp();  // lanes 1..31 wait for the MMA lane before the CTA barrier
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int h = (warp - 4) >> 2;                 // 0 or 1
+        const int quarter = warp & 3;                  // TMEM lane quarter of this warp
+        const int r = quarter * 32 + lane;             // query row within the tile
+        const int i = t * kPfM + r;                    // query position
+        const int hq = h0 + h;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t s_tmem = tmem + h * 128 + lane_base;
+        const uint32_t o_tmem = tmem + 256 + h * 128 + lane_base;
+        const float c = a.scale_log2;
+        // running max (log2 units) and sum; a sink logit starts them at (sigma, 1)
+        float m_run = -INFINITY, l_run = 0.f;
+        if (a.sink_logit != nullptr) {
+            m_run = a.sink_logit[hq] * kLog2eF;
+            l_run = 1.f;
+        }
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            const bool got = mbar_wait(&s_full[h], j & 1);
+            __syncwarp();      // tcgen05.ld below is warp-collective
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[128];
+            tmem_ld32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_ld32(s_tmem + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+            tmem_ld32(s_tmem + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+            tmem_ld_wait();
+            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+            const int c0 = tl.at(j) * kPfN;
+            if (!tile_dense(kind, t * kPfM, c0, a.sink, a.recent, a.window)) {
+#pragma unroll
+                for (int cc = 0; cc < 128; ++cc)
+                    if (!key_attended(kind, i, c0 + cc, a.sink, a.recent, a.window))
+                        sr[cc] = __float_as_uint(-INFINITY);
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int cc = 0; cc < 128; ++cc) mx = fmaxf(mx, __uint_as_float(sr[cc]));
+            const float m_tile = mx * c;               // scale > 0 keeps the order
+            // keep the stale max unless the new one is more than 2^8 larger
+            float m_use = m_run, alpha = 1.f;
+            if (m_tile > m_run + 8.f) {
+                m_use = m_tile;
+                alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_tile);
+            }
+            const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+            float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+            uint32_t pw[64];
+#pragma unroll
+            for (int cc = 0; cc < 128; cc += 4) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
+                const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
+                const float p3 = ex2_approx(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
+                ls0 += p0;
+                ls1 += p1;
+                ls2 += p2;
+                ls3 += p3;
+                pw[cc / 2] = pack_bf16x2(p0, p1);
+                pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
+            }
+            l_run = l_run * alpha + ((ls0 + ls1) + (ls2 + ls3));
+            m_run = m_use;
+            tmem_st32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
+            tmem_st32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
+            // O holds the previous tiles' sum (its PV is complete: this S was
+            // issued after it); rescale it when the max moved
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                for (int cb = 0; cb < 128; cb += 32) {
+                    uint32_t orr[32];
+                    tmem_ld32(o_tmem + cb, orr);
+                    tmem_ld_wait();
+                    reg_fence32(orr);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                    tmem_st32(o_tmem + cb, orr);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[h]);
+        }
+        // ------------------------------------------------------------ epilogue
+        const bool o_ready = ok && n_kv > 0 && mbar_wait(&o_done[h], (n_kv - 1) & 1);
+        if (__all_sync(0xffffffffu, o_ready)) {
+            tc_fence_after();
+            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            __nv_bfloat16 *orow = a.out + (((size_t)b * a.L + i) * a.hq + hq) * 128;
+#pragma unroll
+            for (int cb = 0; cb < 128; cb += 32) {
+                uint32_t orr[32];
+                tmem_ld32(o_tmem + cb, orr);
+                tmem_ld_wait();
+                reg_fence32(orr);
+                if (i < a.L) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + cb);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(orr[e]) * inv_l, __uint_as_float(orr[e + 1]) * inv_l);
+                        v.y = pack_bf16x2(__uint_as_float(orr[e + 2]) * inv_l, __uint_as_float(orr[e + 3]) * inv_l);
+                        v.z = pack_bf16x2(__uint_as_float(orr[e + 4]) * inv_l, __uint_as_float(orr[e + 5]) * inv_l);
+                        v.w = pack_bf16x2(__uint_as_float(orr[e + 6]) * inv_l, __uint_as_float(orr[e + 7]) * inv_l);
+                        dst[e / 8] = v;
+                    }
+                }
+            }
+            if (a.lse != nullptr && i < a.L)
+                a.lse[((size_t)b * a.hq + hq) * a.L + i] =
+                    l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2F : -INFINITY;
+        } else if (!ok) {
+            abort_flag = 1;
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// [B][L][H][128] bf16 viewed as a 4-D tensor (128, H, L, B), loaded as
+// 64-column x 128-row boxes with the 128-byte swizzle.
+inline bool make_tmap(CUtensorMap *m, const void *base, int B, int L, int H) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {256, (cuuint64_t)H * 256, (cuuint64_t)L * H * 256};
+    const cuuint32_t box[4] = {64, 1, kPfM, 1};
+    const cuuint32_t elem[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+              elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_full, int sink,
+                          int ring, const void *q, const void *k, const void *v, int32_t L, void *out,
+                          float *lse, cudaStream_t stream, char *err, size_t err_len) {
+    PrefillArgs a;
+    memset(&a, 0, sizeof a);
+    const int B = p->batch;
+    if (!make_tmap(&a.tm_q, q, B, L, p->num_q_heads) || !make_tmap(&a.tm_k, k, B, L, p->num_kv_heads) ||
+        !make_tmap(&a.tm_v, v, B, L, p->num_kv_heads)) {
+        snprintf(err, err_len, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
+        return DUO_ERR_CUDA;
+    }
+    a.out = (__nv_bfloat16 *)out;
+    a.lse = lse;
+    a.sink_logit = p->sink_logit;
+    a.L = L;
+    a.hq = p->num_q_heads;
+    a.hkv = p->num_kv_heads;
+    a.n_qtiles = (L + kPfM - 1) / kPfM;
+    a.sink = sliding ? 0 : sink;
+    a.recent = sliding ? 0 : ring;
+    a.window = sliding ? ring : 0;
+    a.scale_log2 = p->softmax_scale * kLog2eF;
+    for (int g = 0; g < p->num_kv_heads; ++g)
+        a.kind[g] = sliding ? kKindSliding : (is_full[g] ? kKindFull : kKindStreaming);
+    static bool smem_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !smem_set[dev]) {
+        if (cudaFuncSetAttribute(prefill_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kPfSmem) != cudaSuccess) {
+            snprintf(err, err_len, "cudaFuncSetAttribute(prefill_fwd) failed");
+            return DUO_ERR_CUDA;
+        }
+        if (dev >= 0 && dev < 64) smem_set[dev] = true;
+    }
+    if (a.n_qtiles > 65535) {
+        snprintf(err, err_len, "sequence too long for one prefill launch");
+        return DUO_ERR_INVALID_ARG;
+    }
+    const dim3 grid((unsigned)(B * (p->num_q_heads / 2)), (unsigned)a.n_qtiles);
+    prefill_fwd<<<grid, kPfThreads, kPfSmem, stream>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        snprintf(err, err_len, "prefill_fwd launch: %s", cudaGetErrorString(e));
+        return DUO_ERR_CUDA;
+    }
+    return DUO_OK;
+}
+
+}  // namespace duo

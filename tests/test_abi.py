@@ -1,0 +1,154 @@
+"""The C ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before touching a device (CPU only, no kernel runs)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import kv_cache_reduction_b200 as duo
+from kv_cache_reduction_b200 import build as duo_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    duo_build.build()
+    return duo.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        names += re.findall(r"DUO_API\s+[\w\s\*]+?\b(duo_\w+)\s*\(", text)
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("duo_kv_append", "duo_attn_prefill", "duo_attn_decode", "duo_decode_workspace_bytes",
+              "duo_get_device_status", "duo_status_string", "duo_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(duo.EXPORTED) <= set(declared_functions())
+
+
+def test_library_exports_nothing_else(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", duo.LIBRARY_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    ours = {n for n in exported if n.startswith("duo_")}
+    assert ours == set(declared_functions())
+
+
+def test_library_has_no_gpu_driver_dependency(lib):
+    out = subprocess.run(["ldd", duo.LIBRARY_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libtorch" not in out
+
+
+def test_status_strings(lib):
+    for code in range(0, -8, -1):
+        assert duo.duo_status_string(code) not in ("", "unknown status")
+    assert duo.duo_status_string(-99) == "unknown status"
+
+
+def _params(**kw):
+    base = dict(batch=2, full_mask=(1, 0, 0, 1, 0, 0, 0, 0))
+    base.update(kw)
+    return duo.DuoParams(**base)
+
+
+def _call_append(p, cache=None):
+    lib = duo.load_library()
+    pc = p.as_c()
+    c = cache or duo._Cache(0x1000, 0x1000, 64, 0x1000, 0x1000, 0x1000, 0x1000)
+    return lib.duo_kv_append(ctypes.byref(pc), ctypes.byref(c), 0x1000, 0x1000, 1, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=64), duo.DUO_ERR_UNSUPPORTED),
+    (dict(num_q_heads=40), duo.DUO_ERR_UNSUPPORTED),
+    (dict(num_kv_heads=65, num_q_heads=390), duo.DUO_ERR_UNSUPPORTED),
+    (dict(batch=0), duo.DUO_ERR_INVALID_ARG),
+    (dict(softmax_scale=0.0), duo.DUO_ERR_INVALID_ARG),
+    (dict(softmax_scale=float("inf")), duo.DUO_ERR_INVALID_ARG),
+    (dict(recent=0), duo.DUO_ERR_INVALID_ARG),
+    (dict(sink=-1), duo.DUO_ERR_INVALID_ARG),
+    (dict(sink=8000, recent=500), duo.DUO_ERR_INVALID_ARG),
+    (dict(window=-3), duo.DUO_ERR_INVALID_ARG),
+    (dict(window=9000), duo.DUO_ERR_INVALID_ARG),
+    (dict(full_mask=(2, 0, 0, 0, 0, 0, 0, 0)), duo.DUO_ERR_INVALID_ARG),
+])
+def test_bad_params_are_rejected_before_any_launch(lib, kw, code):
+    assert _call_append(_params(**kw)) == code
+    assert duo.duo_last_error() != ""
+
+
+def test_bad_pointers_are_rejected(lib):
+    p = _params()
+    pc = p.as_c()
+    ok = dict(full_k=0x1000, full_v=0x1000, capacity=64, strm_k=0x1000, strm_v=0x1000,
+              seq_len=0x1000, ring_head=0x1000)
+    for key, bad in [("full_k", 0), ("strm_v", 0), ("seq_len", 0), ("full_k", 0x1008),
+                     ("capacity", 0), ("ring_head", 0x1002)]:
+        c = duo._Cache(**{**ok, key: bad})
+        assert lib.duo_kv_append(ctypes.byref(pc), ctypes.byref(c), 0x1000, 0x1000, 1, None) == \
+            duo.DUO_ERR_INVALID_ARG, key
+    c = duo._Cache(**ok)
+    assert lib.duo_kv_append(ctypes.byref(pc), ctypes.byref(c), 0, 0x1000, 1, None) == duo.DUO_ERR_INVALID_ARG
+    assert lib.duo_kv_append(ctypes.byref(pc), ctypes.byref(c), 0x1004, 0x1000, 1, None) == duo.DUO_ERR_INVALID_ARG
+    assert lib.duo_kv_append(ctypes.byref(pc), ctypes.byref(c), 0x1000, 0x1000, -1, None) == duo.DUO_ERR_INVALID_ARG
+    # n_new == 0 is a no-op that touches nothing
+    assert lib.duo_kv_append(ctypes.byref(pc), ctypes.byref(c), 0, 0, 0, None) == duo.DUO_OK
+    # a null params pointer
+    assert lib.duo_kv_append(None, ctypes.byref(c), 0x1000, 0x1000, 1, None) == duo.DUO_ERR_INVALID_ARG
+
+
+def test_sliding_layer_needs_no_mask_or_full_cache(lib):
+    p = duo.DuoParams(batch=1, window=512, full_mask=())
+    pc = p.as_c()
+    pc.full_mask = None
+    c = duo._Cache(None, None, 0, 0x1000, 0x1000, 0x1000, 0x1000)
+    rc = lib.duo_kv_append(ctypes.byref(pc), ctypes.byref(c), 0x1000, 0x1000, 1, None)
+    # passes every host check; without a GPU the device check then fails
+    assert rc in (duo.DUO_ERR_CUDA, duo.DUO_ERR_DEVICE, duo.DUO_OK)
+    assert rc != duo.DUO_ERR_INVALID_ARG
+
+
+def test_decode_argument_checks(lib):
+    p = _params()
+    pc = p.as_c()
+    c = duo._Cache(0x1000, 0x1000, 64, 0x1000, 0x1000, 0x1000, 0x1000)
+    call = lambda msl, q=0x1000, out=0x1000, ws=0x1000, wsb=1 << 30: lib.duo_attn_decode(
+        ctypes.byref(pc), ctypes.byref(c), q, msl, out, None, ws, wsb, None)
+    assert call(65) == duo.DUO_ERR_INVALID_ARG      # longer than the capacity
+    assert call(-1) == duo.DUO_ERR_INVALID_ARG
+    assert call(10, q=0) == duo.DUO_ERR_INVALID_ARG
+    assert call(10, out=0x1001) == duo.DUO_ERR_INVALID_ARG
+
+
+def test_prefill_argument_checks(lib):
+    p = _params()
+    pc = p.as_c()
+    f = lib.duo_attn_prefill
+    assert f(ctypes.byref(pc), 0x1000, 0x1000, 0x1000, -5, 0x1000, None, None) == duo.DUO_ERR_INVALID_ARG
+    assert f(ctypes.byref(pc), 0x1000, 0, 0x1000, 16, 0x1000, None, None) == duo.DUO_ERR_INVALID_ARG
+    assert f(ctypes.byref(pc), 0x1000, 0x1000, 0x1000, 16, 0x1000, 0x1004, None) == duo.DUO_ERR_INVALID_ARG
+    assert f(ctypes.byref(pc), 0, 0, 0, 0, 0, None, None) == duo.DUO_OK   # empty prefill
+
+
+def test_workspace_size_is_host_arithmetic(lib):
+    p = _params(batch=32)
+    n = duo.duo_decode_workspace_bytes(p, 32768)
+    assert n > 0 and n % 4 == 0
+    assert duo.duo_decode_workspace_bytes(p, 64) <= n
+    assert duo.duo_decode_workspace_bytes(_params(head_dim=64), 128) == 0
