@@ -24,7 +24,6 @@ import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 import numpy as np
@@ -71,11 +70,23 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time: every rank contributes its own elapsed time."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling)."""
+    return base + 7919 * rank
+
+
+def aggregate(units_per_rank: float, world: int, seconds_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / seconds_max
 
 
 # ------------------------------------------------------------------ clocks
@@ -148,7 +159,7 @@ class DecodeB32:
         B, n = w.batch, w.seq_len
         self.params = duo.DuoParams(B, 48, 8, 128, inputs.SINK, inputs.RECENT, 0, 128 ** -0.5,
                                     w.full_mask, None)
-        seed = w.seed + 7919 * rank
+        seed = rank_seed(w.seed, rank)
         self.cache = duo.DuoCache.allocate(self.params, n)
         for i, t in enumerate((self.cache.full_k, self.cache.full_v, self.cache.strm_k,
                                self.cache.strm_v)):
@@ -167,6 +178,7 @@ class DecodeB32:
         self.bytes = rows * 2 * 128 * 2 + 2 * self.q.numel() * 2
         self.launches_per_step = 2
         self.unit = "GB/s"
+        self.kernel = "decode_split + decode_merge (one duo_attn_decode call)"
 
     def step(self):
         duo.duo_attn_decode(self.params, self.cache, self.q, self.w.seq_len, self.out, self.lse,
@@ -224,7 +236,174 @@ class DecodeB32:
                           f"(6 query heads each), float64, {t_total:.1f} s"}
 
 
-WORKLOADS = {"decode_b32": DecodeB32}
+def attended_pairs(L: int, span):
+    """Number of (query, key) pairs a head attends over an L-token prefill:
+    L(L+1)/2 for a full head, sum_i min(i+1, span) for a band of `span` keys."""
+    if span is None:
+        return L * (L + 1) // 2
+    m = min(L, span)
+    return m * (m + 1) // 2 + (L - m) * span
+
+
+class Stack40:
+    """One decode step through the 40-layer stack: B=16 sequences at context
+    131072; layers 3, 7, ..., 39 are DuoAttention layers (2 of 8 heads full),
+    the other 30 sliding-window layers (window 512) with sink logits.  The 40
+    decode calls are captured once in a CUDA graph and replayed per step."""
+
+    def __init__(self, rank: int):
+        w = self.w = inputs.workload("stack40")
+        B, n = w.batch, w.seq_len
+        masks = inputs.stack_layer_masks(w)
+        seed = rank_seed(w.seed, rank)
+        rng = np.random.default_rng(seed)
+        self.layers = []
+        self.bytes = 0
+        max_ws = 0
+        for li, mask in enumerate(masks):
+            if mask is None:
+                sig = inputs.randn_f32((48,), seed * 100 + li, "cuda")
+                p = duo.DuoParams(B, 48, 8, 128, 0, 0, inputs.WINDOW, 128 ** -0.5, (0,) * 8, sig)
+                span = inputs.WINDOW
+            else:
+                p = duo.DuoParams(B, 48, 8, 128, inputs.SINK, inputs.RECENT, 0, 128 ** -0.5, mask, None)
+                span = inputs.SINK + inputs.RECENT
+            cache = duo.DuoCache.allocate(p, n)
+            for i, t in enumerate((cache.full_k, cache.full_v, cache.strm_k, cache.strm_v)):
+                if t is not None:
+                    inputs.randn_bf16_into(t, (seed * 100 + li) * 10 + i)
+            cache.seq_len.fill_(n)
+            cache.ring_head.copy_(torch.as_tensor(rng.integers(0, p.ring_slots - p.sink if mask is None
+                                                               else inputs.RECENT, size=B),
+                                                  dtype=torch.int32))
+            q = inputs.randn_bf16((B, 48, 128), seed * 100 + li + 50, "cuda")
+            out = torch.empty((B, 48, 128), dtype=torch.bfloat16, device="cuda")
+            lse = torch.empty((B, 48), dtype=torch.float32, device="cuda")
+            self.layers.append((p, cache, q, out, lse))
+            rows = B * (p.n_full * n + p.n_ring * min(n, span))
+            self.bytes += rows * 512 + 2 * q.numel() * 2
+            max_ws = max(max_ws, duo.duo_decode_workspace_bytes(p, n))
+        self.ws = torch.empty((max_ws + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+        self.launches_per_step = 2 * len(self.layers)
+        self.unit = "GB/s"
+        self.kernel = "40 x (decode_split + decode_merge), one CUDA graph"
+        self.graph = None
+
+    def eager_step(self, qs=None):
+        for i, (p, cache, q, out, lse) in enumerate(self.layers):
+            duo.duo_attn_decode(p, cache, q if qs is None else qs[i], self.w.seq_len, out, lse, self.ws)
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.eager_step()          # warms up attribute setting outside capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.eager_step()
+        torch.cuda.synchronize()
+
+    def step(self):
+        if self.graph is None:
+            self.capture()
+        self.graph.replay()
+
+    def e2e_buffers(self):
+        self.h_q = [l[2].cpu().pin_memory() for l in self.layers]
+        self.h_out = [torch.empty(l[3].shape, dtype=l[3].dtype).pin_memory() for l in self.layers]
+        self.h_lse = [torch.empty(l[4].shape, dtype=l[4].dtype).pin_memory() for l in self.layers]
+        self.d_q = [torch.empty_like(l[2]) for l in self.layers]
+        h2d = sum(t.numel() * 2 for t in self.h_q)
+        d2h = sum(t.numel() * 2 for t in self.h_out) + sum(t.numel() * 4 for t in self.h_lse)
+        return h2d, d2h
+
+    def e2e_step(self):
+        for i in range(len(self.layers)):
+            self.d_q[i].copy_(self.h_q[i], non_blocking=True)
+        self.eager_step(self.d_q)
+        for i, l in enumerate(self.layers):
+            self.h_out[i].copy_(l[3], non_blocking=True)
+            self.h_lse[i].copy_(l[4], non_blocking=True)
+
+    def config(self):
+        return {"workload": "stack40: one decode step through 40 layers (10 DuoAttention layers "
+                            "3,7,...,39 with 2 of 8 heads full, 30 sliding-window layers of 512 "
+                            "with sink logits), B=16, context 131072, CUDA graph",
+                "batch_per_gpu": self.w.batch, "context": self.w.seq_len, "layers": 40,
+                "l2": "inputs larger than L2 (22.6 GB of cache per step)"}
+
+    def oracle_sample(self, budget_s: float = 15.0):
+        import oracle
+        done_bytes, t_total, used = 0, 0.0, 0
+        for li in (3, 0):                      # one DuoAttention layer, one sliding layer
+            p, cache, q, _, _ = self.layers[li]
+            ol = oracle.Layer(1, 48, 8, 128, p.sink, p.recent, p.window, p.softmax_scale,
+                              tuple(p.full_mask),
+                              None if p.sink_logit is None else p.sink_logit.cpu().numpy())
+            for b in range(2):
+                hc = oracle.Cache(ol, cache.capacity if p.n_full else 1)
+                if p.n_full:
+                    hc.full_k = inputs.bits(cache.full_k[b:b + 1])
+                    hc.full_v = inputs.bits(cache.full_v[b:b + 1])
+                hc.strm_k = inputs.bits(cache.strm_k[b:b + 1])
+                hc.strm_v = inputs.bits(cache.strm_v[b:b + 1])
+                hc.seq_len = cache.seq_len[b:b + 1].cpu().numpy().astype(np.int32)
+                hc.ring_head = cache.ring_head[b:b + 1].cpu().numpy().astype(np.int32)
+                t0 = time.perf_counter()
+                oracle.attn_decode(ol, hc, inputs.bits(q[b:b + 1]))
+                t_total += time.perf_counter() - t0
+                n = self.w.seq_len
+                span = p.window if p.window else p.sink + p.recent
+                done_bytes += (p.n_full * n + p.n_ring * min(n, span)) * 512 + 2 * 48 * 256
+                used += 1
+                if t_total >= budget_s:
+                    break
+        return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+                "kind": "oracle",
+                "sample": f"{used} (layer, sequence) slices of one step (layers 3 and 0), "
+                          f"float64, {t_total:.1f} s"}
+
+
+class Prefill:
+    """Prefill of one layer: prefill_16k (B=1, L=16384, 2 of 8 heads full) or
+    sliding_32k (B=2, L=32768, window 512, sink logits, RMSNorm'd Q/K)."""
+
+    def __init__(self, rank: int, name: str):
+        w = self.w = inputs.workload(name)
+        B, L = w.batch, w.seq_len
+        seed = rank_seed(w.seed, rank)
+        sig = inputs.randn_f32((48,), seed + 9, "cuda") if w.sink_logit else None
+        self.params = duo.DuoParams(B, 48, 8, 128, inputs.SINK, inputs.RECENT, w.window,
+                                    128 ** -0.5, w.full_mask, sig)
+        self.q = inputs.randn_bf16((B, L, 48, 128), seed, "cuda")
+        self.k = inputs.randn_bf16((B, L, 8, 128), seed + 1, "cuda")
+        self.v = inputs.randn_bf16((B, L, 8, 128), seed + 2, "cuda")
+        if w.rmsnorm:
+            self.q, self.k = inputs.rmsnorm_bf16(self.q), inputs.rmsnorm_bf16(self.k)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty((B, 48, L), dtype=torch.float32, device="cuda")
+        pairs = 0
+        for g in range(8):
+            span = w.window if w.window else (None if w.full_mask[g] else inputs.SINK + inputs.RECENT)
+            pairs += 6 * attended_pairs(L, span)
+        self.flops = 4 * 128 * pairs * B
+        self.launches_per_step = 1
+        self.unit = "TFLOP/s"
+        self.kernel = "prefill_fwd"
+
+    def step(self):
+        duo.duo_attn_prefill(self.params, self.q, self.k, self.v, self.out, self.lse)
+
+    def config(self):
+        return {"workload": f"{self.w.name}: prefill B={self.w.batch}, L={self.w.seq_len}",
+                "window": self.w.window, "full_mask": list(self.w.full_mask)}
+
+
+WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40,
+             "prefill_16k": lambda rank: Prefill(rank, "prefill_16k"),
+             "sliding_32k": lambda rank: Prefill(rank, "sliding_32k")}
 
 
 # ------------------------------------------------------------------ timing
@@ -241,46 +420,85 @@ def time_steps(fn, steps, stream, world):
     return start.elapsed_time(stop) / 1e3
 
 
-def run_ours(args, world, rank):
-    wl = WORKLOADS[args.workload](rank)
+def measure(wl, steps, warmup, world):
+    """Warm-up, then `steps` timed steps (CUDA events on the launching stream,
+    barrier + synchronize on both sides); returns (seconds per step of the
+    slowest rank, clock summary)."""
     stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         wl.step()
     torch.cuda.synchronize()
-    if duo.duo_get_device_status() != duo.DUO_OK:
-        raise RuntimeError("device status error during warm-up")
+    status = duo.duo_get_device_status()
+    if status != duo.DUO_OK:
+        raise RuntimeError(f"device status {status} during warm-up")
     with ClockSampler(torch.cuda.current_device()) as clk:
-        t = time_steps(wl.step, args.steps, stream, world)
+        t = time_steps(wl.step, steps, stream, world)
     t = max_over_ranks(t, world)
-    clocks = clk.summary()
-    # end to end: host buffers, copies inside the timed region
-    h2d, d2h = wl.e2e_buffers()
-    for _ in range(max(1, args.warmup)):
-        wl.e2e_step()
-    torch.cuda.synchronize()
-    t_e2e = max_over_ranks(time_steps(wl.e2e_step, args.steps, stream, world), world)
-    if duo.duo_get_device_status() != duo.DUO_OK:
-        raise RuntimeError("device status error during timing")
+    status = duo.duo_get_device_status()
+    if status != duo.DUO_OK:
+        raise RuntimeError(f"device status {status} during timing")
+    return t / steps, clk.summary()
+
+
+def roofline(wl, per_step, pk, pk_kind):
+    if wl.unit == "GB/s":
+        achieved = wl.bytes / per_step / 1e9
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)"}
+    achieved = wl.flops / per_step / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": None,
+            "peak_source": f"{pk_kind} bf16_tflops (burst cuBLAS GEMM)"}
+
+
+def units(wl):
+    return wl.bytes / 1e9 if wl.unit == "GB/s" else wl.flops / 1e12
+
+
+def run_ours(args, world, rank):
     pk, pk_kind = peaks()
-    per_step = t / args.steps
-    value = wl.bytes * world / per_step / 1e9
-    achieved = wl.bytes / per_step / 1e9
+    wl = WORKLOADS[args.workload](rank)
+    per_step, clocks = measure(wl, args.steps, args.warmup, world)
+    value = aggregate(units(wl), world, per_step)
+    rf = roofline(wl, per_step, pk, pk_kind)
+    rf["kernel"] = wl.kernel
     res = {"metric": METRIC, "value": round(value, 2), "unit": wl.unit, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 4),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-           "data": "synthetic (seeded N(0,1) bf16 caches and queries)",
-           "config": {**wl.config(), "parallelism": f"dp{world} (independent batches)"},
-           "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
-                        "peak": pk["hbm_gbs"], "unit": "GB/s",
-                        "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
-                        "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)",
-                        "kernel": "decode_split + decode_merge (one duo_attn_decode call)"},
-           "e2e": {"value": round(wl.bytes * world / (t_e2e / args.steps) / 1e9, 2),
-                   "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-           "gpu_launches": wl.launches_per_step * args.steps,
-           "clocks": clocks}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+           "data": "synthetic (seeded N(0,1) bf16 inputs and caches)",
+           "config": {**wl.config(), "parallelism": f"dp{world} (independent batches, no collective)"},
+           "roofline": rf, "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks}
+    # end to end through the public API: pinned host inputs, copies in the timed region
+    if hasattr(wl, "e2e_step"):
+        h2d, d2h = wl.e2e_buffers()
+        for _ in range(args.warmup):
+            wl.e2e_step()
+        torch.cuda.synchronize()
+        t_e2e = max_over_ranks(time_steps(wl.e2e_step, args.steps, torch.cuda.current_stream(), world),
+                               world) / args.steps
+        res["e2e"] = {"value": round(aggregate(units(wl), world, t_e2e), 2), "unit": wl.unit,
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "ms_per_step": round(t_e2e * 1e3, 4)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(wl, "oracle_sample"):
         res["cpu_baseline"] = wl.oracle_sample(args.cpu_budget)
+    # the other workloads of the path, on this GPU, as context for the main line
+    if args.secondary and args.workload == "decode_b32":
+        del wl
+        torch.cuda.empty_cache()
+        sec = {}
+        for name in ("stack40", "prefill_16k", "sliding_32k"):
+            w2 = WORKLOADS[name](rank)
+            st = max(3, min(args.steps, 10))
+            ps, ck = measure(w2, st, args.warmup, world)
+            r2 = roofline(w2, ps, pk, pk_kind)
+            sec[name] = {"value": round(aggregate(units(w2), world, ps), 2), "unit": w2.unit,
+                         "ms_per_step": round(ps * 1e3, 4), "steps": st, "frac": r2["frac"],
+                         "bound": r2["bound"], "kernel": w2.kernel,
+                         "gpu_launches": w2.launches_per_step * st, "clocks": ck}
+            del w2
+            torch.cuda.empty_cache()
+        res["secondary"] = sec
     return res
 
 
@@ -318,6 +536,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b32")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--secondary", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time the 40-layer stack and the two prefill workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

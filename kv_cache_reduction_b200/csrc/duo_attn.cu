@@ -6,7 +6,7 @@
 #include <cstdio>
 #include <cstring>
 
-#include "../../include/duo_attn.h"
+#include "duo_attn.h"
 #include "decode.cuh"
 #include "kv_append.cuh"
 #include "prefill.cuh"

@@ -98,7 +98,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     __shared__ uint64_t q_full, k_full[kPfStages], v_full[kPfStages], kv_empty[kPfStages];
     __shared__ uint64_t s_full[2], p_full[2], o_done[2];
     __shared__ uint32_t tmem_base;
-    __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // work tile: x = (b, g, head pair), y = query tile, heaviest tiles first
@@ -124,7 +123,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             mbar_init(&p_full[h], 4);
             mbar_init(&o_done[h], 1);
         }
-        abort_flag = 0;
         fence_mbar_init();
     }
     __syncwarp();      // reconverge before the CTA barrier (bar.sync is warp-aligned)
@@ -150,10 +148,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                                 h0 + h, t * kPfM, b, &q_full);
             for (int j = 0; j < n_kv; ++j) {
                 const int st = j % kPfStages;
-                if (j >= kPfStages && !mbar_wait(&kv_empty[st], ((j / kPfStages) - 1) & 1)) {
-                    abort_flag = 1;
-                    break;
-                }
+                if (j >= kPfStages && !mbar_wait(&kv_empty[st], ((j / kPfStages) - 1) & 1)) break;
                 const int row = tl.at(j) * kPfN;
                 mbar_expect_tx(&k_full[st], kTileBytes);
                 for (int half = 0; half < 2; ++half)
@@ -207,7 +202,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 }
                 mma_commit(&kv_empty[st]);
             }
-            if (!ok) abort_flag = 1;
         }
         __syncwarp();  // lanes 1..31 wait for the MMA lane before the CTA barrier
     } else if (warp >= 4) {
@@ -327,8 +321,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             if (a.lse != nullptr && i < a.L)
                 a.lse[((size_t)b * a.hq + hq) * a.L + i] =
                     l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2F : -INFINITY;
-        } else if (!ok) {
-            abort_flag = 1;
         }
         __syncwarp();
     }
