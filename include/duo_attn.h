@@ -149,6 +149,24 @@ DUO_API int duo_attn_decode(const duo_params *params, const duo_cache *cache, co
                     int32_t max_seq_len, void *out, float *lse, void *workspace,
                     size_t workspace_bytes, void *stream);
 
+/* duo_attn_decode without a caller workspace, for callers that cannot
+ * allocate device memory at call time (an engine plugin that must not
+ * allocate inside its execute hook, a server with a fixed memory budget, a
+ * latency-critical loop that cannot afford cudaMalloc's device-wide
+ * synchronisation).  The pages have no counterpart: this is an interface
+ * convenience, not part of the method.
+ * The split partials live in a 16 MiB array inside the library, reserved on
+ * every GPU that loads it until the process exits; the call allocates
+ * nothing.  The first call on a device looks up that array's address, so make
+ * it before any stream capture begins.  A layer whose
+ * duo_decode_workspace_bytes exceeds 16 MiB returns DUO_ERR_WORKSPACE with
+ * nothing launched.  All calls on a device share the array: calls whose
+ * kernels may overlap on the GPU (different streams or threads) race, so
+ * issue them on one stream.  Arguments, outputs and errors otherwise as
+ * duo_attn_decode. */
+DUO_API int duo_attn_decode_static(const duo_params *params, const duo_cache *cache, const void *q,
+                                   int32_t max_seq_len, void *out, float *lse, void *stream);
+
 /* Reads and clears the device status word of the current device after
  * synchronising `stream`: DUO_OK, DUO_ERR_TIMEOUT or DUO_ERR_CAPACITY (the
  * first error any kernel recorded since the last read), or DUO_ERR_CUDA. */

@@ -36,7 +36,8 @@ DUO_ERR_CAPACITY = -6
 DUO_ERR_DEVICE = -7
 
 EXPORTED = ("duo_kv_append", "duo_attn_prefill", "duo_decode_workspace_bytes", "duo_attn_decode",
-            "duo_get_device_status", "duo_status_string", "duo_last_error")
+            "duo_attn_decode_static", "duo_get_device_status", "duo_status_string",
+            "duo_last_error")
 
 
 class DuoLibraryMissing(RuntimeError):
@@ -85,6 +86,8 @@ def load_library(path: str = LIBRARY_PATH) -> ctypes.CDLL:
     lib.duo_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.duo_attn_decode.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, vp, ctypes.c_size_t, vp]
     lib.duo_attn_decode.restype = ctypes.c_int
+    lib.duo_attn_decode_static.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, vp]
+    lib.duo_attn_decode_static.restype = ctypes.c_int
     lib.duo_get_device_status.argtypes = [vp]
     lib.duo_get_device_status.restype = ctypes.c_int
     lib.duo_status_string.argtypes = [ctypes.c_int]
@@ -213,6 +216,17 @@ def duo_attn_decode(params: DuoParams, cache: DuoCache, q: torch.Tensor, max_seq
     _check(load_library().duo_attn_decode(ctypes.byref(p), ctypes.byref(c), _ptr(q), int(max_seq_len),
                                           _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
                                           _stream(stream)))
+
+
+def duo_attn_decode_static(params: DuoParams, cache: DuoCache, q: torch.Tensor, max_seq_len: int,
+                           out: torch.Tensor, lse: Optional[torch.Tensor], stream=None) -> None:
+    """duo_attn_decode with the library's built-in 16 MiB scratch instead of a
+    caller workspace, for callers that cannot allocate device memory when they
+    decode.  Calls that may overlap on the GPU share that scratch and race."""
+    p, c = params.as_c(), cache.as_c()
+    _check(load_library().duo_attn_decode_static(ctypes.byref(p), ctypes.byref(c), _ptr(q),
+                                                 int(max_seq_len), _ptr(out), _ptr(lse),
+                                                 _stream(stream)))
 
 
 def duo_get_device_status(stream=None) -> int:

@@ -39,7 +39,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    cmd += ["-o", LIB + ".tmp", os.path.join(CSRC, "duo_attn.cu")]
+    cmd += ["-o", LIB + ".tmp"] + sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     subprocess.check_call(cmd)
     os.replace(LIB + ".tmp", LIB)
     return LIB
