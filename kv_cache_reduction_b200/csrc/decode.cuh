@@ -1,4 +1,4 @@
-// decode.cuh -- one-token split-KV decode over the hybrid cache.
+// decode.cuh -- one-token split-KV decode over the hybrid cache, on tcgen05.
 //
 // DuoAttention Laguna Adapter card (Summary, Why It Works): a full-context
 // KV head attends over every cached token, a streaming head over its sink
@@ -7,14 +7,27 @@
 // optional per-query-head sink logit (Laguna XS 2.1 article, attention-sink
 // item).  The six query heads of a GQA group share every K/V row read.
 //
-// Work items are (sequence, KV head, split).  A CTA streams its split's K
-// and V rows from HBM into shared memory with bulk async copies (a
-// dedicated producer warp, STAGES-deep mbarrier ring), and eight compute
-// warps run the dot products and the online softmax in fp32 registers.
-// Its partial result (running max, sum, unnormalised output, in log2
-// units) goes to the workspace; decode_merge folds the splits and the sink
-// logit into the final output and log-sum-exp.
+// Work items are (sequence, KV head, split).  One persistent CTA per SM
+// walks its share of the items (a balanced static split):
+//   warps 0-3  softmax and epilogue; thread r owns token r of a 128-token tile
+//              (and dimension r of the output)
+//   warp 4     producer: TMA loads of 128-token K and V tiles (2-D tensor
+//              maps, 64-column boxes, 128-byte swizzle, no multicast) into a
+//              three-stage ring
+//   warp 5     TMEM owner and MMA issuer, "swap AB" so that tokens fill M:
+//                S^T[128 tok x 16] = K_tile[128 x 128] . Q^T   (Q: 6 heads + zero rows)
+//                O^T[128 d  x 16] += V_tile^T . P^T            (P^T written by the softmax)
+//              QK of tile t+1 is issued before PV of tile t.
+// Ring heads load their whole slot array in slot order and mask the slots
+// that hold no valid token (attention does not depend on key order, keys are
+// stored after RoPE).  Rows of V that belong to invalid tokens are zeroed in
+// shared memory before the PV product, so stale cache memory never reaches
+// it.  Each item leaves (m, l, acc) in log2 units in the workspace;
+// decode_merge folds the splits and the sink logit.  Every reduction has a
+// fixed order, so the result is bitwise reproducible.
 #pragma once
+
+#include <cuda.h>
 
 #include "kv_append.cuh"
 #include "ptx.cuh"
@@ -22,19 +35,22 @@
 namespace duo {
 
 constexpr int kD = 128;
-constexpr int kGroup = 6;                 // query heads per KV head
-constexpr int kHalf = kGroup / 2;         // heads per compute group
-constexpr int kDecTile = 64;              // tokens per pipeline stage
-constexpr int kDecStages = 4;
-constexpr int kDecComputeWarps = 8;
-constexpr int kDecThreads = (kDecComputeWarps + 1) * 32;
-constexpr int kRowBytes = kD * 2;         // one token of one head, bf16
-constexpr int kStageBytes = kDecTile * kRowBytes * 2;   // K + V
-constexpr int kPartFloats = kGroup * (kD + 2);          // m[6], l[6], acc[6][128]
-constexpr size_t kDecSmem = (size_t)kDecStages * kStageBytes + 1024;
+constexpr int kGroup = 6;                  // query heads per KV head
+constexpr int kNPad = 16;                  // MMA N: the group's heads padded with zero rows
+constexpr int kTok = 128;                  // tokens per tile (MMA M)
+constexpr int kDecStages = 3;
+constexpr uint32_t kDecTileBytes = kTok * kD * 2;        // 32 KB: one K or V tile
+constexpr uint32_t kDecHalfBytes = kDecTileBytes / 2;    // one 64-column swizzled box
+constexpr uint32_t kDecStageBytes = 2 * kDecTileBytes;   // K + V
+constexpr uint32_t kOpBytes = kNPad * kD * 2;            // 4 KB: Q or P^T operand
+constexpr size_t kDecSmem = 1024 + kDecStages * kDecStageBytes + 3 * kOpBytes;
+constexpr int kDecThreads = 192;
+constexpr int kPartFloats = kGroup * (kD + 2);           // m[6], l[6], acc[6][128]
+constexpr uint32_t kDecTmemCols = 64;                    // S^T x2 (16 each) + O^T (16)
 
 struct DecodeArgs {
-    const __nv_bfloat16 *full_k, *full_v, *strm_k, *strm_v;
+    CUtensorMap tm_fk, tm_fv;       // full caches as 2-D (128, B*n_full*capacity)
+    CUtensorMap tm_rk, tm_rv;       // ring caches as 2-D (128, B*n_ring*slots)
     const int32_t *seq_len, *ring_head;
     const __nv_bfloat16 *q;         // [B][Hq][D]
     const float *sink_logit;        // [Hq] or null
@@ -44,268 +60,416 @@ struct DecodeArgs {
     int64_t capacity;
     int32_t batch, hkv, n_full, n_ring;
     int32_t sink, ring, slots;
-    int32_t chunk_full, splits_full, chunk_ring, splits_ring, max_splits;
+    int32_t chunk_full, splits_full, chunk_ring, splits_ring, max_splits, n_items;
     float scale_log2;               // softmax_scale * log2(e)
+    int32_t withhold_tile;          // test hook: CTA 0 issues no load from this tile on (-1: off)
     int8_t full_head[64];           // full rank -> KV head
     int8_t ring_head_of[64];        // ring rank -> KV head
     HeadTable heads;
 };
 
-// Tokens of one work item: logical index e in [e_begin, e_end) maps to a
-// cache row.  Full heads: row e.  Ring heads: sink slot e for e < n_sink,
-// else ring slot sink + (ring_base + e - n_sink) mod ring.
-struct Span {
-    const char *k_base;
-    const char *v_base;
-    int32_t e_begin, e_end;
-    int32_t n_sink, ring_base;
+// One work item: rows [row0 + e_begin, row0 + e_end) of a cache tensor map.
+// For a ring item the index e is the slot; slot validity follows the ring
+// state (sink slots below n_sink; ring slots among the cnt written last).
+struct Item {
+    int b, g, split;
     bool ring;
+    int32_t row0, e_begin, e_end;
+    int32_t n_sink, cnt, ring_base;
+    int n_tiles;
 };
 
-__device__ __forceinline__ int32_t span_slot(const Span &s, int32_t e, int32_t sink, int32_t ring) {
-    if (!s.ring || e < s.n_sink) return e;
-    int32_t r = s.ring_base + (e - s.n_sink);
-    if (r >= ring) r -= ring;
-    return sink + r;
-}
-
-// Issues the copies for tokens [e0, e0 + count) into one stage.
-__device__ __forceinline__ void issue_tile(const Span &s, int32_t e0, int32_t count, char *stage,
-                                           uint64_t *bar, int32_t sink, int32_t ring) {
-    mbar_expect_tx(bar, (uint32_t)count * kRowBytes * 2);
-    int32_t e = e0;
-    const int32_t e1 = e0 + count;
-    while (e < e1) {
-        // extend a run of consecutive slots
-        const int32_t slot0 = span_slot(s, e, sink, ring);
-        int32_t run = 1;
-        while (e + run < e1 && span_slot(s, e + run, sink, ring) == slot0 + run) ++run;
-        const uint32_t bytes = (uint32_t)run * kRowBytes;
-        char *dk = stage + (size_t)(e - e0) * kRowBytes;
-        char *dv = stage + kDecTile * kRowBytes + (size_t)(e - e0) * kRowBytes;
-        bulk_g2s(dk, s.k_base + (size_t)slot0 * kRowBytes, bytes, bar);
-        bulk_g2s(dv, s.v_base + (size_t)slot0 * kRowBytes, bytes, bar);
-        e += run;
-    }
-}
-
-__global__ void __launch_bounds__(kDecThreads, 1) decode_split(const DecodeArgs a) {
-    extern __shared__ __align__(1024) char dsmem_raw[];
-    char *smem = (char *)(((uintptr_t)dsmem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t full_bar[kDecStages], empty_bar[kDecStages];
-    __shared__ float red_m[32][kHalf], red_l[32][kHalf];
-
-    // ---------------------------------------------------------------- work item
-    const int32_t n_full_items = a.batch * a.n_full * a.splits_full;
-    int32_t w = blockIdx.x;
-    int b, g, split;
-    Span s;
+__device__ __forceinline__ Item item_of(const DecodeArgs &a, int w) {
+    Item it;
+    const int n_full_items = a.batch * a.n_full * a.splits_full;
     if (w < n_full_items) {
         const int unit = w / a.splits_full;
-        split = w % a.splits_full;
-        b = unit / a.n_full;
+        it.split = w % a.splits_full;
+        it.b = unit / a.n_full;
         const int r = unit % a.n_full;
-        g = a.full_head[r];
-        const int32_t n = a.seq_len[b];
-        const size_t base = (((size_t)b * a.n_full + r) * a.capacity) * kRowBytes;
-        s.k_base = (const char *)a.full_k + base;
-        s.v_base = (const char *)a.full_v + base;
-        s.e_begin = split * a.chunk_full;
-        s.e_end = min(n, s.e_begin + a.chunk_full);
-        s.ring = false;
-        s.n_sink = 0;
-        s.ring_base = 0;
+        it.g = a.full_head[r];
+        it.ring = false;
+        it.row0 = (int32_t)(((int64_t)it.b * a.n_full + r) * a.capacity);
+        const int32_t n = a.seq_len[it.b];
+        it.e_begin = it.split * a.chunk_full;
+        it.e_end = min(n, it.e_begin + a.chunk_full);
+        it.n_sink = 0;
+        it.cnt = 0;
+        it.ring_base = 0;
     } else {
         w -= n_full_items;
         const int unit = w / a.splits_ring;
-        split = w % a.splits_ring;
-        b = unit / a.n_ring;
+        it.split = w % a.splits_ring;
+        it.b = unit / a.n_ring;
         const int r = unit % a.n_ring;
-        g = a.ring_head_of[r];
-        const int32_t n = a.seq_len[b];
-        const int32_t n_sink = min(n, a.sink);
-        const int32_t cnt = min(max(n - a.sink, 0), a.ring);
-        int32_t base_r = (a.ring_head[b] - cnt) % a.ring;
-        if (base_r < 0) base_r += a.ring;
-        const size_t base = (((size_t)b * a.n_ring + r) * a.slots) * kRowBytes;
-        s.k_base = (const char *)a.strm_k + base;
-        s.v_base = (const char *)a.strm_v + base;
-        s.e_begin = split * a.chunk_ring;
-        s.e_end = min(n_sink + cnt, s.e_begin + a.chunk_ring);
-        s.ring = true;
-        s.n_sink = n_sink;
-        s.ring_base = base_r;
+        it.g = a.ring_head_of[r];
+        it.ring = true;
+        it.row0 = (int32_t)(((int64_t)it.b * a.n_ring + r) * a.slots);
+        const int32_t n = a.seq_len[it.b];
+        it.n_sink = min(n, a.sink);
+        it.cnt = min(max(n - a.sink, 0), a.ring);
+        int32_t base = (a.ring_head[it.b] - it.cnt) % a.ring;
+        it.ring_base = base < 0 ? base + a.ring : base;
+        it.e_begin = it.split * a.chunk_ring;
+        // nothing valid past the sink while the ring is empty
+        const int32_t last = (it.cnt == 0) ? it.n_sink : a.slots;
+        it.e_end = min(last, it.e_begin + a.chunk_ring);
     }
-    const int32_t total = max(s.e_end - s.e_begin, 0);
-    const int32_t n_tiles = (total + kDecTile - 1) / kDecTile;
+    it.n_tiles = it.e_end > it.e_begin ? (it.e_end - it.e_begin + kTok - 1) / kTok : 0;
+    return it;
+}
 
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
+__device__ __forceinline__ bool token_valid(const Item &it, int32_t e, int32_t sink, int32_t ring) {
+    if (e >= it.e_end) return false;
+    if (!it.ring) return true;
+    if (e < sink) return e < it.n_sink;
+    int32_t r = e - sink - it.ring_base;
+    if (r < 0) r += ring;
+    return r < it.cnt;
+}
+
+// Byte offset of element (row, k) in a [16 rows][128] bf16 K-major operand
+// stored as two 64-column halves with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t op_offset(int row, int k) {
+    const int half = k >> 6, kk = k & 63;
+    return half * 2048 + (row >> 3) * 1024 + (row & 7) * 128 + ((((kk >> 3) ^ (row & 7))) << 4) +
+           (kk & 7) * 2;
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int c0, int c1, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(tmap), "r"(c0), "r"(c1), "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+                   "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
+__device__ __forceinline__ void reg_fence8(uint32_t (&r)[8]) {
+    asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]));
+}
+
+// Named barrier over the four softmax warps (threads 0..127).
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t v_addr, uint32_t p_addr,
+                                         uint32_t idesc, bool first) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        mma_ss(o_tmem, smem_desc_sw128(v_addr + k * 2048, kDecHalfBytes, 1024),
+               smem_desc_sw128(p_addr + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), idesc,
+               (first && k == 0) ? 0u : 1u);
+}
+
+__global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_constant__ DecodeArgs a) {
+    extern __shared__ __align__(16) char dsmem_base[];
+    char *smem = dsmem_base + ((1024u - (smem_u32(dsmem_base) & 1023u)) & 1023u);
+    char *sKV = smem;                                         // [stages][K 32 KB | V 32 KB]
+    char *sQ = smem + kDecStages * kDecStageBytes;            // [2 items][4 KB]
+    char *sP = sQ + 2 * kOpBytes;                             // 4 KB
+    __shared__ uint64_t kv_full[kDecStages], kv_empty[kDecStages];
+    __shared__ uint64_t s_full[2], p_full, o_done, q_ready[2];
+    __shared__ uint32_t tmem_base;
+    __shared__ float red_max[2][4][kGroup], red_sum[4][kGroup];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDecStages; ++i) {
-            mbar_init(&full_bar[i], 1);
-            mbar_init(&empty_bar[i], kDecComputeWarps);
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
         }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&q_ready[i], 4);
+        }
+        mbar_init(&p_full, 4);
+        mbar_init(&o_done, 1);
         fence_mbar_init();
     }
-    __syncwarp();      // reconverge before the CTA barrier (bar.sync is warp-aligned)
+    if (warp < 4) {
+        // operand rows 6..15 stay zero for the whole kernel
+        for (int i = threadIdx.x; i < 3 * (int)kOpBytes / 16; i += 128)
+            reinterpret_cast<uint4 *>(sQ)[i] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+    }
+    if (warp == 5) {
+        tmem_alloc(&tmem_base, kDecTmemCols);
+        tmem_relinquish();
+    }
+    __syncwarp();
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
 
-    // ---------------------------------------------------------------- producer warp
-    if (warp == kDecComputeWarps) {
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
         if (lane == 0) {
-            for (int t = 0; t < n_tiles; ++t) {
-                const int st = t % kDecStages;
-                if (t >= kDecStages && !mbar_wait(&empty_bar[st], ((t / kDecStages) - 1) & 1)) break;
-                const int32_t e0 = s.e_begin + t * kDecTile;
-                issue_tile(s, e0, min(kDecTile, s.e_end - e0), smem + (size_t)st * kStageBytes,
-                           &full_bar[st], a.sink, a.ring);
+            if (a.n_full > 0) {
+                prefetch_tmap(&a.tm_fk);
+                prefetch_tmap(&a.tm_fv);
+            }
+            if (a.n_ring > 0) {
+                prefetch_tmap(&a.tm_rk);
+                prefetch_tmap(&a.tm_rv);
+            }
+            int jg = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x) {
+                const Item it = item_of(a, w);
+                const CUtensorMap *tk = it.ring ? &a.tm_rk : &a.tm_fk;
+                const CUtensorMap *tv = it.ring ? &a.tm_rv : &a.tm_fv;
+                for (int t = 0; t < it.n_tiles; ++t, ++jg) {
+                    const int st = jg % kDecStages;
+                    if (jg >= kDecStages && !(ok = mbar_wait(&kv_empty[st], ((jg / kDecStages) - 1) & 1))) break;
+                    // failure-detection test: stop feeding this CTA so that the
+                    // consumers' bounded waits expire (nothing stays in flight)
+                    if (blockIdx.x == 0 && jg == a.withhold_tile) { ok = false; break; }
+                    char *ks = sKV + st * kDecStageBytes;
+                    const int row = it.row0 + it.e_begin + t * kTok;
+                    mbar_expect_tx(&kv_full[st], kDecStageBytes);
+                    tma_load_2d(ks, tk, 0, row, &kv_full[st]);
+                    tma_load_2d(ks + kDecHalfBytes, tk, 64, row, &kv_full[st]);
+                    tma_load_2d(ks + kDecTileBytes, tv, 0, row, &kv_full[st]);
+                    tma_load_2d(ks + kDecTileBytes + kDecHalfBytes, tv, 64, row, &kv_full[st]);
+                }
             }
         }
-        __syncwarp();  // lanes 1..31 wait for the producer lane before any CTA barrier
-        // the producer warp joins the final reduction below
-    }
-
-    // ---------------------------------------------------------------- compute warps
-    // 32 groups of 8 lanes: group j handles heads [3*(j/16), 3*(j/16)+3) for
-    // tokens j%16, j%16+16, ... of every tile; lane l of the group owns the
-    // d-slices [8l, 8l+8) and [64+8l, 64+8l+8).  Pairs of adjacent d are
-    // held packed and multiplied with the f32x2 FMA.
-    const int grp = threadIdx.x >> 3;          // 0..31 for compute warps
-    const int l8 = threadIdx.x & 7;
-    const int half = grp >> 4;
-    const int tok0 = grp & 15;
-    // groups of one warp may run different trip counts on a short tile, so
-    // every shuffle names only the 8 lanes of its own group
-    const unsigned gmask = 0xFFu << (lane & 24);
-    f2 qf[kHalf][8];
-    f2 acc[kHalf][8];
-    float m[kHalf], lsum[kHalf];
+        __syncwarp();
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_qk = idesc_bf16_f32(kTok, kNPad, 0, 0);
+            const uint32_t id_pv = idesc_bf16_f32(kD, kNPad, 1, 0);
+            const uint32_t kv_addr = smem_u32(sKV), q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
+            const uint32_t o_tmem = tmem + 2 * kNPad;
+            int jg = 0, ic = 0;            // tiles and non-empty items so far
+            bool ok = true;
+            bool pend = false;             // a PV is owed for the previous tile
+            int pend_st = 0;
+            bool pend_first = false;
+            for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x) {
+                const Item it = item_of(a, w);
+                if (it.n_tiles == 0) continue;
+                if (!(ok = mbar_wait(&q_ready[ic & 1], (ic >> 1) & 1))) break;
+                for (int t = 0; t < it.n_tiles && ok; ++t, ++jg) {
+                    const int st = jg % kDecStages;
+                    if (!(ok = mbar_wait(&kv_full[st], (jg / kDecStages) & 1))) break;
+                    tc_fence_after();
 #pragma unroll
-    for (int h = 0; h < kHalf; ++h) {
-        m[h] = -INFINITY;
-        lsum[h] = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[h][i] = f2_splat(0.f);
-    }
-    bool ok = true;
-    if (warp < kDecComputeWarps) {
-        const int hq0 = g * kGroup + half * kHalf;
-#pragma unroll
-        for (int h = 0; h < kHalf; ++h) {
-            const uint4 *qrow = (const uint4 *)(a.q + ((size_t)b * a.hkv * kGroup + hq0 + h) * kD);
-            const uint4 c0 = qrow[l8], c1 = qrow[l8 + 8];
-            const uint32_t qw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                qf[h][i] = f2_make(bf16lo(qw[i]) * a.scale_log2, bf16hi(qw[i]) * a.scale_log2);
-        }
-        for (int t = 0; t < n_tiles && ok; ++t) {
-            const int st = t % kDecStages;
-            if (!mbar_wait(&full_bar[st], (t / kDecStages) & 1)) { ok = false; break; }
-            const char *kt = smem + (size_t)st * kStageBytes;
-            const char *vt = kt + kDecTile * kRowBytes;
-            const int count = min(kDecTile, s.e_end - (s.e_begin + t * kDecTile));
-#pragma unroll 1
-            for (int tt = tok0; tt < count; tt += 16) {
-                const uint4 k0 = *(const uint4 *)(kt + tt * kRowBytes + l8 * 16);
-                const uint4 k1 = *(const uint4 *)(kt + tt * kRowBytes + (l8 + 8) * 16);
-                const uint4 v0 = *(const uint4 *)(vt + tt * kRowBytes + l8 * 16);
-                const uint4 v1 = *(const uint4 *)(vt + tt * kRowBytes + (l8 + 8) * 16);
-                const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-                const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                f2 x[kHalf];
-#pragma unroll
-                for (int h = 0; h < kHalf; ++h) x[h] = f2_splat(0.f);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const f2 kf = f2_make(bf16lo(kw[i]), bf16hi(kw[i]));
-#pragma unroll
-                    for (int h = 0; h < kHalf; ++h) x[h] = f2_fma(qf[h][i], kf, x[h]);
-                }
-                float sc[kHalf];
-#pragma unroll
-                for (int h = 0; h < kHalf; ++h) sc[h] = f2_sum(x[h]);
-#pragma unroll
-                for (int off = 1; off < 8; off <<= 1)
-#pragma unroll
-                    for (int h = 0; h < kHalf; ++h) sc[h] += __shfl_xor_sync(gmask, sc[h], off);
-                f2 pp[kHalf];
-#pragma unroll
-                for (int h = 0; h < kHalf; ++h) {
-                    if (sc[h] > m[h]) {
-                        const f2 alpha = f2_splat(ex2_approx(m[h] - sc[h]));
-                        lsum[h] *= alpha.x;
-                        m[h] = sc[h];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) acc[h][i] = f2_mul(acc[h][i], alpha);
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = (k >> 2) * kDecHalfBytes + (k & 3) * 32;
+                        const uint32_t qoff = (ic & 1) * kOpBytes + (k >> 2) * 2048 + (k & 3) * 32;
+                        mma_ss(tmem + (jg & 1) * kNPad,
+                               smem_desc_sw128(kv_addr + st * kDecStageBytes + off, 16, 1024),
+                               smem_desc_sw128(q_addr + qoff, 16, 1024), id_qk, k > 0);
                     }
-                    const float p = ex2_approx(sc[h] - m[h]);
-                    lsum[h] += p;
-                    pp[h] = f2_splat(p);
+                    mma_commit(&s_full[jg & 1]);
+                    if (pend) {
+                        // PV of the previous tile, one tile behind its QK
+                        if (!(ok = mbar_wait(&p_full, (jg - 1) & 1))) break;
+                        tc_fence_after();
+                        issue_pv(o_tmem, kv_addr + pend_st * kDecStageBytes + kDecTileBytes, p_addr,
+                                 id_pv, pend_first);
+                        mma_commit(&o_done);
+                        mma_commit(&kv_empty[pend_st]);
+                    }
+                    pend = true;
+                    pend_st = st;
+                    pend_first = (t == 0);
                 }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const f2 vf = f2_make(bf16lo(vw[i]), bf16hi(vw[i]));
-#pragma unroll
-                    for (int h = 0; h < kHalf; ++h) acc[h][i] = f2_fma(pp[h], vf, acc[h][i]);
-                }
+                ++ic;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty_bar[st]);
+            if (ok && pend && mbar_wait(&p_full, (jg - 1) & 1)) {
+                tc_fence_after();
+                issue_pv(o_tmem, kv_addr + pend_st * kDecStageBytes + kDecTileBytes, p_addr, id_pv,
+                         pend_first);
+                mma_commit(&o_done);
+                mma_commit(&kv_empty[pend_st]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int r = threadIdx.x;                           // token row / output dimension
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t o_tmem = tmem + 2 * kNPad + lane_base;
+        const float c = a.scale_log2;
+        // Stages the 6 query rows of the first non-empty item at or after w
+        // as the swizzled K-major Q operand in buffer `buf`.
+        auto stage_q = [&](int w, int buf) {
+            for (; w < a.n_items; w += gridDim.x) {
+                const Item nx = item_of(a, w);
+                if (nx.n_tiles == 0) continue;
+                if (r < kGroup * 16) {
+                    const int h = r >> 4, ch = r & 15;
+                    const uint4 v = reinterpret_cast<const uint4 *>(
+                        a.q + ((size_t)nx.b * a.hkv * kGroup + nx.g * kGroup + h) * kD)[ch];
+                    *reinterpret_cast<uint4 *>(sQ + buf * kOpBytes + op_offset(h, ch * 8)) = v;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&q_ready[buf]);
+                return;
+            }
+        };
+        int jg = 0, ic = 0;                // tiles and non-empty items so far
+        bool ok = true;
+        stage_q(blockIdx.x, 0);
+        for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x) {
+            const Item it = item_of(a, w);
+            float m_run[kGroup], l_part[kGroup];
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) {
+                m_run[h] = -INFINITY;
+                l_part[h] = 0.f;
+            }
+            for (int t = 0; t < it.n_tiles; ++t, ++jg) {
+                const bool got = mbar_wait(&s_full[jg & 1], (jg >> 1) & 1);
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sr[8];
+                tmem_ld8(tmem + (jg & 1) * kNPad + lane_base, sr);
+                tmem_ld_wait();
+                reg_fence8(sr);
+                const int32_t e = it.e_begin + t * kTok + r;
+                const bool valid = token_valid(it, e, a.sink, a.ring);
+                float s[kGroup], mx[kGroup];
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    s[h] = valid ? __uint_as_float(sr[h]) : -INFINITY;
+                    mx[h] = s[h];
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                    for (int h = 0; h < kGroup; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], off));
+                if (lane == 0)
+#pragma unroll
+                    for (int h = 0; h < kGroup; ++h) red_max[jg & 1][warp][h] = mx[h];
+                softmax_sync();
+                float alpha[kGroup], m_sub[kGroup];
+                bool rescale = false;
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    const float m_tile = fmaxf(fmaxf(red_max[jg & 1][0][h], red_max[jg & 1][1][h]),
+                                               fmaxf(red_max[jg & 1][2][h], red_max[jg & 1][3][h])) * c;
+                    alpha[h] = 1.f;
+                    // keep the stale max unless the new one is more than 2^8 larger
+                    if (m_tile > m_run[h] + 8.f) {
+                        alpha[h] = (m_run[h] == -INFINITY) ? 0.f : ex2_approx(m_run[h] - m_tile);
+                        m_run[h] = m_tile;
+                        rescale = true;
+                    }
+                    m_sub[h] = (m_run[h] == -INFINITY) ? 0.f : m_run[h];
+                }
+                float p[kGroup];
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) {
+                    p[h] = ex2_approx(fmaf(s[h], c, -m_sub[h]));
+                    l_part[h] = fmaf(l_part[h], alpha[h], p[h]);
+                }
+                // the previous PV must be done with P^T and with O^T
+                if (jg > 0) {
+                    const bool prev = mbar_wait(&o_done, (jg - 1) & 1);
+                    __syncwarp();
+                    if (!__all_sync(0xffffffffu, prev)) { ok = false; break; }
+                    tc_fence_after();
+                }
+                if (t > 0 && rescale) {
+                    uint32_t orr[8];
+                    tmem_ld8(o_tmem, orr);
+                    tmem_ld_wait();
+                    reg_fence8(orr);
+#pragma unroll
+                    for (int h = 0; h < kGroup; ++h) orr[h] = __float_as_uint(__uint_as_float(orr[h]) * alpha[h]);
+                    tmem_st8(o_tmem, orr);
+                    tmem_st_wait();
+                }
+                if (!valid) {
+                    // stale cache rows must not reach the PV product (0 x NaN)
+                    char *vrow = sKV + (jg % kDecStages) * kDecStageBytes + kDecTileBytes + r * 128;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        reinterpret_cast<uint4 *>(vrow)[i] = make_uint4(0, 0, 0, 0);
+                        reinterpret_cast<uint4 *>(vrow + kDecHalfBytes)[i] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h)
+                    *reinterpret_cast<__nv_bfloat16 *>(sP + op_offset(h, r)) = __float2bfloat16_rn(p[h]);
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full);
+            }
+            if (!ok) break;
+            if (it.n_tiles > 0) {
+                // the MMA warp may start the next item's QK while this epilogue runs
+                ++ic;
+                stage_q(w + gridDim.x, ic & 1);
+            }
+            // ------------------------------------------------------------ item epilogue
+            float acc[kGroup];
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) acc[h] = 0.f;
+            if (it.n_tiles > 0) {
+                const bool done = mbar_wait(&o_done, (jg - 1) & 1);
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, done)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t orr[8];
+                tmem_ld8(o_tmem, orr);
+                tmem_ld_wait();
+                reg_fence8(orr);
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) acc[h] = __uint_as_float(orr[h]);
+            }
+            // l: sum of the 128 per-token partials, in a fixed order
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) l_part[h] += __shfl_xor_sync(0xffffffffu, l_part[h], off);
+            if (lane == 0)
+#pragma unroll
+                for (int h = 0; h < kGroup; ++h) red_sum[warp][h] = l_part[h];
+            softmax_sync();
+            float *part = a.part + (((size_t)it.b * a.hkv + it.g) * a.max_splits + it.split) * kPartFloats;
+#pragma unroll
+            for (int h = 0; h < kGroup; ++h) part[2 * kGroup + h * kD + r] = acc[h];
+            if (r < kGroup) {
+                part[r] = m_run[r];
+                part[kGroup + r] = (red_sum[0][r] + red_sum[1][r]) + (red_sum[2][r] + red_sum[3][r]);
+            }
+            softmax_sync();    // red_sum is reused by the next item
         }
         __syncwarp();
     }
-    __syncthreads();   // every copy has landed and been consumed; stages are free
-
-    // ---------------------------------------------------------------- combine the 32 groups
-    float *red_acc = (float *)smem;              // [kGroup][kD]
-    for (int i = threadIdx.x; i < kGroup * kD; i += blockDim.x) red_acc[i] = 0.f;
-    if (warp < kDecComputeWarps && l8 == 0) {
-#pragma unroll
-        for (int h = 0; h < kHalf; ++h) {
-            red_m[grp][h] = m[h];
-            red_l[grp][h] = lsum[h];
-        }
-    }
-    __syncwarp();
+    tc_fence_before();
     __syncthreads();
-    if (warp < kDecComputeWarps) {
-#pragma unroll
-        for (int h = 0; h < kHalf; ++h) {
-            float M = -INFINITY;
-            for (int j = 0; j < 16; ++j) M = fmaxf(M, red_m[half * 16 + j][h]);
-            const float f = (m[h] == -INFINITY) ? 0.f : ex2_approx(m[h] - M);
-            float *dst = red_acc + (half * kHalf + h) * kD;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int d = (i < 4 ? 8 * l8 : 64 + 8 * l8) + 2 * (i & 3);
-                atomicAdd(dst + d, acc[h][i].x * f);
-                atomicAdd(dst + d + 1, acc[h][i].y * f);
-            }
-        }
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kDecTmemCols);
     }
-    __syncthreads();
-    float *part = a.part + (((size_t)b * a.hkv + g) * a.max_splits + split) * kPartFloats;
-    if (threadIdx.x < kGroup) {
-        const int hh = threadIdx.x, hf = hh / kHalf, h = hh % kHalf;
-        float M = -INFINITY;
-        for (int j = 0; j < 16; ++j) M = fmaxf(M, red_m[hf * 16 + j][h]);
-        float L = 0.f;
-        if (M != -INFINITY)
-            for (int j = 0; j < 16; ++j) {
-                const float mj = red_m[hf * 16 + j][h];
-                if (mj != -INFINITY) L += red_l[hf * 16 + j][h] * ex2_approx(mj - M);
-            }
-        part[hh] = M;
-        part[kGroup + hh] = L;
-    }
-    for (int i = threadIdx.x; i < kGroup * kD; i += blockDim.x) part[2 * kGroup + i] = red_acc[i];
 }
 
 // Folds the splits of every (sequence, query head) and the sink logit:
 // O = sum_s 2^(m_s - M) acc_s / (sum_s 2^(m_s - M) l_s + 2^(sigma*log2e - M)).
-__global__ void __launch_bounds__(kD) decode_merge(const DecodeArgs a) {
+__global__ void __launch_bounds__(kD) decode_merge(const __grid_constant__ DecodeArgs a) {
     const int bh = blockIdx.x;
     const int b = bh / (a.hkv * kGroup);
     const int h = bh % (a.hkv * kGroup);

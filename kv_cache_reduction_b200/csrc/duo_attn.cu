@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "duo_attn.h"
@@ -140,41 +141,70 @@ int set_smem_once(Kernel kernel, size_t bytes, const char *name, bool (&done)[64
 
 // ------------------------------------------------------------------ decode plan
 struct DecodePlan {
-    int chunk_full = duo::kDecTile, splits_full = 0;
-    int chunk_ring = duo::kDecTile, splits_ring = 0;
+    int chunk_full = duo::kTok, splits_full = 0;
+    int chunk_ring = duo::kTok, splits_ring = 0;
     int max_splits = 1;
     int64_t items = 0;
+    int grid = 0;
 };
 
-int round_up(int64_t x, int m) { return (int)((x + m - 1) / m * m); }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Splits long full-head caches so that the grid holds about eight CTAs per
-// SM in total (one CTA is resident per SM), and ring heads into pieces of
-// whole tiles when there are too few of them to fill the GPU.
+// Items are processed by one persistent CTA per SM, round robin.  Full-head
+// caches are cut into equal chunks of whole 128-token tiles; the chunk count
+// is the one that minimises the estimated makespan (tiles of the busiest
+// CTA plus a small per-item cost).  Ring heads take one item each unless
+// there are too few of them to occupy the SMs.
 DecodePlan plan_decode(const duo_params *p, const Layout &L, int64_t max_n, int sms) {
     DecodePlan d;
     const int64_t ring_units = (int64_t)p->batch * L.n_ring;
     const int64_t full_units = (int64_t)p->batch * L.n_full;
-    const int ring_valid = L.slots;
+    const int64_t ring_tiles = cdiv(L.slots, duo::kTok);
+    const double item_cost = 0.5;      // pipeline fill and epilogue, in tiles
     if (ring_units > 0) {
-        int want = (int)std::max<int64_t>(1, (2 * sms + ring_units - 1) / ring_units);
-        if (full_units > 0 && max_n > 4 * ring_valid) want = 1;   // full heads fill the GPU
-        const int max_pieces = (ring_valid + duo::kDecTile - 1) / duo::kDecTile;
-        want = std::min(want, max_pieces);
-        d.chunk_ring = round_up((ring_valid + want - 1) / want, duo::kDecTile);
-        d.splits_ring = (ring_valid + d.chunk_ring - 1) / d.chunk_ring;
+        int64_t want = 1;
+        if (full_units == 0 || max_n <= 4 * L.slots)
+            want = std::min<int64_t>(ring_tiles, std::max<int64_t>(1, cdiv(sms, ring_units)));
+        d.chunk_ring = (int)(cdiv(ring_tiles, want) * duo::kTok);
+        d.splits_ring = (int)cdiv(L.slots, d.chunk_ring);
     }
+    const int64_t ring_items = ring_units * d.splits_ring;
+    const double ring_cost = ring_items > 0 ? (double)cdiv(d.chunk_ring, duo::kTok) + item_cost : 0.0;
     if (full_units > 0) {
         const int64_t n = std::max<int64_t>(max_n, 1);
-        const int64_t budget = std::max<int64_t>(8 * (int64_t)sms - ring_units * d.splits_ring, 4 * sms);
-        int64_t chunk = (full_units * n + budget - 1) / budget;
-        chunk = std::max<int64_t>(round_up(chunk, duo::kDecTile), 256);
-        d.chunk_full = (int)std::min<int64_t>(chunk, round_up(n, duo::kDecTile));
-        d.splits_full = (int)((n + d.chunk_full - 1) / d.chunk_full);
+        const int64_t tiles = cdiv(n, duo::kTok);
+        double best = 1e300;
+        for (int64_t s = 1; s <= std::min<int64_t>(tiles, 1024); ++s) {
+            const int64_t chunk_tiles = cdiv(tiles, s);
+            const int64_t splits = cdiv(tiles, chunk_tiles);
+            const int64_t items = full_units * splits;
+            const double cost = (double)cdiv(items, sms) * ((double)chunk_tiles + item_cost) +
+                                (double)cdiv(ring_items, sms) * ring_cost;
+            if (cost < best - 1e-9) {
+                best = cost;
+                d.chunk_full = (int)(chunk_tiles * duo::kTok);
+                d.splits_full = (int)splits;
+            }
+        }
     }
     d.max_splits = std::max(1, std::max(d.splits_full, d.splits_ring));
-    d.items = full_units * d.splits_full + ring_units * d.splits_ring;
+    d.items = full_units * d.splits_full + ring_items;
+    d.grid = (int)std::min<int64_t>(d.items, sms);
     return d;
+}
+
+// A cache viewed as a 2-D tensor (128 columns, rows) loaded in 64-column x
+// 128-row boxes with the 128-byte swizzle.
+bool cache_tmap(CUtensorMap *m, void *base, int64_t rows) {
+    duo::EncodeTiledFn fn = duo::encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {duo::kD, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {duo::kD * 2};
+    const cuuint32_t box[2] = {64, duo::kTok};
+    const cuuint32_t elem[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, elem,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 size_t workspace_bytes(const duo_params *p, const DecodePlan &d) {
@@ -265,6 +295,9 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     if (!q || !out) return fail(DUO_ERR_INVALID_ARG, "q / out is NULL");
     if (!aligned16(q) || !aligned16(out) || (lse && !aligned16(lse)))
         return fail(DUO_ERR_INVALID_ARG, "q / out / lse must be 16-byte aligned");
+    if ((int64_t)params->batch * L.n_full * (L.n_full ? cache->capacity : 0) > INT32_MAX ||
+        (int64_t)params->batch * L.n_ring * L.slots > INT32_MAX)
+        return fail(DUO_ERR_UNSUPPORTED, "cache rows exceed 2^31 (tensor-map coordinates are 32-bit)");
     int sms = 148;
     if ((rc = check_device(&sms))) return rc;
     const DecodePlan d = plan_decode(params, L, max_seq_len, sms);
@@ -272,11 +305,16 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     if (!workspace || workspace_size < need || ((uintptr_t)workspace & 255u))
         return fail(DUO_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
                     workspace_size);
-    duo::DecodeArgs a{};
-    a.full_k = (const __nv_bfloat16 *)cache->full_k;
-    a.full_v = (const __nv_bfloat16 *)cache->full_v;
-    a.strm_k = (const __nv_bfloat16 *)cache->strm_k;
-    a.strm_v = (const __nv_bfloat16 *)cache->strm_v;
+    duo::DecodeArgs a;
+    memset(&a, 0, sizeof a);
+    if (L.n_full > 0 &&
+        (!cache_tmap(&a.tm_fk, cache->full_k, (int64_t)params->batch * L.n_full * cache->capacity) ||
+         !cache_tmap(&a.tm_fv, cache->full_v, (int64_t)params->batch * L.n_full * cache->capacity)))
+        return fail(DUO_ERR_CUDA, "cuTensorMapEncodeTiled failed for the full cache");
+    if (L.n_ring > 0 &&
+        (!cache_tmap(&a.tm_rk, cache->strm_k, (int64_t)params->batch * L.n_ring * L.slots) ||
+         !cache_tmap(&a.tm_rv, cache->strm_v, (int64_t)params->batch * L.n_ring * L.slots)))
+        return fail(DUO_ERR_CUDA, "cuTensorMapEncodeTiled failed for the ring cache");
     a.seq_len = cache->seq_len;
     a.ring_head = cache->ring_head;
     a.q = (const __nv_bfloat16 *)q;
@@ -297,7 +335,13 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     a.chunk_ring = d.chunk_ring;
     a.splits_ring = d.splits_ring;
     a.max_splits = d.max_splits;
+    a.n_items = (int32_t)d.items;
     a.scale_log2 = params->softmax_scale * duo::kLog2eF;
+    // Test hook for the failure-detection path: DUO_TEST_WITHHOLD_TILE=t makes
+    // the first CTA's producer stop before tile t; its consumers then time out
+    // and the call reports DUO_ERR_TIMEOUT through duo_get_device_status().
+    const char *withhold = getenv("DUO_TEST_WITHHOLD_TILE");
+    a.withhold_tile = withhold ? atoi(withhold) : -1;
     memcpy(a.full_head, L.full_head, sizeof a.full_head);
     memcpy(a.ring_head_of, L.ring_head_of, sizeof a.ring_head_of);
     a.heads = L.heads;
@@ -305,7 +349,7 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     static bool smem_set[64] = {};
     if ((rc = set_smem_once(duo::decode_split, duo::kDecSmem, "decode_split", smem_set))) return rc;
     if (d.items > 0) {
-        duo::decode_split<<<(unsigned)d.items, duo::kDecThreads, duo::kDecSmem, st>>>(a);
+        duo::decode_split<<<(unsigned)d.grid, duo::kDecThreads, duo::kDecSmem, st>>>(a);
         if ((rc = launch_status("decode_split"))) return rc;
     }
     duo::decode_merge<<<(unsigned)((int64_t)params->batch * params->num_q_heads), duo::kD, 0, st>>>(a);

@@ -163,44 +163,70 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         __syncwarp();  // lanes 1..31 wait for the producer lane before the CTA barrier
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Each head alternates S_h = Q_h K_j^T and O_h += P_h V_j.  The two
+        // heads are polled independently, so one head's softmax never holds
+        // back the other head's next product.  S_h(j+1) overwrites P_h(j),
+        // so it waits for P_h(j) V_j to complete.
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(kPfM, kPfN, 0, 0);
             const uint32_t id_pv = idesc_bf16_f32(kPfM, 128, 0, 1);
             const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
             bool ok = mbar_wait(&q_full, 0);
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int st = j % kPfStages;
-                const uint32_t par = (j / kPfStages) & 1;
-                if (!(ok = mbar_wait(&k_full[st], par))) break;
-                tc_fence_after();
-                for (int h = 0; h < 2 && ok; ++h) {
-                    // S_h aliases P_h: the previous P_h V must be done reading it
-                    if (j > 0 && !(ok = mbar_wait(&o_done[h], (j - 1) & 1))) break;
-                    tc_fence_after();
-                    const uint32_t s_tmem = tmem + h * 128;
+            tc_fence_after();
+            int jh[2] = {0, 0};              // next key tile of each head
+            bool want_qk[2] = {true, true};  // next product of each head is S (else PV)
+            int pv_in_stage[kPfStages] = {};
+            unsigned long long idle_since = clock64();
+            while (ok && (jh[0] < n_kv || jh[1] < n_kv)) {
+                bool progressed = false;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (k >> 2) * kHalfTileBytes + (k & 3) * 32;
-                        mma_ss(s_tmem, smem_desc_sw128(q_addr + h * kTileBytes + off, 16, 1024),
-                               smem_desc_sw128(k_addr + st * kTileBytes + off, 16, 1024), id_qk,
-                               k > 0);
+                for (int h = 0; h < 2; ++h) {
+                    const int j = jh[h];
+                    if (j >= n_kv) continue;
+                    const int st = j % kPfStages;
+                    const uint32_t par = (j / kPfStages) & 1;
+                    if (want_qk[h]) {
+                        if ((j > 0 && !mbar_test(&o_done[h], (j - 1) & 1)) || !mbar_test(&k_full[st], par))
+                            continue;
+                        tc_fence_after();
+                        const uint32_t s_tmem = tmem + h * 128;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const uint32_t off = (k >> 2) * kHalfTileBytes + (k & 3) * 32;
+                            mma_ss(s_tmem, smem_desc_sw128(q_addr + h * kTileBytes + off, 16, 1024),
+                                   smem_desc_sw128(k_addr + st * kTileBytes + off, 16, 1024), id_qk,
+                                   k > 0);
+                        }
+                        mma_commit(&s_full[h]);
+                        want_qk[h] = false;
+                    } else {
+                        if (!mbar_test(&p_full[h], j & 1) || !mbar_test(&v_full[st], par)) continue;
+                        tc_fence_after();
+                        const uint32_t p_tmem = tmem + h * 128;
+                        const uint32_t o_tmem = tmem + 256 + h * 128;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(o_tmem, p_tmem + k * 8,
+                                   smem_desc_sw128(v_addr + st * kTileBytes + k * 2048, kHalfTileBytes, 1024),
+                                   id_pv, (j > 0 || k > 0) ? 1u : 0u);
+                        mma_commit(&o_done[h]);
+                        if (++pv_in_stage[st] == 2) {          // both heads are done with this stage
+                            pv_in_stage[st] = 0;
+                            mma_commit(&kv_empty[st]);
+                        }
+                        want_qk[h] = true;
+                        jh[h] = j + 1;
                     }
-                    mma_commit(&s_full[h]);
+                    progressed = true;
                 }
-                if (!ok || !(ok = mbar_wait(&v_full[st], par))) break;
-                for (int h = 0; h < 2 && ok; ++h) {
-                    if (!(ok = mbar_wait(&p_full[h], j & 1))) break;
-                    tc_fence_after();
-                    const uint32_t p_tmem = tmem + h * 128;
-                    const uint32_t o_tmem = tmem + 256 + h * 128;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_ts(o_tmem, p_tmem + k * 8,
-                               smem_desc_sw128(v_addr + st * kTileBytes + k * 2048, kHalfTileBytes, 1024),
-                               id_pv, (j > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(&o_done[h]);
+                if (progressed) {
+                    idle_since = clock64();
+                } else if (clock64() - idle_since <= DUO_WAIT_CYCLES) {
+                    __nanosleep(32);     // leave issue slots to the softmax warps
+                } else {
+                    record_status(-5 /* DUO_ERR_TIMEOUT */);
+                    ok = false;
                 }
-                mma_commit(&kv_empty[st]);
             }
         }
         __syncwarp();  // lanes 1..31 wait for the MMA lane before the CTA barrier
@@ -238,15 +264,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
             reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
             const int c0 = tl.at(j) * kPfN;
-            if (!tile_dense(kind, t * kPfM, c0, a.sink, a.recent, a.window)) {
+            const bool dense = tile_dense(kind, t * kPfM, c0, a.sink, a.recent, a.window);
+            if (!dense) {
 #pragma unroll
                 for (int cc = 0; cc < 128; ++cc)
                     if (!key_attended(kind, i, c0 + cc, a.sink, a.recent, a.window))
                         sr[cc] = __float_as_uint(-INFINITY);
             }
-            float mx = -INFINITY;
+            float mx8[8];
 #pragma unroll
-            for (int cc = 0; cc < 128; ++cc) mx = fmaxf(mx, __uint_as_float(sr[cc]));
+            for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
+#pragma unroll
+            for (int cc = 8; cc < 128; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(sr[cc]));
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float m_tile = mx * c;               // scale > 0 keeps the order
             // keep the stale max unless the new one is more than 2^8 larger
             float m_use = m_run, alpha = 1.f;
@@ -257,18 +288,35 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
             float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
             uint32_t pw[64];
+            if (dense) {
+                // one exponential in four on the FMA pipe, the rest on the MUFU
 #pragma unroll
-            for (int cc = 0; cc < 128; cc += 4) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
-                const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
-                const float p3 = ex2_approx(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
-                ls0 += p0;
-                ls1 += p1;
-                ls2 += p2;
-                ls3 += p3;
-                pw[cc / 2] = pack_bf16x2(p0, p1);
-                pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                for (int cc = 0; cc < 128; cc += 4) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
+                    const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
+                    const float p3 = exp2_poly(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
+                    ls0 += p0;
+                    ls1 += p1;
+                    ls2 += p2;
+                    ls3 += p3;
+                    pw[cc / 2] = pack_bf16x2(p0, p1);
+                    pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                }
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < 128; cc += 4) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
+                    const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
+                    const float p3 = ex2_approx(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
+                    ls0 += p0;
+                    ls1 += p1;
+                    ls2 += p2;
+                    ls3 += p3;
+                    pw[cc / 2] = pack_bf16x2(p0, p1);
+                    pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                }
             }
             l_run = l_run * alpha + ((ls0 + ls1) + (ls2 + ls3));
             m_run = m_use;
