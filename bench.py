@@ -283,7 +283,7 @@ class Stack40:
             rows = B * (p.n_full * n + p.n_ring * min(n, span))
             self.bytes += rows * 512 + 2 * q.numel() * 2
             max_ws = max(max_ws, duo.duo_decode_workspace_bytes(p, n))
-        self.ws = torch.empty((max_ws + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+        self.ws = torch.zeros((max_ws + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
         self.launches_per_step = 2 * len(self.layers)
         self.unit = "GB/s"
         self.kernel = "40 x (decode_split + decode_merge), one CUDA graph"
@@ -401,7 +401,43 @@ class Prefill:
                 "window": self.w.window, "full_mask": list(self.w.full_mask)}
 
 
-WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40,
+class DecodeSmall:
+    """B=1: a 1024-token prompt is prefilled and appended, then each step
+    appends one token and decodes it (full heads {0,3,5,6}).  Latency-bound:
+    reported in microseconds per step."""
+
+    def __init__(self, rank: int):
+        w = self.w = inputs.workload("decode_small")
+        seed = rank_seed(w.seed, rank)
+        self.params = duo.DuoParams(1, 48, 8, 128, inputs.SINK, inputs.RECENT, 0, 128 ** -0.5,
+                                    w.full_mask, None)
+        self.cap = w.seq_len + 4096
+        self.cache = duo.DuoCache.allocate(self.params, self.cap)
+        q = inputs.randn_bf16((1, w.seq_len, 48, 128), seed, "cuda")
+        k = inputs.randn_bf16((1, w.seq_len, 8, 128), seed + 1, "cuda")
+        v = inputs.randn_bf16((1, w.seq_len, 8, 128), seed + 2, "cuda")
+        out = torch.empty_like(q)
+        duo.duo_attn_prefill(self.params, q, k, v, out, None)
+        duo.duo_kv_append(self.params, self.cache, k, v)
+        self.k1 = inputs.randn_bf16((1, 1, 8, 128), seed + 3, "cuda")
+        self.v1 = inputs.randn_bf16((1, 1, 8, 128), seed + 4, "cuda")
+        self.q1 = inputs.randn_bf16((1, 48, 128), seed + 5, "cuda")
+        self.out = torch.empty((1, 48, 128), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty((1, 48), dtype=torch.float32, device="cuda")
+        self.ws = duo.workspace_for(self.params, self.cap)
+        self.launches_per_step = 4      # append scatter + commit, decode split + merge
+        self.unit = "us/step"
+        self.kernel = "kv_append_scatter + kv_append_commit + decode_split + decode_merge"
+
+    def step(self):
+        duo.duo_kv_append(self.params, self.cache, self.k1, self.v1)
+        duo.duo_attn_decode(self.params, self.cache, self.q1, self.cap, self.out, self.lse, self.ws)
+
+    def config(self):
+        return {"workload": "decode_small: B=1, 1024-token prompt, then append one token + decode per step"}
+
+
+WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40, "decode_small": DecodeSmall,
              "prefill_16k": lambda rank: Prefill(rank, "prefill_16k"),
              "sliding_32k": lambda rank: Prefill(rank, "sliding_32k")}
 
@@ -440,6 +476,33 @@ def measure(wl, steps, warmup, world):
     return t / steps, clk.summary()
 
 
+CSRC = os.path.join(ROOT, "kv_cache_reduction_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu capture, or None once the
+    kernel's sources differ from the ones that were profiled."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("decode.cuh", "ptx.cuh", "kv_append.cuh"):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    digest = h.hexdigest()[:16]
+    try:
+        with open(TRAFFIC_FILE) as fh:
+            for line in fh:
+                if line.startswith("#") or not line.strip():
+                    continue
+                kv = dict(tok.split("=", 1) for tok in line.split())
+                if kv.get("kernel") == kernel and kv.get("workload") == workload and \
+                        kv.get("sources") == digest:
+                    return int(kv["dram_bytes_per_launch"])
+    except OSError:
+        pass
+    return None
+
+
 def roofline(wl, per_step, pk, pk_kind):
     if wl.unit == "GB/s":
         achieved = wl.bytes / per_step / 1e9
@@ -463,6 +526,9 @@ def run_ours(args, world, rank):
     value = aggregate(units(wl), world, per_step)
     rf = roofline(wl, per_step, pk, pk_kind)
     rf["kernel"] = wl.kernel
+    if args.workload == "decode_b32":
+        rf["traffic"] = measured_traffic("decode_split", "decode_b32")
+        rf["traffic_unit"] = "bytes per launch (ncu dram read + write)"
     res = {"metric": METRIC, "value": round(value, 2), "unit": wl.unit, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 4),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -487,15 +553,20 @@ def run_ours(args, world, rank):
         del wl
         torch.cuda.empty_cache()
         sec = {}
-        for name in ("stack40", "prefill_16k", "sliding_32k"):
+        for name in ("stack40", "prefill_16k", "sliding_32k", "decode_small"):
             w2 = WORKLOADS[name](rank)
             st = max(3, min(args.steps, 10))
             ps, ck = measure(w2, st, args.warmup, world)
-            r2 = roofline(w2, ps, pk, pk_kind)
-            sec[name] = {"value": round(aggregate(units(w2), world, ps), 2), "unit": w2.unit,
-                         "ms_per_step": round(ps * 1e3, 4), "steps": st, "frac": r2["frac"],
-                         "bound": r2["bound"], "kernel": w2.kernel,
-                         "gpu_launches": w2.launches_per_step * st, "clocks": ck}
+            if w2.unit == "us/step":
+                sec[name] = {"value": round(ps * 1e6, 2), "unit": "us/step", "higher_is_better": False,
+                             "steps": st, "kernel": w2.kernel,
+                             "gpu_launches": w2.launches_per_step * st, "clocks": ck}
+            else:
+                r2 = roofline(w2, ps, pk, pk_kind)
+                sec[name] = {"value": round(aggregate(units(w2), world, ps), 2), "unit": w2.unit,
+                             "ms_per_step": round(ps * 1e3, 4), "steps": st, "frac": r2["frac"],
+                             "bound": r2["bound"], "kernel": w2.kernel,
+                             "gpu_launches": w2.launches_per_step * st, "clocks": ck}
             del w2
             torch.cuda.empty_cache()
         res["secondary"] = sec
@@ -533,7 +604,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b32")
+    ap.add_argument("--workload", choices=sorted(k for k in WORKLOADS if k != "decode_small"),
+                    default="decode_b32")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--secondary", action=argparse.BooleanOptionalAction, default=True,

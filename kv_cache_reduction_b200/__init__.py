@@ -242,6 +242,7 @@ def duo_last_error() -> str:
 
 
 def workspace_for(params: DuoParams, max_seq_len: int, device="cuda") -> torch.Tensor:
-    """Allocates a decode workspace of the size the library asks for (torch memory)."""
+    """Allocates a zero-filled decode workspace of the size the library asks for
+    (torch memory).  It may be reused by any later call that fits in it."""
     n = max(duo_decode_workspace_bytes(params, max_seq_len), 256)
-    return torch.empty((n + 255) // 256 * 256, dtype=torch.uint8, device=device)
+    return torch.zeros((n + 255) // 256 * 256, dtype=torch.uint8, device=device)

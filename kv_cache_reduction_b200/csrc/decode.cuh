@@ -461,6 +461,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
     }
     tc_fence_before();
     __syncthreads();
+    // this CTA's partials are written: the merge grid may start launching
+    // (it still waits for the whole grid before reading them)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (warp == 5) {
         tc_fence_after();
         tmem_dealloc(tmem, kDecTmemCols);
@@ -470,6 +473,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
 // Folds the splits of every (sequence, query head) and the sink logit:
 // O = sum_s 2^(m_s - M) acc_s / (sum_s 2^(m_s - M) l_s + 2^(sigma*log2e - M)).
 __global__ void __launch_bounds__(kD) decode_merge(const __grid_constant__ DecodeArgs a) {
+    // launched as a programmatic dependent of decode_split: wait until that
+    // grid has completed and its partials are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int bh = blockIdx.x;
     const int b = bh / (a.hkv * kGroup);
     const int h = bh % (a.hkv * kGroup);

@@ -352,7 +352,20 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
         duo::decode_split<<<(unsigned)d.grid, duo::kDecThreads, duo::kDecSmem, st>>>(a);
         if ((rc = launch_status("decode_split"))) return rc;
     }
-    duo::decode_merge<<<(unsigned)((int64_t)params->batch * params->num_q_heads), duo::kD, 0, st>>>(a);
+    // the merge is a programmatic dependent launch: it is scheduled while
+    // decode_split drains and waits on the device for its results
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((int64_t)params->batch * params->num_q_heads));
+    cfg.blockDim = dim3(duo::kD);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, duo::decode_merge, a) != cudaSuccess)
+        return fail(DUO_ERR_CUDA, "decode_merge launch: %s", cudaGetErrorString(cudaGetLastError()));
     return launch_status("decode_merge");
 }
 

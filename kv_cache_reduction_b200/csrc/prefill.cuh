@@ -7,19 +7,25 @@
 // An optional per-query-head sink logit (Laguna XS 2.1 article, attention
 // sinks) joins the softmax denominator with a zero value vector.
 //
-// One CTA computes a 128-row query tile for two query heads of the same GQA
-// group, so both heads share every K/V tile in shared memory:
-//   warp 0     TMA producer: Q of both heads once, then K and V tiles into
+// A CTA computes 128-row query tiles for two query heads of one GQA group,
+// so both heads share every K/V tile in shared memory.  CTAs are persistent
+// (one per SM) and walk a static list of (sequence, head pair, query tile)
+// work tiles, heaviest query tiles first.  Keys come in 128-key tiles.
+//   warps 0-3  softmax of head 0, warps 4-7 softmax of head 1: thread r owns
+//              query row r; reads S from TMEM, writes P (bf16) back over the
+//              first 64 columns of S, rescales O in TMEM only when the running
+//              max grew by more than 2^8, and writes O / l and the log-sum-exp
+//              at the end of each work tile
+//   warp 8     TMA producer: Q of both heads per work tile, K and V tiles into
 //              a two-stage ring (128-byte swizzled, no multicast)
-//   warp 1     TMEM allocator and MMA issuer (one thread):
-//              S_h = Q_h K^T  (tcgen05.mma, both operands in shared memory)
-//              O_h += P_h V   (tcgen05.mma, P_h read from tensor memory)
-//   warps 4-7  softmax of head 0, warps 8-11 softmax of head 1: thread r
-//              owns query row r, reads S from TMEM, writes P (bf16) back
-//              over S, rescales O in TMEM only when the running max grew by
-//              more than 2^8, and writes O / l and the log-sum-exp at the end.
+//   warp 9     TMEM allocator and MMA issuer (one thread), in the order
+//                PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ...
+//              with S_h = Q_h K^T (both operands in shared memory) and
+//              O_h += P_h V (P_h read from tensor memory).  S_h(j+1) overwrites
+//              the columns PV_h(j) reads; the tcgen05 MMAs of one thread execute
+//              in issue order, so it is issued right behind it without a wait.
 // TMEM: S0 | S1 | O0 | O1, 128 fp32 columns each (512 in total).  Key tiles
-// that no row of the query tile attends to are never loaded.
+// that no row of a query tile attends to are never loaded.
 #pragma once
 
 #include <cuda.h>
@@ -30,11 +36,14 @@ namespace duo {
 
 constexpr int kPfM = 128;                  // query rows per tile
 constexpr int kPfN = 128;                  // keys per tile
-constexpr int kPfThreads = 384;            // 12 warps
+constexpr int kPfThreads = 320;            // 10 warps
 constexpr int kPfStages = 2;
-constexpr uint32_t kTileBytes = kPfM * 128 * 2;      // 128 rows x 128 bf16 = 32 KB
-constexpr uint32_t kHalfTileBytes = kTileBytes / 2;  // one 64-column swizzled box
-constexpr size_t kPfSmem = 2 * kTileBytes + 2 * kPfStages * kTileBytes + 1024;
+constexpr uint32_t kQTileBytes = kPfM * 128 * 2;     // 32 KB: one head's Q tile
+constexpr uint32_t kQHalfBytes = kQTileBytes / 2;    // 64-column swizzled box
+constexpr uint32_t kKVTileBytes = kPfN * 128 * 2;    // 32 KB: one K or V tile
+constexpr uint32_t kKVHalfBytes = kKVTileBytes / 2;
+constexpr uint32_t kPfStageBytes = 2 * kKVTileBytes;
+constexpr size_t kPfSmem = 1024 + 2 * kQTileBytes + kPfStages * kPfStageBytes;
 
 enum : int { kKindFull = 0, kKindStreaming = 1, kKindSliding = 2 };
 
@@ -45,22 +54,23 @@ struct PrefillArgs {
     __nv_bfloat16 *out;    // [B][L][Hq][128]
     float *lse;            // [B][Hq][L] or null
     const float *sink_logit;
-    int32_t L, hq, hkv, n_qtiles;
+    int32_t L, hq, hkv, n_qtiles, n_work, batch_pairs;
     int32_t sink, recent, window;
     float scale_log2;
     int8_t kind[64];       // per KV head
 };
 
 // Key tiles of query tile t for one head kind: an optional run of sink
-// tiles [0, n_sink_tiles) followed by the band [band_lo, t].
+// tiles [0, n_sink_tiles) followed by the band [band_lo, last].
 struct TileList {
-    int n_sink_tiles, band_lo, t;
-    __device__ int count() const { return n_sink_tiles + (t - band_lo + 1); }
+    int n_sink_tiles, band_lo, last;
+    __device__ int count() const { return n_sink_tiles + (last - band_lo + 1); }
     __device__ int at(int j) const { return j < n_sink_tiles ? j : band_lo + (j - n_sink_tiles); }
 };
 
-__device__ __forceinline__ TileList tile_list(int kind, int t, int sink, int recent, int window) {
-    TileList tl{0, 0, t};
+__device__ __forceinline__ TileList tile_list(int kind, int t, int L, int sink, int recent, int window) {
+    // keys past the last query of the tile, or past the sequence, are never attended
+    TileList tl{0, 0, min((t * kPfM + kPfM - 1) / kPfN, (L - 1) / kPfN)};
     if (kind == kKindFull) return tl;
     const int span = kind == kKindStreaming ? recent : window;
     const int first = t * kPfM - span + 1;           // lowest key of the band (row t*128)
@@ -89,33 +99,38 @@ __device__ __forceinline__ bool tile_dense(int kind, int r0, int c0, int sink, i
     return c0 > r1 - window;
 }
 
+// Work tile w: query tile t (heaviest first) of head pair p of sequence b.
+struct PfWork {
+    int b, h0, g, t;
+};
+
+__device__ __forceinline__ PfWork work_of(const PrefillArgs &a, int w) {
+    const int pairs = a.hq / 2;
+    const int per_t = a.batch_pairs;
+    PfWork wk;
+    wk.t = a.n_qtiles - 1 - w / per_t;
+    const int bp = w % per_t;
+    wk.b = bp / pairs;
+    wk.h0 = (bp % pairs) * 2;
+    wk.g = wk.h0 / (a.hq / a.hkv);
+    return wk;
+}
+
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_constant__ PrefillArgs a) {
-    extern __shared__ __align__(1024) char psmem_raw[];
-    char *smem = (char *)(((uintptr_t)psmem_raw + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(16) char psmem_base[];
+    char *smem = psmem_base + ((1024u - (smem_u32(psmem_base) & 1023u)) & 1023u);
     char *sQ = smem;                                   // [2 heads][32 KB]
-    char *sK = smem + 2 * kTileBytes;                  // [stages][32 KB]
-    char *sV = sK + kPfStages * kTileBytes;            // [stages][32 KB]
-    __shared__ uint64_t q_full, k_full[kPfStages], v_full[kPfStages], kv_empty[kPfStages];
+    char *sKV = smem + 2 * kQTileBytes;                // [stages][K 32 KB | V 32 KB]
+    __shared__ uint64_t q_full, q_empty, kv_full[kPfStages], kv_empty[kPfStages];
     __shared__ uint64_t s_full[2], p_full[2], o_done[2];
     __shared__ uint32_t tmem_base;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // work tile: x = (b, g, head pair), y = query tile, heaviest tiles first
-    const int pairs = a.hq / 2;
-    const int bgp = blockIdx.x;
-    const int b = bgp / pairs;
-    const int h0 = (bgp % pairs) * 2;
-    const int g = h0 / (a.hq / a.hkv);
-    const int t = a.n_qtiles - 1 - (int)blockIdx.y;
-    const int kind = a.kind[g];
-    const TileList tl = tile_list(kind, t, a.sink, a.recent, a.window);
-    const int n_kv = tl.count();
-
     if (threadIdx.x == 0) {
         mbar_init(&q_full, 1);
+        mbar_init(&q_empty, 1);
         for (int s = 0; s < kPfStages; ++s) {
-            mbar_init(&k_full[s], 1);
-            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
         for (int h = 0; h < 2; ++h) {
@@ -125,228 +140,233 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         }
         fence_mbar_init();
     }
-    __syncwarp();      // reconverge before the CTA barrier (bar.sync is warp-aligned)
-    if (warp == 1) {
+    if (warp == 9) {
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
+    __syncwarp();      // reconverge before the CTA barrier (bar.sync is warp-aligned)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
 
-    if (warp == 0) {
+    if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&a.tm_q);
             prefetch_tmap(&a.tm_k);
             prefetch_tmap(&a.tm_v);
-            mbar_expect_tx(&q_full, 2 * kTileBytes);
-            for (int h = 0; h < 2; ++h)
-                for (int half = 0; half < 2; ++half)
-                    tma_load_4d(sQ + h * kTileBytes + half * kHalfTileBytes, &a.tm_q, half * 64,
-                                h0 + h, t * kPfM, b, &q_full);
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % kPfStages;
-                if (j >= kPfStages && !mbar_wait(&kv_empty[st], ((j / kPfStages) - 1) & 1)) break;
-                const int row = tl.at(j) * kPfN;
-                mbar_expect_tx(&k_full[st], kTileBytes);
-                for (int half = 0; half < 2; ++half)
-                    tma_load_4d(sK + st * kTileBytes + half * kHalfTileBytes, &a.tm_k, half * 64, g,
-                                row, b, &k_full[st]);
-                mbar_expect_tx(&v_full[st], kTileBytes);
-                for (int half = 0; half < 2; ++half)
-                    tma_load_4d(sV + st * kTileBytes + half * kHalfTileBytes, &a.tm_v, half * 64, g,
-                                row, b, &v_full[st]);
+            int jg = 0, wc = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < a.n_work && ok; w += gridDim.x, ++wc) {
+                const PfWork wk = work_of(a, w);
+                const TileList tl = tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window);
+                // Q of the previous work tile must no longer be read by the MMA
+                if (wc > 0 && !(ok = mbar_wait(&q_empty, (wc - 1) & 1))) break;
+                mbar_expect_tx(&q_full, 2 * kQTileBytes);
+                for (int h = 0; h < 2; ++h)
+                    for (int half = 0; half < 2; ++half)
+                        tma_load_4d(sQ + h * kQTileBytes + half * kQHalfBytes, &a.tm_q, half * 64,
+                                    wk.h0 + h, wk.t * kPfM, wk.b, &q_full);
+                const int n_kv = tl.count();
+                for (int j = 0; j < n_kv; ++j, ++jg) {
+                    const int st = jg % kPfStages;
+                    if (jg >= kPfStages && !(ok = mbar_wait(&kv_empty[st], ((jg / kPfStages) - 1) & 1))) break;
+                    const int row = tl.at(j) * kPfN;
+                    char *kst = sKV + st * kPfStageBytes;
+                    mbar_expect_tx(&kv_full[st], kPfStageBytes);
+                    for (int half = 0; half < 2; ++half) {
+                        tma_load_4d(kst + half * kKVHalfBytes, &a.tm_k, half * 64, wk.g, row, wk.b, &kv_full[st]);
+                        tma_load_4d(kst + kKVTileBytes + half * kKVHalfBytes, &a.tm_v, half * 64, wk.g, row,
+                                    wk.b, &kv_full[st]);
+                    }
+                }
             }
         }
         __syncwarp();  // lanes 1..31 wait for the producer lane before the CTA barrier
-    } else if (warp == 1) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
-        // Each head alternates S_h = Q_h K_j^T and O_h += P_h V_j.  The two
-        // heads are polled independently, so one head's softmax never holds
-        // back the other head's next product.  S_h(j+1) overwrites P_h(j),
-        // so it waits for P_h(j) V_j to complete.
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(kPfM, kPfN, 0, 0);
             const uint32_t id_pv = idesc_bf16_f32(kPfM, 128, 0, 1);
-            const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-            bool ok = mbar_wait(&q_full, 0);
-            tc_fence_after();
-            int jh[2] = {0, 0};              // next key tile of each head
-            bool want_qk[2] = {true, true};  // next product of each head is S (else PV)
-            int pv_in_stage[kPfStages] = {};
-            unsigned long long idle_since = clock64();
-            while (ok && (jh[0] < n_kv || jh[1] < n_kv)) {
-                bool progressed = false;
+            const uint32_t q_addr = smem_u32(sQ), kv_addr = smem_u32(sKV);
+            auto issue_qk = [&](int h, int st) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int j = jh[h];
-                    if (j >= n_kv) continue;
-                    const int st = j % kPfStages;
-                    const uint32_t par = (j / kPfStages) & 1;
-                    if (want_qk[h]) {
-                        if ((j > 0 && !mbar_test(&o_done[h], (j - 1) & 1)) || !mbar_test(&k_full[st], par))
-                            continue;
-                        tc_fence_after();
-                        const uint32_t s_tmem = tmem + h * 128;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const uint32_t off = (k >> 2) * kHalfTileBytes + (k & 3) * 32;
-                            mma_ss(s_tmem, smem_desc_sw128(q_addr + h * kTileBytes + off, 16, 1024),
-                                   smem_desc_sw128(k_addr + st * kTileBytes + off, 16, 1024), id_qk,
-                                   k > 0);
-                        }
-                        mma_commit(&s_full[h]);
-                        want_qk[h] = false;
-                    } else {
-                        if (!mbar_test(&p_full[h], j & 1) || !mbar_test(&v_full[st], par)) continue;
-                        tc_fence_after();
-                        const uint32_t p_tmem = tmem + h * 128;
-                        const uint32_t o_tmem = tmem + 256 + h * 128;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            mma_ts(o_tmem, p_tmem + k * 8,
-                                   smem_desc_sw128(v_addr + st * kTileBytes + k * 2048, kHalfTileBytes, 1024),
-                                   id_pv, (j > 0 || k > 0) ? 1u : 0u);
-                        mma_commit(&o_done[h]);
-                        if (++pv_in_stage[st] == 2) {          // both heads are done with this stage
-                            pv_in_stage[st] = 0;
-                            mma_commit(&kv_empty[st]);
-                        }
-                        want_qk[h] = true;
-                        jh[h] = j + 1;
-                    }
-                    progressed = true;
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t qoff = h * kQTileBytes + (k >> 2) * kQHalfBytes + (k & 3) * 32;
+                    const uint32_t koff = st * kPfStageBytes + (k >> 2) * kKVHalfBytes + (k & 3) * 32;
+                    mma_ss(tmem + h * 128, smem_desc_sw128(q_addr + qoff, 16, 1024),
+                           smem_desc_sw128(kv_addr + koff, 16, 1024), id_qk, k > 0);
                 }
-                if (progressed) {
-                    idle_since = clock64();
-                } else if (clock64() - idle_since <= DUO_WAIT_CYCLES) {
-                    __nanosleep(32);     // leave issue slots to the softmax warps
-                } else {
-                    record_status(-5 /* DUO_ERR_TIMEOUT */);
-                    ok = false;
+                mma_commit(&s_full[h]);
+            };
+            auto issue_pv = [&](int h, int st, bool first) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tmem + 256 + h * 128, tmem + h * 128 + k * 8,
+                           smem_desc_sw128(kv_addr + st * kPfStageBytes + kKVTileBytes + k * 2048,
+                                           kKVHalfBytes, 1024),
+                           id_pv, (first && k == 0) ? 0u : 1u);
+                mma_commit(&o_done[h]);
+            };
+            int jg = 0, wc = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < a.n_work && ok; w += gridDim.x, ++wc) {
+                const PfWork wk = work_of(a, w);
+                const TileList tl = tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window);
+                const int n_kv = tl.count();
+                if (!(ok = mbar_wait(&q_full, wc & 1))) break;
+                if (!(ok = mbar_wait(&kv_full[jg % kPfStages], (jg / kPfStages) & 1))) break;
+                tc_fence_after();
+                issue_qk(0, jg % kPfStages);
+                issue_qk(1, jg % kPfStages);
+                if (n_kv == 1) mma_commit(&q_empty);
+                for (int j = 0; j < n_kv && ok; ++j, ++jg) {
+                    const int st = jg % kPfStages;
+                    const bool more = j + 1 < n_kv;
+                    const int st1 = (jg + 1) % kPfStages;
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        if (!(ok = mbar_wait(&p_full[h], jg & 1))) break;
+                        tc_fence_after();
+                        issue_pv(h, st, j == 0);
+                        if (more) {
+                            if (h == 0 && !(ok = mbar_wait(&kv_full[st1], ((jg + 1) / kPfStages) & 1))) break;
+                            tc_fence_after();
+                            issue_qk(h, st1);
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit(&kv_empty[st]);
+                    if (j + 2 == n_kv) mma_commit(&q_empty);   // the work tile's last S products are issued
                 }
             }
         }
         __syncwarp();  // lanes 1..31 wait for the MMA lane before the CTA barrier
-    } else if (warp >= 4) {
+    } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int h = (warp - 4) >> 2;                 // 0 or 1
+        const int h = warp >> 2;                       // 0 or 1
         const int quarter = warp & 3;                  // TMEM lane quarter of this warp
         const int r = quarter * 32 + lane;             // query row within the tile
-        const int i = t * kPfM + r;                    // query position
-        const int hq = h0 + h;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t s_tmem = tmem + h * 128 + lane_base;
         const uint32_t o_tmem = tmem + 256 + h * 128 + lane_base;
         const float c = a.scale_log2;
-        // running max (log2 units) and sum; a sink logit starts them at (sigma, 1)
-        float m_run = -INFINITY, l_run = 0.f;
-        if (a.sink_logit != nullptr) {
-            m_run = a.sink_logit[hq] * kLog2eF;
-            l_run = 1.f;
-        }
+        int jg = 0;
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            const bool got = mbar_wait(&s_full[h], j & 1);
-            __syncwarp();      // tcgen05.ld below is warp-collective
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t sr[128];
-            tmem_ld32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_ld32(s_tmem + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-            tmem_ld32(s_tmem + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-            tmem_ld_wait();
-            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-            const int c0 = tl.at(j) * kPfN;
-            const bool dense = tile_dense(kind, t * kPfM, c0, a.sink, a.recent, a.window);
-            if (!dense) {
-#pragma unroll
-                for (int cc = 0; cc < 128; ++cc)
-                    if (!key_attended(kind, i, c0 + cc, a.sink, a.recent, a.window))
-                        sr[cc] = __float_as_uint(-INFINITY);
+        for (int w = blockIdx.x; w < a.n_work && ok; w += gridDim.x) {
+            const PfWork wk = work_of(a, w);
+            const int kind = a.kind[wk.g];
+            const TileList tl = tile_list(kind, wk.t, a.L, a.sink, a.recent, a.window);
+            const int n_kv = tl.count();
+            const int i = wk.t * kPfM + r;             // query position
+            const int hq = wk.h0 + h;
+            // running max (log2 units) and sum; a sink logit starts them at (sigma, 1)
+            float m_run = -INFINITY, l_run = 0.f;
+            if (a.sink_logit != nullptr) {
+                m_run = a.sink_logit[hq] * kLog2eF;
+                l_run = 1.f;
             }
-            float mx8[8];
+            for (int j = 0; j < n_kv; ++j, ++jg) {
+                const bool got = mbar_wait(&s_full[h], jg & 1);
+                __syncwarp();      // tcgen05.ld below is warp-collective
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sr[128];
+                tmem_ld32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_ld32(s_tmem + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+                tmem_ld32(s_tmem + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+                tmem_ld_wait();
+                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+                const int c0 = tl.at(j) * kPfN;
+                const bool dense = tile_dense(kind, wk.t * kPfM, c0, a.sink, a.recent, a.window);
+                if (!dense) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
-#pragma unroll
-            for (int cc = 8; cc < 128; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(sr[cc]));
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            const float m_tile = mx * c;               // scale > 0 keeps the order
-            // keep the stale max unless the new one is more than 2^8 larger
-            float m_use = m_run, alpha = 1.f;
-            if (m_tile > m_run + 8.f) {
-                m_use = m_tile;
-                alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_tile);
-            }
-            const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-            float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
-            uint32_t pw[64];
-            if (dense) {
-                // one exponential in four on the FMA pipe, the rest on the MUFU
-#pragma unroll
-                for (int cc = 0; cc < 128; cc += 4) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
-                    const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
-                    const float p3 = exp2_poly(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
-                    ls0 += p0;
-                    ls1 += p1;
-                    ls2 += p2;
-                    ls3 += p3;
-                    pw[cc / 2] = pack_bf16x2(p0, p1);
-                    pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                    for (int cc = 0; cc < kPfN; ++cc)
+                        if (!key_attended(kind, i, c0 + cc, a.sink, a.recent, a.window))
+                            sr[cc] = __float_as_uint(-INFINITY);
                 }
-            } else {
+                float mx8[8];
 #pragma unroll
-                for (int cc = 0; cc < 128; cc += 4) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
-                    const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
-                    const float p3 = ex2_approx(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
-                    ls0 += p0;
-                    ls1 += p1;
-                    ls2 += p2;
-                    ls3 += p3;
-                    pw[cc / 2] = pack_bf16x2(p0, p1);
-                    pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
+#pragma unroll
+                for (int cc = 8; cc < kPfN; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(sr[cc]));
+                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                const float m_tile = mx * c;           // scale > 0 keeps the order
+                // keep the stale max unless the new one is more than 2^8 larger
+                float m_use = m_run, alpha = 1.f;
+                if (m_tile > m_run + 8.f) {
+                    m_use = m_tile;
+                    alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_tile);
                 }
-            }
-            l_run = l_run * alpha + ((ls0 + ls1) + (ls2 + ls3));
-            m_run = m_use;
-            tmem_st32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
-            tmem_st32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
-            // O holds the previous tiles' sum (its PV is complete: this S was
-            // issued after it); rescale it when the max moved
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+                float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+                uint32_t pw[64];
+                if (dense) {
+                    // one exponential in four on the FMA pipe, the rest on the MUFU
 #pragma unroll
-                for (int cb = 0; cb < 128; cb += 32) {
-                    uint32_t orr[32];
-                    tmem_ld32(o_tmem + cb, orr);
-                    tmem_ld_wait();
-                    reg_fence32(orr);
+                    for (int cc = 0; cc < kPfN; cc += 4) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
+                        const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
+                        const float p3 = exp2_poly(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
+                        ls0 += p0;
+                        ls1 += p1;
+                        ls2 += p2;
+                        ls3 += p3;
+                        pw[cc / 2] = pack_bf16x2(p0, p1);
+                        pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                    }
+                } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                    tmem_st32(o_tmem + cb, orr);
+                    for (int cc = 0; cc < kPfN; cc += 4) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
+                        const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
+                        const float p3 = ex2_approx(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
+                        ls0 += p0;
+                        ls1 += p1;
+                        ls2 += p2;
+                        ls3 += p3;
+                        pw[cc / 2] = pack_bf16x2(p0, p1);
+                        pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                    }
                 }
+                l_run = l_run * alpha + ((ls0 + ls1) + (ls2 + ls3));
+                m_run = m_use;
+                tmem_st32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
+                tmem_st32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
+                // O holds the previous key tiles' sum (its PV is complete: this S
+                // was computed after it); rescale it when the max moved
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                    for (int cb = 0; cb < 128; cb += 32) {
+                        uint32_t orr[32];
+                        tmem_ld32(o_tmem + cb, orr);
+                        tmem_ld_wait();
+                        reg_fence32(orr);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                        tmem_st32(o_tmem + cb, orr);
+                    }
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[h]);
             }
-            tmem_st_wait();
-            tc_fence_before();
+            if (!ok) break;
+            // ------------------------------------------------------------ work-tile epilogue
+            const bool o_fin = mbar_wait(&o_done[h], (jg - 1) & 1);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[h]);
-        }
-        // ------------------------------------------------------------ epilogue
-        const bool o_ready = ok && n_kv > 0 && mbar_wait(&o_done[h], (n_kv - 1) & 1);
-        if (__all_sync(0xffffffffu, o_ready)) {
+            if (!__all_sync(0xffffffffu, o_fin)) { ok = false; break; }
             tc_fence_after();
             const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-            __nv_bfloat16 *orow = a.out + (((size_t)b * a.L + i) * a.hq + hq) * 128;
+            __nv_bfloat16 *orow = a.out + (((size_t)wk.b * a.L + i) * a.hq + hq) * 128;
 #pragma unroll
             for (int cb = 0; cb < 128; cb += 32) {
                 uint32_t orr[32];
@@ -367,14 +387,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 }
             }
             if (a.lse != nullptr && i < a.L)
-                a.lse[((size_t)b * a.hq + hq) * a.L + i] =
+                a.lse[((size_t)wk.b * a.hq + hq) * a.L + i] =
                     l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2F : -INFINITY;
+            // O has been read: the first PV of the next work tile may overwrite it
+            tc_fence_before();
         }
         __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -399,13 +421,13 @@ inline EncodeTiledFn encode_fn() {
 }
 
 // [B][L][H][128] bf16 viewed as a 4-D tensor (128, H, L, B), loaded as
-// 64-column x 128-row boxes with the 128-byte swizzle.
-inline bool make_tmap(CUtensorMap *m, const void *base, int B, int L, int H) {
+// 64-column x `rows`-row boxes with the 128-byte swizzle.
+inline bool make_tmap(CUtensorMap *m, const void *base, int B, int L, int H, int rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
     const cuuint64_t strides[3] = {256, (cuuint64_t)H * 256, (cuuint64_t)L * H * 256};
-    const cuuint32_t box[4] = {64, 1, kPfM, 1};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
     const cuuint32_t elem[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
               elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -418,8 +440,9 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     PrefillArgs a;
     memset(&a, 0, sizeof a);
     const int B = p->batch;
-    if (!make_tmap(&a.tm_q, q, B, L, p->num_q_heads) || !make_tmap(&a.tm_k, k, B, L, p->num_kv_heads) ||
-        !make_tmap(&a.tm_v, v, B, L, p->num_kv_heads)) {
+    if (!make_tmap(&a.tm_q, q, B, L, p->num_q_heads, kPfM) ||
+        !make_tmap(&a.tm_k, k, B, L, p->num_kv_heads, kPfN) ||
+        !make_tmap(&a.tm_v, v, B, L, p->num_kv_heads, kPfN)) {
         snprintf(err, err_len, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
         return DUO_ERR_CUDA;
     }
@@ -447,11 +470,16 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
         }
         if (dev >= 0 && dev < 64) smem_set[dev] = true;
     }
-    if (a.n_qtiles > 65535) {
-        snprintf(err, err_len, "sequence too long for one prefill launch");
+    a.batch_pairs = B * (p->num_q_heads / 2);
+    const int64_t n_work = (int64_t)a.batch_pairs * a.n_qtiles;
+    if (n_work > INT32_MAX) {
+        snprintf(err, err_len, "too many query tiles for one prefill launch");
         return DUO_ERR_INVALID_ARG;
     }
-    const dim3 grid((unsigned)(B * (p->num_q_heads / 2)), (unsigned)a.n_qtiles);
+    a.n_work = (int32_t)n_work;
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const unsigned grid = (unsigned)std::min<int64_t>(n_work, sms);
     prefill_fwd<<<grid, kPfThreads, kPfSmem, stream>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {

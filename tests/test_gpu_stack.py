@@ -69,7 +69,7 @@ def test_stack40_graph_replay_matches_eager(cuda_device):
         state.append((p, cache, q, torch.empty((B, 48, 128), dtype=torch.bfloat16, device="cuda"),
                       torch.empty((B, 48), dtype=torch.float32, device="cuda")))
         max_ws = max(max_ws, duo.duo_decode_workspace_bytes(p, n))
-    ws = torch.empty(max_ws, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max_ws, dtype=torch.uint8, device="cuda")
 
     def step():
         for p, cache, q, out, lse in state:
