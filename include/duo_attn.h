@@ -167,6 +167,28 @@ DUO_API int duo_attn_decode(const duo_params *params, const duo_cache *cache, co
 DUO_API int duo_attn_decode_static(const duo_params *params, const duo_cache *cache, const void *q,
                                    int32_t max_seq_len, void *out, float *lse, void *stream);
 
+/* KV-cache accounting for one layer (host arithmetic only, no device access).
+ * The DuoAttention card (sections Benefits and Changes In This Submission)
+ * measures KV-cache size and active KV-cache utilisation of the static Duo
+ * cache; this gives those numbers for the layout above:
+ *   duo_bytes        = B * (n_full * capacity + n_ring * ring_slots) * D * 2 B * 2 (K and V)
+ *   full_cache_bytes = B * num_kv_heads * capacity * D * 2 B * 2 (every head keeps all tokens)
+ *   active_bytes     = bytes of duo_bytes that hold a valid token when every sequence
+ *                      holds seq_len tokens (full heads: min(seq_len, capacity) rows;
+ *                      ring heads: min(seq_len, ring_slots) slots)
+ *   utilization      = active_bytes / duo_bytes (0 when duo_bytes is 0)
+ * Returns DUO_OK, or DUO_ERR_INVALID_ARG for bad params, capacity < 0,
+ * seq_len < 0 or a NULL out. */
+typedef struct {
+    uint64_t duo_bytes;
+    uint64_t full_cache_bytes;
+    uint64_t active_bytes;
+    double utilization;
+} duo_cache_stats;
+
+DUO_API int duo_cache_bytes(const duo_params *params, int64_t capacity, int64_t seq_len,
+                            duo_cache_stats *out);
+
 /* Reads and clears the device status word of the current device after
  * synchronising `stream`: DUO_OK, DUO_ERR_TIMEOUT or DUO_ERR_CAPACITY (the
  * first error any kernel recorded since the last read), or DUO_ERR_CUDA. */

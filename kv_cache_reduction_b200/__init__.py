@@ -36,8 +36,8 @@ DUO_ERR_CAPACITY = -6
 DUO_ERR_DEVICE = -7
 
 EXPORTED = ("duo_kv_append", "duo_attn_prefill", "duo_decode_workspace_bytes", "duo_attn_decode",
-            "duo_attn_decode_static", "duo_get_device_status", "duo_status_string",
-            "duo_last_error")
+            "duo_attn_decode_static", "duo_cache_bytes", "duo_get_device_status",
+            "duo_status_string", "duo_last_error")
 
 
 class DuoLibraryMissing(RuntimeError):
@@ -56,6 +56,11 @@ class _Params(ctypes.Structure):
                 ("sink", ctypes.c_int32), ("recent", ctypes.c_int32),
                 ("window", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
                 ("full_mask", ctypes.c_void_p), ("sink_logit", ctypes.c_void_p)]
+
+
+class CacheStats(ctypes.Structure):
+    _fields_ = [("duo_bytes", ctypes.c_uint64), ("full_cache_bytes", ctypes.c_uint64),
+                ("active_bytes", ctypes.c_uint64), ("utilization", ctypes.c_double)]
 
 
 class _Cache(ctypes.Structure):
@@ -88,6 +93,8 @@ def load_library(path: str = LIBRARY_PATH) -> ctypes.CDLL:
     lib.duo_attn_decode.restype = ctypes.c_int
     lib.duo_attn_decode_static.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, vp]
     lib.duo_attn_decode_static.restype = ctypes.c_int
+    lib.duo_cache_bytes.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(CacheStats)]
+    lib.duo_cache_bytes.restype = ctypes.c_int
     lib.duo_get_device_status.argtypes = [vp]
     lib.duo_get_device_status.restype = ctypes.c_int
     lib.duo_status_string.argtypes = [ctypes.c_int]
@@ -227,6 +234,15 @@ def duo_attn_decode_static(params: DuoParams, cache: DuoCache, q: torch.Tensor, 
     _check(load_library().duo_attn_decode_static(ctypes.byref(p), ctypes.byref(c), _ptr(q),
                                                  int(max_seq_len), _ptr(out), _ptr(lse),
                                                  _stream(stream)))
+
+
+def duo_cache_bytes(params: DuoParams, capacity: int, seq_len: int) -> CacheStats:
+    """KV-cache size of a layer against a full cache, and its active utilisation
+    when every sequence holds seq_len tokens (host arithmetic)."""
+    p, st = params.as_c(), CacheStats()
+    _check(load_library().duo_cache_bytes(ctypes.byref(p), int(capacity), int(seq_len),
+                                          ctypes.byref(st)))
+    return st
 
 
 def duo_get_device_status(stream=None) -> int:

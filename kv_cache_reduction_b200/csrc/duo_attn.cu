@@ -384,6 +384,26 @@ int duo_attn_prefill(const duo_params *params, const void *q, const void *k, con
                                out, lse, (cudaStream_t)stream, g_err, sizeof g_err);
 }
 
+int duo_cache_bytes(const duo_params *params, int64_t capacity, int64_t seq_len,
+                    duo_cache_stats *out) {
+    Layout L;
+    const int rc = check_params(params, &L);
+    if (rc) return rc;
+    if (capacity < 0 || seq_len < 0 || !out)
+        return fail(DUO_ERR_INVALID_ARG, "need capacity >= 0, seq_len >= 0 and a non-NULL out");
+    const uint64_t row = (uint64_t)params->head_dim * 2u * 2u;   // K and V, bf16
+    const uint64_t B = (uint64_t)params->batch;
+    const uint64_t full_rows = (uint64_t)L.n_full * (uint64_t)capacity;
+    const uint64_t ring_rows = (uint64_t)L.n_ring * (uint64_t)L.slots;
+    out->duo_bytes = B * (full_rows + ring_rows) * row;
+    out->full_cache_bytes = B * (uint64_t)params->num_kv_heads * (uint64_t)capacity * row;
+    const uint64_t act_full = (uint64_t)L.n_full * (uint64_t)std::min(seq_len, capacity);
+    const uint64_t act_ring = (uint64_t)L.n_ring * (uint64_t)std::min<int64_t>(seq_len, L.slots);
+    out->active_bytes = B * (act_full + act_ring) * row;
+    out->utilization = out->duo_bytes ? (double)out->active_bytes / (double)out->duo_bytes : 0.0;
+    return DUO_OK;
+}
+
 int duo_get_device_status(void *stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
         return fail(DUO_ERR_CUDA, "stream synchronize failed: %s", cudaGetErrorString(cudaGetLastError()));
