@@ -11,14 +11,17 @@
 // so both heads share every K/V tile in shared memory.  CTAs are persistent
 // (one per SM) and walk a static list of (sequence, head pair, query tile)
 // work tiles, heaviest query tiles first.  Keys come in 128-key tiles.
-//   warps 0-3  softmax of head 0, warps 4-7 softmax of head 1: thread r owns
-//              query row r; reads S from TMEM, writes P (bf16) back over the
-//              first 64 columns of S, rescales O in TMEM only when the running
-//              max grew by more than 2^8, and writes O / l and the log-sum-exp
-//              at the end of each work tile
-//   warp 8     TMA producer: Q of both heads per work tile, K and V tiles into
+//   warps 0-7  softmax of head 0, warps 8-15 softmax of head 1: each query
+//              row is split over two warps (64 keys each, the row max joined
+//              through shared memory); they read S from TMEM, write P (bf16)
+//              back over the first 64 columns of S, rescale O in TMEM only when
+//              the running max grew by more than 2^8, and write O / l and the
+//              log-sum-exp at the end of each work tile.  The two heads take
+//              turns for the exponentials, so that the MUFU units serve one head
+//              while the tensor core runs the other head's PV and next S
+//   warp 16    TMA producer: Q of both heads per work tile, K and V tiles into
 //              a two-stage ring (128-byte swizzled, no multicast)
-//   warp 9     TMEM allocator and MMA issuer (one thread), in the order
+//   warp 17    TMEM allocator and MMA issuer (one thread), in the order
 //                PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ...
 //              with S_h = Q_h K^T (both operands in shared memory) and
 //              O_h += P_h V (P_h read from tensor memory).  S_h(j+1) overwrites
@@ -36,7 +39,7 @@ namespace duo {
 
 constexpr int kPfM = 128;                  // query rows per tile
 constexpr int kPfN = 128;                  // keys per tile
-constexpr int kPfThreads = 320;            // 10 warps
+constexpr int kPfThreads = 576;            // 18 warps
 constexpr int kPfStages = 2;
 constexpr uint32_t kQTileBytes = kPfM * 128 * 2;     // 32 KB: one head's Q tile
 constexpr uint32_t kQHalfBytes = kQTileBytes / 2;    // 64-column swizzled box
@@ -122,7 +125,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     char *sQ = smem;                                   // [2 heads][32 KB]
     char *sKV = smem + 2 * kQTileBytes;                // [stages][K 32 KB | V 32 KB]
     __shared__ uint64_t q_full, q_empty, kv_full[kPfStages], kv_empty[kPfStages];
-    __shared__ uint64_t s_full[2], p_full[2], o_done[2];
+    __shared__ uint64_t s_full[2], p_full[2], o_done[2], turn[2];
+    // row-half exchanges between the eight softmax warps of a head (bounded
+    // mbarrier waits, so that a timed-out warp cannot strand its partners)
+    __shared__ uint64_t xmax[2][2], xsum[2];           // [tile parity][head], [head]
+    __shared__ float red_max[2][2][2][kPfM];           // [tile parity][head][column half][row]
+    __shared__ float red_sum[2][2][kPfM];              // [head][column half][row]
     __shared__ uint32_t tmem_base;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -135,12 +143,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         }
         for (int h = 0; h < 2; ++h) {
             mbar_init(&s_full[h], 1);
-            mbar_init(&p_full[h], 4);
+            mbar_init(&p_full[h], 8);
             mbar_init(&o_done[h], 1);
+            mbar_init(&turn[h], 8);
+            mbar_init(&xmax[0][h], 8);
+            mbar_init(&xmax[1][h], 8);
+            mbar_init(&xsum[h], 8);
         }
+        for (int w8 = 0; w8 < 8; ++w8) mbar_arrive(&turn[0]);   // head 0 takes the first turn
         fence_mbar_init();
     }
-    if (warp == 9) {
+    if (warp == 17) {
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
@@ -150,7 +163,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     tc_fence_after();
     const uint32_t tmem = tmem_base;
 
-    if (warp == 8) {
+    if (warp == 16) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&a.tm_q);
@@ -184,7 +197,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             }
         }
         __syncwarp();  // lanes 1..31 wait for the producer lane before the CTA barrier
-    } else if (warp == 9) {
+    } else if (warp == 17) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(kPfM, kPfN, 0, 0);
@@ -244,59 +257,65 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         __syncwarp();  // lanes 1..31 wait for the MMA lane before the CTA barrier
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int h = warp >> 2;                       // 0 or 1
+        const int h = warp >> 3;                       // head of the pair
         const int quarter = warp & 3;                  // TMEM lane quarter of this warp
+        const int half = (warp >> 2) & 1;              // key columns [64*half, 64*half + 64)
         const int r = quarter * 32 + lane;             // query row within the tile
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t s_tmem = tmem + h * 128 + lane_base;
         const uint32_t o_tmem = tmem + 256 + h * 128 + lane_base;
         const float c = a.scale_log2;
-        int jg = 0;
+        int jg = 0, wc = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < a.n_work && ok; w += gridDim.x) {
+        for (int w = blockIdx.x; w < a.n_work && ok; w += gridDim.x, ++wc) {
             const PfWork wk = work_of(a, w);
             const int kind = a.kind[wk.g];
             const TileList tl = tile_list(kind, wk.t, a.L, a.sink, a.recent, a.window);
             const int n_kv = tl.count();
             const int i = wk.t * kPfM + r;             // query position
             const int hq = wk.h0 + h;
-            // running max (log2 units) and sum; a sink logit starts them at (sigma, 1)
+            // running max (log2 units) and this half's share of the sum; a sink
+            // logit starts them at (sigma, 1), counted once (in half 0)
             float m_run = -INFINITY, l_run = 0.f;
             if (a.sink_logit != nullptr) {
                 m_run = a.sink_logit[hq] * kLog2eF;
-                l_run = 1.f;
+                l_run = half == 0 ? 1.f : 0.f;
             }
             for (int j = 0; j < n_kv; ++j, ++jg) {
                 const bool got = mbar_wait(&s_full[h], jg & 1);
                 __syncwarp();      // tcgen05.ld below is warp-collective
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sr[128];
-                tmem_ld32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_ld32(s_tmem + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-                tmem_ld32(s_tmem + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+                uint32_t sr[64];
+                tmem_ld32(s_tmem + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(s_tmem + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                 tmem_ld_wait();
                 reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                 reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
                 const int c0 = tl.at(j) * kPfN;
                 const bool dense = tile_dense(kind, wk.t * kPfM, c0, a.sink, a.recent, a.window);
                 if (!dense) {
 #pragma unroll
-                    for (int cc = 0; cc < kPfN; ++cc)
-                        if (!key_attended(kind, i, c0 + cc, a.sink, a.recent, a.window))
+                    for (int cc = 0; cc < 64; ++cc)
+                        if (!key_attended(kind, i, c0 + half * 64 + cc, a.sink, a.recent, a.window))
                             sr[cc] = __float_as_uint(-INFINITY);
                 }
                 float mx8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
 #pragma unroll
-                for (int cc = 8; cc < kPfN; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(sr[cc]));
-                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-                const float m_tile = mx * c;           // scale > 0 keeps the order
+                for (int cc = 8; cc < 64; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(sr[cc]));
+                const float mx_half = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                            fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                // join the two halves of the row (both have read their S by now,
+                // so P may overwrite any of the first 64 columns afterwards)
+                red_max[jg & 1][h][half][r] = mx_half;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xmax[jg & 1][h]);
+                const bool joined = mbar_wait(&xmax[jg & 1][h], (jg >> 1) & 1);
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, joined)) { ok = false; break; }
+                const float m_tile = fmaxf(mx_half, red_max[jg & 1][h][half ^ 1][r]) * c;
                 // keep the stale max unless the new one is more than 2^8 larger
                 float m_use = m_run, alpha = 1.f;
                 if (m_tile > m_run + 8.f) {
@@ -304,26 +323,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_tile);
                 }
                 const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+                // this head's turn on the MUFU units
+                const bool my_turn = mbar_wait(&turn[h], jg & 1);
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, my_turn)) { ok = false; break; }
                 float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
-                uint32_t pw[64];
-                if (dense) {
-                    // one exponential in four on the FMA pipe, the rest on the MUFU
 #pragma unroll
-                    for (int cc = 0; cc < kPfN; cc += 4) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
-                        const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
-                        const float p3 = exp2_poly(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
-                        ls0 += p0;
-                        ls1 += p1;
-                        ls2 += p2;
-                        ls3 += p3;
-                        pw[cc / 2] = pack_bf16x2(p0, p1);
-                        pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
-                    }
-                } else {
+                for (int ch = 0; ch < 2; ++ch) {
+                    uint32_t pw[16];
 #pragma unroll
-                    for (int cc = 0; cc < kPfN; cc += 4) {
+                    for (int e = 0; e < 32; e += 4) {
+                        const int cc = ch * 32 + e;
                         const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
                         const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
                         const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
@@ -332,26 +342,29 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                         ls1 += p1;
                         ls2 += p2;
                         ls3 += p3;
-                        pw[cc / 2] = pack_bf16x2(p0, p1);
-                        pw[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                        pw[e / 2] = pack_bf16x2(p0, p1);
+                        pw[e / 2 + 1] = pack_bf16x2(p2, p3);
                     }
+                    // P of keys [64*half + 32*ch, +32) -> TMEM columns [32*half + 16*ch, +16)
+                    tmem_st16(s_tmem + half * 32 + ch * 16, pw);
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&turn[h ^ 1]);
                 l_run = l_run * alpha + ((ls0 + ls1) + (ls2 + ls3));
                 m_run = m_use;
-                tmem_st32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
-                tmem_st32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
                 // O holds the previous key tiles' sum (its PV is complete: this S
-                // was computed after it); rescale it when the max moved
+                // was computed after it); rescale this half's 64 columns when the
+                // max moved
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                    for (int cb = 0; cb < 128; cb += 32) {
+                    for (int cb = 0; cb < 64; cb += 32) {
                         uint32_t orr[32];
-                        tmem_ld32(o_tmem + cb, orr);
+                        tmem_ld32(o_tmem + half * 64 + cb, orr);
                         tmem_ld_wait();
                         reg_fence32(orr);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                        tmem_st32(o_tmem + cb, orr);
+                        tmem_st32(o_tmem + half * 64 + cb, orr);
                     }
                 }
                 tmem_st_wait();
@@ -361,16 +374,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             }
             if (!ok) break;
             // ------------------------------------------------------------ work-tile epilogue
-            const bool o_fin = mbar_wait(&o_done[h], (jg - 1) & 1);
+            red_sum[h][half][r] = l_run;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xsum[h]);
+            const bool o_fin = mbar_wait(&o_done[h], (jg - 1) & 1) && mbar_wait(&xsum[h], wc & 1);
             __syncwarp();
             if (!__all_sync(0xffffffffu, o_fin)) { ok = false; break; }
             tc_fence_after();
-            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-            __nv_bfloat16 *orow = a.out + (((size_t)wk.b * a.L + i) * a.hq + hq) * 128;
+            const float l_row = red_sum[h][0][r] + red_sum[h][1][r];
+            const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+            __nv_bfloat16 *orow = a.out + (((size_t)wk.b * a.L + i) * a.hq + hq) * 128 + half * 64;
 #pragma unroll
-            for (int cb = 0; cb < 128; cb += 32) {
+            for (int cb = 0; cb < 64; cb += 32) {
                 uint32_t orr[32];
-                tmem_ld32(o_tmem + cb, orr);
+                tmem_ld32(o_tmem + half * 64 + cb, orr);
                 tmem_ld_wait();
                 reg_fence32(orr);
                 if (i < a.L) {
@@ -386,17 +403,19 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     }
                 }
             }
-            if (a.lse != nullptr && i < a.L)
+            if (a.lse != nullptr && i < a.L && half == 0)
                 a.lse[((size_t)wk.b * a.hq + hq) * a.L + i] =
-                    l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2F : -INFINITY;
-            // O has been read: the first PV of the next work tile may overwrite it
+                    l_row > 0.f ? (m_run + __log2f(l_row)) * kLn2F : -INFINITY;
+            // O is read before this warp's first p_full arrival of the next work
+            // tile, and red_sum before its next row-max exchange, so neither the
+            // next PV nor the next epilogue can overwrite them early
             tc_fence_before();
         }
         __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == 17) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

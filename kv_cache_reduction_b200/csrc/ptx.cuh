@@ -296,24 +296,6 @@ __device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
     return f2_from_bits(d);
 }
 
-// 2^x on the FMA pipe for x in [-125, 128): x = j + f with j the nearest
-// integer (Cody-Waite style split by adding 1.5 * 2^23) and f in
-// [-0.5, 0.5]; 2^f from a degree-3 Chebyshev least-squares fit (relative
-// error below 1.1e-4, kv_cache_reduction_b200/exp2_poly.py); 2^j is added
-// to the exponent field.
-constexpr float kExp2C0 = 0.99992448091506958f;
-constexpr float kExp2C1 = 0.69312101602554321f;
-constexpr float kExp2C2 = 0.24264007806777954f;
-constexpr float kExp2C3 = 0.05592203512787819f;
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.f);
-    const float t = x + 12582912.f;
-    const float j = t - 12582912.f;
-    const float f = x - j;
-    const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Packs two floats to bf16x2 (round to nearest even): lo -> bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
