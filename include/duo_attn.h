@@ -118,6 +118,10 @@ typedef struct {
 DUO_API int duo_kv_append(const duo_params *params, const duo_cache *cache, const void *k,
                   const void *v, int32_t n_new, void *stream);
 
+/* Bytes of device workspace duo_attn_prefill uses for dynamic work-tile
+ * scheduling (the same for every layer). */
+DUO_API size_t duo_prefill_workspace_bytes(void);
+
 /* Prefill attention over a sequence that starts at position 0 (empty cache).
  * q: device bf16 [B][L][Hq][D]; k, v: device bf16 [B][L][Hkv][D]; L = seq_len.
  * out: device bf16 [B][L][Hq][D].  lse: device fp32 [B][Hq][L] (natural-log
@@ -126,9 +130,17 @@ DUO_API int duo_kv_append(const duo_params *params, const duo_cache *cache, cons
  * j <= i; streaming: j < sink or i - recent < j <= i; sliding:
  * i - window < j <= i).  Computed with tcgen05 tensor cores (bf16 inputs,
  * fp32 accumulation, probabilities rounded to bf16 before the PV product).
+ * workspace: NULL, or device memory of at least duo_prefill_workspace_bytes()
+ * bytes, 16-byte aligned, owned by the caller; its contents need not be
+ * initialised (the call zeroes it on the stream).  With a workspace the
+ * persistent CTAs claim work tiles from a counter in it (balanced when the
+ * heads' costs differ); without one they take a fixed stride of the list.
+ * Calls that may run at the same time need separate workspaces.  A smaller
+ * or misaligned workspace returns DUO_ERR_WORKSPACE.
  * The cache is not touched: call duo_kv_append(n_new = L) to fill it. */
 DUO_API int duo_attn_prefill(const duo_params *params, const void *q, const void *k, const void *v,
-                     int32_t seq_len, void *out, float *lse, void *stream);
+                     int32_t seq_len, void *out, float *lse, void *workspace,
+                     size_t workspace_bytes, void *stream);
 
 /* Bytes of device workspace duo_attn_decode needs for this layer when no
  * sequence holds more than max_seq_len tokens.  Returns 0 on invalid params. */

@@ -35,7 +35,8 @@ DUO_ERR_TIMEOUT = -5
 DUO_ERR_CAPACITY = -6
 DUO_ERR_DEVICE = -7
 
-EXPORTED = ("duo_kv_append", "duo_attn_prefill", "duo_decode_workspace_bytes", "duo_attn_decode",
+EXPORTED = ("duo_kv_append", "duo_prefill_workspace_bytes", "duo_attn_prefill",
+            "duo_decode_workspace_bytes", "duo_attn_decode",
             "duo_attn_decode_static", "duo_cache_bytes", "duo_get_device_status",
             "duo_status_string", "duo_last_error")
 
@@ -85,7 +86,9 @@ def load_library(path: str = LIBRARY_PATH) -> ctypes.CDLL:
     P, C, vp = ctypes.POINTER(_Params), ctypes.POINTER(_Cache), ctypes.c_void_p
     lib.duo_kv_append.argtypes = [P, C, vp, vp, ctypes.c_int32, vp]
     lib.duo_kv_append.restype = ctypes.c_int
-    lib.duo_attn_prefill.argtypes = [P, vp, vp, vp, ctypes.c_int32, vp, vp, vp]
+    lib.duo_prefill_workspace_bytes.argtypes = []
+    lib.duo_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.duo_attn_prefill.argtypes = [P, vp, vp, vp, ctypes.c_int32, vp, vp, vp, ctypes.c_size_t, vp]
     lib.duo_attn_prefill.restype = ctypes.c_int
     lib.duo_decode_workspace_bytes.argtypes = [P, ctypes.c_int32]
     lib.duo_decode_workspace_bytes.restype = ctypes.c_size_t
@@ -201,13 +204,21 @@ def duo_kv_append(params: DuoParams, cache: DuoCache, k: torch.Tensor, v: torch.
                                         _stream(stream)))
 
 
+def duo_prefill_workspace_bytes() -> int:
+    return int(load_library().duo_prefill_workspace_bytes())
+
+
 def duo_attn_prefill(params: DuoParams, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                      out: torch.Tensor, lse: Optional[torch.Tensor] = None,
-                     seq_len: Optional[int] = None, stream=None) -> None:
+                     seq_len: Optional[int] = None, stream=None,
+                     workspace: Optional[torch.Tensor] = None) -> None:
+    """workspace: None (static work-tile order) or a device tensor of at least
+    duo_prefill_workspace_bytes() bytes (dynamic, balanced order)."""
     L = int(q.shape[1]) if seq_len is None else int(seq_len)
     p = params.as_c()
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load_library().duo_attn_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), L, _ptr(out),
-                                           _ptr(lse), _stream(stream)))
+                                           _ptr(lse), _ptr(workspace), nbytes, _stream(stream)))
 
 
 def duo_decode_workspace_bytes(params: DuoParams, max_seq_len: int) -> int:

@@ -31,6 +31,7 @@ constexpr int kMaxHkv = 64;
 constexpr int kMaxWindow = 8192;
 constexpr int kMaxRing = 8192;
 constexpr int64_t kMaxPos = (int64_t)1 << 30;
+constexpr size_t kPrefillWorkspaceBytes = 16;   // the prefill work-tile counter
 
 struct Layout {
     bool sliding;
@@ -369,11 +370,17 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     return launch_status("decode_merge");
 }
 
+size_t duo_prefill_workspace_bytes(void) { return kPrefillWorkspaceBytes; }
+
 int duo_attn_prefill(const duo_params *params, const void *q, const void *k, const void *v,
-                     int32_t seq_len, void *out, float *lse, void *stream) {
+                     int32_t seq_len, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                     void *stream) {
     Layout L;
     int rc = check_params(params, &L);
     if (rc) return rc;
+    if (workspace && (workspace_bytes < kPrefillWorkspaceBytes || !aligned16(workspace)))
+        return fail(DUO_ERR_WORKSPACE, "prefill workspace: need %zu bytes, 16-byte aligned (got %zu)",
+                    kPrefillWorkspaceBytes, workspace_bytes);
     if (seq_len < 0 || seq_len > kMaxPos) return fail(DUO_ERR_INVALID_ARG, "seq_len must be in [0, 2^30]");
     if (seq_len == 0) return DUO_OK;
     if (!q || !k || !v || !out) return fail(DUO_ERR_INVALID_ARG, "q / k / v / out is NULL");
@@ -381,7 +388,7 @@ int duo_attn_prefill(const duo_params *params, const void *q, const void *k, con
         return fail(DUO_ERR_INVALID_ARG, "q / k / v / out / lse must be 16-byte aligned");
     if ((rc = check_device(nullptr))) return rc;
     return duo::launch_prefill(params, L.sliding, L.heads.is_full, L.sink, L.ring, q, k, v, seq_len,
-                               out, lse, (cudaStream_t)stream, g_err, sizeof g_err);
+                               out, lse, (int32_t *)workspace, (cudaStream_t)stream, g_err, sizeof g_err);
 }
 
 int duo_cache_bytes(const duo_params *params, int64_t capacity, int64_t seq_len,

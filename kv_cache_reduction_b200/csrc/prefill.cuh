@@ -19,8 +19,11 @@
 //              log-sum-exp at the end of each work tile.  The two heads take
 //              turns for the exponentials, so that the MUFU units serve one head
 //              while the tensor core runs the other head's PV and next S
-//   warp 16    TMA producer: Q of both heads per work tile, K and V tiles into
-//              a two-stage ring (128-byte swizzled, no multicast)
+//   warp 16    TMA producer: claims the work tiles (an atomic counter in the
+//              caller's workspace, else a static stride over the list) and
+//              hands them on through a shared-memory ring; loads Q of both
+//              heads per work tile, K and V tiles into a two-stage ring
+//              (128-byte swizzled, no multicast)
 //   warp 17    TMEM allocator and MMA issuer (one thread), in the order
 //                PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ...
 //              with S_h = Q_h K^T (both operands in shared memory) and
@@ -41,6 +44,7 @@ constexpr int kPfM = 128;                  // query rows per tile
 constexpr int kPfN = 128;                  // keys per tile
 constexpr int kPfThreads = 576;            // 18 warps
 constexpr int kPfStages = 2;
+constexpr int kPfSlots = 4;                // work-tile ring between the producer and the consumers
 constexpr uint32_t kQTileBytes = kPfM * 128 * 2;     // 32 KB: one head's Q tile
 constexpr uint32_t kQHalfBytes = kQTileBytes / 2;    // 64-column swizzled box
 constexpr uint32_t kKVTileBytes = kPfN * 128 * 2;    // 32 KB: one K or V tile
@@ -57,6 +61,7 @@ struct PrefillArgs {
     __nv_bfloat16 *out;    // [B][L][Hq][128]
     float *lse;            // [B][Hq][L] or null
     const float *sink_logit;
+    int32_t *work_counter; // zeroed before the launch, or null for the static order
     int32_t L, hq, hkv, n_qtiles, n_work, batch_pairs;
     int32_t sink, recent, window;
     float scale_log2;
@@ -129,6 +134,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     // row-half exchanges between the eight softmax warps of a head (bounded
     // mbarrier waits, so that a timed-out warp cannot strand its partners)
     __shared__ uint64_t xmax[2][2], xsum[2];           // [tile parity][head], [head]
+    // work tiles claimed by the producer, read by the MMA issuer and the softmax warps
+    __shared__ uint64_t work_full[kPfSlots], work_empty[kPfSlots];
+    __shared__ int work_slot[kPfSlots];
     __shared__ float red_max[2][2][2][kPfM];           // [tile parity][head][column half][row]
     __shared__ float red_sum[2][2][kPfM];              // [head][column half][row]
     __shared__ uint32_t tmem_base;
@@ -150,6 +158,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             mbar_init(&xmax[1][h], 8);
             mbar_init(&xsum[h], 8);
         }
+        for (int sl = 0; sl < kPfSlots; ++sl) {
+            mbar_init(&work_full[sl], 1);
+            mbar_init(&work_empty[sl], 17);     // the MMA issuer and the 16 softmax warps
+        }
         for (int w8 = 0; w8 < 8; ++w8) mbar_arrive(&turn[0]);   // head 0 takes the first turn
         fence_mbar_init();
     }
@@ -169,9 +181,21 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             prefetch_tmap(&a.tm_q);
             prefetch_tmap(&a.tm_k);
             prefetch_tmap(&a.tm_v);
-            int jg = 0, wc = 0;
+            int jg = 0;
             bool ok = true;
-            for (int w = blockIdx.x; w < a.n_work && ok; w += gridDim.x, ++wc) {
+            int w = blockIdx.x;
+            for (int wc = 0; ok; ++wc) {
+                // publish the work tile (an index >= n_work tells the consumers to stop)
+                const int sl = wc % kPfSlots;
+                if (wc >= kPfSlots && !(ok = mbar_wait(&work_empty[sl], ((wc / kPfSlots) - 1) & 1))) break;
+                work_slot[sl] = w;
+                mbar_arrive(&work_full[sl]);
+                if (w >= a.n_work) break;
+                // claim the next one now: the atomic's latency hides behind this tile's loads.
+                // Claims follow the heaviest-first order, so every CTA takes the next
+                // tile when it is free (longest-processing-time-first scheduling)
+                const int w_next = a.work_counter != nullptr ? (int)gridDim.x + atomicAdd(a.work_counter, 1)
+                                                             : w + (int)gridDim.x;
                 const PfWork wk = work_of(a, w);
                 const TileList tl = tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window);
                 // Q of the previous work tile must no longer be read by the MMA
@@ -194,6 +218,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                                     wk.b, &kv_full[st]);
                     }
                 }
+                w = w_next;
             }
         }
         __syncwarp();  // lanes 1..31 wait for the producer lane before the CTA barrier
@@ -222,9 +247,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                            id_pv, (first && k == 0) ? 0u : 1u);
                 mma_commit(&o_done[h]);
             };
-            int jg = 0, wc = 0;
+            int jg = 0;
             bool ok = true;
-            for (int w = blockIdx.x; w < a.n_work && ok; w += gridDim.x, ++wc) {
+            for (int wc = 0; ok; ++wc) {
+                const int sl = wc % kPfSlots;
+                if (!(ok = mbar_wait(&work_full[sl], (wc / kPfSlots) & 1))) break;
+                const int w = work_slot[sl];
+                mbar_arrive(&work_empty[sl]);
+                if (w >= a.n_work) break;
                 const PfWork wk = work_of(a, w);
                 const TileList tl = tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window);
                 const int n_kv = tl.count();
@@ -265,9 +295,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         const uint32_t s_tmem = tmem + h * 128 + lane_base;
         const uint32_t o_tmem = tmem + 256 + h * 128 + lane_base;
         const float c = a.scale_log2;
-        int jg = 0, wc = 0;
+        int jg = 0;
         bool ok = true;
-        for (int w = blockIdx.x; w < a.n_work && ok; w += gridDim.x, ++wc) {
+        for (int wc = 0; ok; ++wc) {
+            const int sl = wc % kPfSlots;
+            const bool have = mbar_wait(&work_full[sl], (wc / kPfSlots) & 1);
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, have)) { ok = false; break; }
+            const int w = work_slot[sl];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&work_empty[sl]);
+            if (w >= a.n_work) break;
             const PfWork wk = work_of(a, w);
             const int kind = a.kind[wk.g];
             const TileList tl = tile_list(kind, wk.t, a.L, a.sink, a.recent, a.window);
@@ -455,7 +493,8 @@ inline bool make_tmap(CUtensorMap *m, const void *base, int B, int L, int H, int
 
 inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_full, int sink,
                           int ring, const void *q, const void *k, const void *v, int32_t L, void *out,
-                          float *lse, cudaStream_t stream, char *err, size_t err_len) {
+                          float *lse, int32_t *work_counter, cudaStream_t stream, char *err,
+                          size_t err_len) {
     PrefillArgs a;
     memset(&a, 0, sizeof a);
     const int B = p->batch;
@@ -491,7 +530,8 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     }
     a.batch_pairs = B * (p->num_q_heads / 2);
     const int64_t n_work = (int64_t)a.batch_pairs * a.n_qtiles;
-    if (n_work > INT32_MAX) {
+    // the counter runs up to n_work + 2 * grid
+    if (n_work > INT32_MAX - 4096) {
         snprintf(err, err_len, "too many query tiles for one prefill launch");
         return DUO_ERR_INVALID_ARG;
     }
@@ -499,6 +539,11 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const unsigned grid = (unsigned)std::min<int64_t>(n_work, sms);
+    a.work_counter = work_counter;
+    if (work_counter != nullptr && cudaMemsetAsync(work_counter, 0, sizeof(int32_t), stream) != cudaSuccess) {
+        snprintf(err, err_len, "zeroing the prefill work counter failed");
+        return DUO_ERR_CUDA;
+    }
     prefill_fwd<<<grid, kPfThreads, kPfSmem, stream>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {

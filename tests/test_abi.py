@@ -140,10 +140,16 @@ def test_prefill_argument_checks(lib):
     p = _params()
     pc = p.as_c()
     f = lib.duo_attn_prefill
-    assert f(ctypes.byref(pc), 0x1000, 0x1000, 0x1000, -5, 0x1000, None, None) == duo.DUO_ERR_INVALID_ARG
-    assert f(ctypes.byref(pc), 0x1000, 0, 0x1000, 16, 0x1000, None, None) == duo.DUO_ERR_INVALID_ARG
-    assert f(ctypes.byref(pc), 0x1000, 0x1000, 0x1000, 16, 0x1000, 0x1004, None) == duo.DUO_ERR_INVALID_ARG
-    assert f(ctypes.byref(pc), 0, 0, 0, 0, 0, None, None) == duo.DUO_OK   # empty prefill
+    a = 0x1000
+    assert f(ctypes.byref(pc), a, a, a, -5, a, None, None, 0, None) == duo.DUO_ERR_INVALID_ARG
+    assert f(ctypes.byref(pc), a, 0, a, 16, a, None, None, 0, None) == duo.DUO_ERR_INVALID_ARG
+    assert f(ctypes.byref(pc), a, a, a, 16, a, 0x1004, None, 0, None) == duo.DUO_ERR_INVALID_ARG
+    assert f(ctypes.byref(pc), 0, 0, 0, 0, 0, None, None, 0, None) == duo.DUO_OK   # empty prefill
+    need = duo.duo_prefill_workspace_bytes()
+    assert need >= 4
+    # a workspace that is too small or misaligned is refused before anything runs
+    assert f(ctypes.byref(pc), a, a, a, 16, a, None, 0x2000, need - 1, None) == duo.DUO_ERR_WORKSPACE
+    assert f(ctypes.byref(pc), a, a, a, 16, a, None, 0x2008, need, None) == duo.DUO_ERR_WORKSPACE
 
 
 def test_workspace_size_is_host_arithmetic(lib):

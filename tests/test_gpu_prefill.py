@@ -18,11 +18,17 @@ from gpu_helpers import LSE_ABS, assert_close, layers
 pytestmark = pytest.mark.gpu
 
 
-def prefill_gpu(params, q, k, v):
+def prefill_gpu(params, q, k, v, dynamic=True):
+    """dynamic: CTAs claim work tiles from a counter in a workspace (the path
+    the benchmark times); else the static stride over the work list."""
     B, L, Hq, D = q.shape
     out = torch.full((B, L, Hq, D), float("nan"), dtype=torch.bfloat16, device="cuda")
     lse = torch.full((B, Hq, L), float("nan"), dtype=torch.float32, device="cuda")
-    duo.duo_attn_prefill(params, q, k, v, out, lse)
+    ws = None
+    if dynamic:
+        # stale contents: the call must zero the counter itself
+        ws = torch.full((duo.duo_prefill_workspace_bytes(),), 0x7f, dtype=torch.uint8, device="cuda")
+    duo.duo_attn_prefill(params, q, k, v, out, lse, workspace=ws)
     torch.cuda.synchronize()
     assert duo.duo_get_device_status() == duo.DUO_OK
     return out, lse
@@ -56,12 +62,13 @@ def compare_rows(out, lse, ref_o, ref_l, rows, B, Hq, L, what):
     return assert_close(torch.from_numpy(got_o), ref_o, torch.from_numpy(got_l), ref_l, what)
 
 
+@pytest.mark.parametrize("dynamic", [True, False])
 @pytest.mark.parametrize("L", [1, 5, 127, 128, 129, 300, 321, 600])
-def test_prefill_duo_layer_all_rows(cuda_device, L):
+def test_prefill_duo_layer_all_rows(cuda_device, L, dynamic):
     B = 2
     p, o = layers(B, full_mask=(1, 0, 0, 1, 0, 1, 1, 0))
     q, k, v = make_qkv(B, L, 40)
-    out, lse = prefill_gpu(p, q, k, v)
+    out, lse = prefill_gpu(p, q, k, v, dynamic)
     ref_o, ref_l = oracle.attn_prefill(o, inputs.bits(q), inputs.bits(k), inputs.bits(v))
     got_o = out.permute(0, 2, 1, 3).reshape(-1, 128)
     assert_close(got_o, ref_o, lse.reshape(-1), ref_l, f"L={L}")
@@ -114,6 +121,31 @@ def test_prefill_attended_sets_exact(cuda_device):
             assert np.all(np.isin(np.round(want), [0.0, 1.0]))
             assert np.array_equal(np.round(got), np.round(want)), f"{kw} chunk {chunk}"
             assert np.abs(lse.reshape(-1).cpu().numpy() - ref_l).max() <= LSE_ABS
+
+
+def test_prefill_schedules_give_identical_bytes(cuda_device):
+    """A work tile's result does not depend on which CTA computes it, so the
+    static and the dynamic schedule (and repeated dynamic runs) agree bit for
+    bit; 4000 tokens give 32 query tiles x 48 pairs, several per CTA."""
+    B, L = 2, 4000
+    p, _ = layers(B, full_mask=(0, 0, 1, 0, 0, 1, 0, 0))
+    q, k, v = make_qkv(B, L, 46)
+    o_s, l_s = prefill_gpu(p, q, k, v, dynamic=False)
+    for _ in range(2):
+        o_d, l_d = prefill_gpu(p, q, k, v, dynamic=True)
+        assert torch.equal(o_s, o_d) and torch.equal(l_s, l_d)
+
+
+def test_prefill_workspace_too_small_is_refused(cuda_device):
+    p, _ = layers(1, full_mask=(1,) * 8)
+    q, k, v = make_qkv(1, 64, 47)
+    out = torch.zeros_like(q)
+    small = torch.zeros(duo.duo_prefill_workspace_bytes() - 1, dtype=torch.uint8, device="cuda")
+    with pytest.raises(duo.DuoError) as e:
+        duo.duo_attn_prefill(p, q, k, v, out, None, workspace=small)
+    assert e.value.code == duo.DUO_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
 
 
 def test_prefill_zero_length_is_noop(cuda_device):
