@@ -50,7 +50,8 @@ constexpr uint32_t kQHalfBytes = kQTileBytes / 2;    // 64-column swizzled box
 constexpr uint32_t kKVTileBytes = kPfN * 128 * 2;    // 32 KB: one K or V tile
 constexpr uint32_t kKVHalfBytes = kKVTileBytes / 2;
 constexpr uint32_t kPfStageBytes = 2 * kKVTileBytes;
-constexpr size_t kPfSmem = 1024 + 2 * kQTileBytes + kPfStages * kPfStageBytes;
+constexpr uint32_t kOStageBytes = 32 * 16 * 2;    // one softmax warp's O chunk: 32 rows x 16 columns
+constexpr size_t kPfSmem = 1024 + 2 * kQTileBytes + kPfStages * kPfStageBytes + 16 * kOStageBytes;
 
 enum : int { kKindFull = 0, kKindStreaming = 1, kKindSliding = 2 };
 
@@ -58,7 +59,7 @@ struct PrefillArgs {
     CUtensorMap tm_q;      // [B][L][Hq][128] bf16, box 64 x 1 x 128 x 1
     CUtensorMap tm_k;      // [B][L][Hkv][128]
     CUtensorMap tm_v;
-    __nv_bfloat16 *out;    // [B][L][Hq][128]
+    CUtensorMap tm_o;      // out [B][L][Hq][128] bf16, box 16 x 1 x 32 x 1, no swizzle
     float *lse;            // [B][Hq][L] or null
     const float *sink_logit;
     int32_t *work_counter; // zeroed before the launch, or null for the static order
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     char *smem = psmem_base + ((1024u - (smem_u32(psmem_base) & 1023u)) & 1023u);
     char *sQ = smem;                                   // [2 heads][32 KB]
     char *sKV = smem + 2 * kQTileBytes;                // [stages][K 32 KB | V 32 KB]
+    char *sO = sKV + kPfStages * kPfStageBytes;        // [softmax warp][32 rows][16 columns] bf16
     __shared__ uint64_t q_full, q_empty, kv_full[kPfStages], kv_empty[kPfStages];
     __shared__ uint64_t s_full[2], p_full[2], o_done[2], turn[2];
     // row-half exchanges between the eight softmax warps of a head (bounded
@@ -181,6 +183,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             prefetch_tmap(&a.tm_q);
             prefetch_tmap(&a.tm_k);
             prefetch_tmap(&a.tm_v);
+            prefetch_tmap(&a.tm_o);
             int jg = 0;
             bool ok = true;
             int w = blockIdx.x;
@@ -421,23 +424,35 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             tc_fence_after();
             const float l_row = red_sum[h][0][r] + red_sum[h][1][r];
             const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
-            __nv_bfloat16 *orow = a.out + (((size_t)wk.b * a.L + i) * a.hq + hq) * 128 + half * 64;
+            // O / l leaves through this warp's 1 KB staging buffer as 32-row x
+            // 16-column TMA stores (rows past L are clipped by the tensor map):
+            // coalesced by the copy engine instead of 32 scattered rows per store
+            char *stage = sO + warp * kOStageBytes;
+            const int row0 = wk.t * kPfM + quarter * 32;   // first row of this warp's boxes
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 32) {
+            for (int cb = 0; cb < 64 && row0 < a.L; cb += 32) {
                 uint32_t orr[32];
                 tmem_ld32(o_tmem + half * 64 + cb, orr);
                 tmem_ld_wait();
                 reg_fence32(orr);
-                if (i < a.L) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + cb);
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(orr[e]) * inv_l, __uint_as_float(orr[e + 1]) * inv_l);
-                        v.y = pack_bf16x2(__uint_as_float(orr[e + 2]) * inv_l, __uint_as_float(orr[e + 3]) * inv_l);
-                        v.z = pack_bf16x2(__uint_as_float(orr[e + 4]) * inv_l, __uint_as_float(orr[e + 5]) * inv_l);
-                        v.w = pack_bf16x2(__uint_as_float(orr[e + 6]) * inv_l, __uint_as_float(orr[e + 7]) * inv_l);
-                        dst[e / 8] = v;
+                for (int c16 = 0; c16 < 32; c16 += 16) {
+                    if (lane == 0) bulk_wait_read_all();   // the previous chunk has left the buffer
+                    __syncwarp();
+                    auto nb = [&](int e) {
+                        return pack_bf16x2(__uint_as_float(orr[c16 + e]) * inv_l,
+                                           __uint_as_float(orr[c16 + e + 1]) * inv_l);
+                    };
+                    const uint4 v0 = make_uint4(nb(0), nb(2), nb(4), nb(6));
+                    const uint4 v1 = make_uint4(nb(8), nb(10), nb(12), nb(14));
+                    uint4 *row = reinterpret_cast<uint4 *>(stage + lane * 32);
+                    row[0] = v0;
+                    row[1] = v1;
+                    fence_proxy_async_smem();              // visible to the copy engine
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_4d(&a.tm_o, stage, half * 64 + cb + c16, hq, row0, wk.b);
+                        bulk_commit_group();
                     }
                 }
             }
@@ -449,6 +464,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             // next PV nor the next epilogue can overwrite them early
             tc_fence_before();
         }
+        if (lane == 0) bulk_wait_all();                    // this warp's O stores have landed
         __syncwarp();
     }
     tc_fence_before();
@@ -479,6 +495,20 @@ inline EncodeTiledFn encode_fn() {
 
 // [B][L][H][128] bf16 viewed as a 4-D tensor (128, H, L, B), loaded as
 // 64-column x `rows`-row boxes with the 128-byte swizzle.
+// The output [B][L][Hq][128] bf16 as 16-column x 32-row boxes, no swizzle
+// (the layout a softmax warp stages: row r at byte 32 r).
+inline bool make_out_tmap(CUtensorMap *m, void *base, int B, int L, int H) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {256, (cuuint64_t)H * 256, (cuuint64_t)L * H * 256};
+    const cuuint32_t box[4] = {16, 1, 32, 1};
+    const cuuint32_t elem[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, elem,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline bool make_tmap(CUtensorMap *m, const void *base, int B, int L, int H, int rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -500,11 +530,11 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     const int B = p->batch;
     if (!make_tmap(&a.tm_q, q, B, L, p->num_q_heads, kPfM) ||
         !make_tmap(&a.tm_k, k, B, L, p->num_kv_heads, kPfN) ||
-        !make_tmap(&a.tm_v, v, B, L, p->num_kv_heads, kPfN)) {
+        !make_tmap(&a.tm_v, v, B, L, p->num_kv_heads, kPfN) ||
+        !make_out_tmap(&a.tm_o, out, B, L, p->num_q_heads)) {
         snprintf(err, err_len, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
         return DUO_ERR_CUDA;
     }
-    a.out = (__nv_bfloat16 *)out;
     a.lse = lse;
     a.sink_logit = p->sink_logit;
     a.L = L;
