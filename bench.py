@@ -421,6 +421,7 @@ class DecodeSmall:
         out = torch.empty_like(q)
         duo.duo_attn_prefill(self.params, q, k, v, out, None)
         duo.duo_kv_append(self.params, self.cache, k, v)
+        self.n = w.seq_len
         self.k1 = inputs.randn_bf16((1, 1, 8, 128), seed + 3, "cuda")
         self.v1 = inputs.randn_bf16((1, 1, 8, 128), seed + 4, "cuda")
         self.q1 = inputs.randn_bf16((1, 48, 128), seed + 5, "cuda")
@@ -433,7 +434,8 @@ class DecodeSmall:
 
     def step(self):
         duo.duo_kv_append(self.params, self.cache, self.k1, self.v1)
-        duo.duo_attn_decode(self.params, self.cache, self.q1, self.cap, self.out, self.lse, self.ws)
+        self.n += 1                       # the host knows every sequence's length
+        duo.duo_attn_decode(self.params, self.cache, self.q1, self.n, self.out, self.lse, self.ws)
 
     def config(self):
         return {"workload": "decode_small: B=1, 1024-token prompt, then append one token + decode per step"}
@@ -445,10 +447,20 @@ WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40, "decode_small": Decode
 
 
 # ------------------------------------------------------------------ timing
+PREROLL_CYCLES = 2_000_000     # ~1 ms device spin queued ahead of the start event
+
+
 def time_steps(fn, steps, stream, world):
+    """Device time of `steps` calls of fn: CUDA events on the launching stream,
+    barrier + synchronize on both sides.  A ~1 ms spin kernel is queued before
+    the start event, so the host's time to issue the first step's launches is
+    not counted as idle device time inside the region (every step's device
+    work still is)."""
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(PREROLL_CYCLES)
     start.record(stream)
     for _ in range(steps):
         fn()
@@ -482,15 +494,23 @@ CSRC = os.path.join(ROOT, "kv_cache_reduction_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
 
 
+KERNEL_SOURCES = {"decode_split": ("decode.cuh", "ptx.cuh", "kv_append.cuh"),
+                  "prefill_fwd": ("prefill.cuh", "ptx.cuh")}
+
+
+def sources_digest(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def measured_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu capture, or None once the
     kernel's sources differ from the ones that were profiled."""
-    import hashlib
-    h = hashlib.sha256()
-    for f in ("decode.cuh", "ptx.cuh", "kv_append.cuh"):
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(fh.read())
-    digest = h.hexdigest()[:16]
+    digest = sources_digest(kernel)
     try:
         with open(TRAFFIC_FILE) as fh:
             for line in fh:
@@ -530,6 +550,9 @@ def run_ours(args, world, rank):
     rf["kernel"] = wl.kernel
     if args.workload == "decode_b32":
         rf["traffic"] = measured_traffic("decode_split", "decode_b32")
+        rf["traffic_unit"] = "bytes per launch (ncu dram read + write)"
+    elif wl.kernel == "prefill_fwd":
+        rf["traffic"] = measured_traffic("prefill_fwd", args.workload)
         rf["traffic_unit"] = "bytes per launch (ncu dram read + write)"
     res = {"metric": METRIC, "value": round(value, 2), "unit": wl.unit, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 4),
