@@ -104,6 +104,30 @@ typedef struct {
     int32_t *ring_head;
 } duo_cache;
 
+/* Optional output gate of the attention (Laguna's gated attention output:
+ * the Laguna attention article "深入理解Laguna的注意力机制", section on
+ * attention output gating, and the Laguna XS 2.1 sliding-window article,
+ * section on the g_proj output gate).  The normalised attention output of
+ * query head h is multiplied by sigmoid(g) before it is rounded and stored:
+ *   DUO_GATE_PER_ELEMENT  one g per (query head, channel), laid out like out;
+ *   DUO_GATE_PER_HEAD     one g per query head, broadcast over the channels,
+ *                         laid out like out without its last dimension
+ *                         (prefill [B][L][Hq], decode [B][Hq]).
+ * g is the model's gate projection output (bf16, device, 16-byte aligned);
+ * computing it is not part of this library.  The pages do not name the gate's
+ * activation: sigmoid is this library's reading.  The log-sum-exp output is
+ * not gated.  A NULL duo_gate pointer, or mode DUO_GATE_NONE, means no gate. */
+typedef enum {
+    DUO_GATE_NONE = 0,
+    DUO_GATE_PER_ELEMENT = 1,
+    DUO_GATE_PER_HEAD = 2
+} duo_gate_mode;
+
+typedef struct {
+    int32_t mode;           /* duo_gate_mode                                 */
+    const void *values;     /* device bf16 gate pre-activations              */
+} duo_gate;
+
 /* Appends n_new tokens to every sequence of the cache.
  * k, v: device bf16 [B][n_new][Hkv][D] (token-major, as a K/V projection
  * writes them).  For each sequence b and token t the position is
@@ -137,10 +161,12 @@ DUO_API size_t duo_prefill_workspace_bytes(void);
  * heads' costs differ); without one they take a fixed stride of the list.
  * Calls that may run at the same time need separate workspaces.  A smaller
  * or misaligned workspace returns DUO_ERR_WORKSPACE.
+ * gate: NULL or an output gate (see duo_gate; values [B][L][Hq][D] or
+ * [B][L][Hq]).
  * The cache is not touched: call duo_kv_append(n_new = L) to fill it. */
 DUO_API int duo_attn_prefill(const duo_params *params, const void *q, const void *k, const void *v,
                      int32_t seq_len, void *out, float *lse, void *workspace,
-                     size_t workspace_bytes, void *stream);
+                     size_t workspace_bytes, const duo_gate *gate, void *stream);
 
 /* Bytes of device workspace duo_attn_decode needs for this layer when no
  * sequence holds more than max_seq_len tokens.  Returns 0 on invalid params. */
@@ -156,10 +182,12 @@ DUO_API size_t duo_decode_workspace_bytes(const duo_params *params, int32_t max_
  * aligned, contents need not be initialised.  A full head reads its seq_len
  * rows, a ring head only its valid sink and ring slots (at most
  * sink + recent or window).  A sequence with seq_len 0 gives out = 0 and
- * lse = -inf (or the sink logit when one is given). */
+ * lse = -inf (or the sink logit when one is given).
+ * gate: NULL or an output gate (see duo_gate; values [B][Hq][D] or [B][Hq]),
+ * applied in the split merge. */
 DUO_API int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void *q,
                     int32_t max_seq_len, void *out, float *lse, void *workspace,
-                    size_t workspace_bytes, void *stream);
+                    size_t workspace_bytes, const duo_gate *gate, void *stream);
 
 /* duo_attn_decode without a caller workspace, for callers that cannot
  * allocate device memory at call time (an engine plugin that must not
@@ -177,7 +205,8 @@ DUO_API int duo_attn_decode(const duo_params *params, const duo_cache *cache, co
  * issue them on one stream.  Arguments, outputs and errors otherwise as
  * duo_attn_decode. */
 DUO_API int duo_attn_decode_static(const duo_params *params, const duo_cache *cache, const void *q,
-                                   int32_t max_seq_len, void *out, float *lse, void *stream);
+                                   int32_t max_seq_len, void *out, float *lse,
+                                   const duo_gate *gate, void *stream);
 
 /* KV-cache accounting for one layer (host arithmetic only, no device access).
  * The DuoAttention card (sections Benefits and Changes In This Submission)

@@ -51,6 +51,30 @@ class DuoError(RuntimeError):
         self.code = code
 
 
+DUO_GATE_NONE, DUO_GATE_PER_ELEMENT, DUO_GATE_PER_HEAD = 0, 1, 2
+
+
+class _Gate(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("values", ctypes.c_void_p)]
+
+
+def _gate(gate: Optional[torch.Tensor], out: torch.Tensor):
+    """A duo_gate for gate pre-activations shaped like out (one per channel) or
+    like out without its last dimension (one per head); None for no gate."""
+    if gate is None:
+        return None
+    if tuple(gate.shape) == tuple(out.shape):
+        mode = DUO_GATE_PER_ELEMENT
+    elif tuple(gate.shape) == tuple(out.shape[:-1]):
+        mode = DUO_GATE_PER_HEAD
+    else:
+        raise ValueError(f"gate shape {tuple(gate.shape)} is neither out's {tuple(out.shape)} "
+                         f"nor out's without the channel dimension")
+    if gate.dtype != torch.bfloat16 or not gate.is_contiguous():
+        raise ValueError("gate must be a contiguous bf16 tensor")
+    return ctypes.byref(_Gate(mode, _ptr(gate)))
+
+
 class _Params(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
@@ -88,13 +112,14 @@ def load_library(path: str = LIBRARY_PATH) -> ctypes.CDLL:
     lib.duo_kv_append.restype = ctypes.c_int
     lib.duo_prefill_workspace_bytes.argtypes = []
     lib.duo_prefill_workspace_bytes.restype = ctypes.c_size_t
-    lib.duo_attn_prefill.argtypes = [P, vp, vp, vp, ctypes.c_int32, vp, vp, vp, ctypes.c_size_t, vp]
+    G = ctypes.POINTER(_Gate)
+    lib.duo_attn_prefill.argtypes = [P, vp, vp, vp, ctypes.c_int32, vp, vp, vp, ctypes.c_size_t, G, vp]
     lib.duo_attn_prefill.restype = ctypes.c_int
     lib.duo_decode_workspace_bytes.argtypes = [P, ctypes.c_int32]
     lib.duo_decode_workspace_bytes.restype = ctypes.c_size_t
-    lib.duo_attn_decode.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.duo_attn_decode.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, vp, ctypes.c_size_t, G, vp]
     lib.duo_attn_decode.restype = ctypes.c_int
-    lib.duo_attn_decode_static.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, vp]
+    lib.duo_attn_decode_static.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, G, vp]
     lib.duo_attn_decode_static.restype = ctypes.c_int
     lib.duo_cache_bytes.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(CacheStats)]
     lib.duo_cache_bytes.restype = ctypes.c_int
@@ -211,14 +236,18 @@ def duo_prefill_workspace_bytes() -> int:
 def duo_attn_prefill(params: DuoParams, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                      out: torch.Tensor, lse: Optional[torch.Tensor] = None,
                      seq_len: Optional[int] = None, stream=None,
-                     workspace: Optional[torch.Tensor] = None) -> None:
+                     workspace: Optional[torch.Tensor] = None,
+                     gate: Optional[torch.Tensor] = None) -> None:
     """workspace: None (static work-tile order) or a device tensor of at least
-    duo_prefill_workspace_bytes() bytes (dynamic, balanced order)."""
+    duo_prefill_workspace_bytes() bytes (dynamic, balanced order).  gate: None,
+    or bf16 gate pre-activations [B][L][Hq][D] (per channel) or [B][L][Hq] (per
+    head); out is then multiplied by sigmoid(gate)."""
     L = int(q.shape[1]) if seq_len is None else int(seq_len)
     p = params.as_c()
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load_library().duo_attn_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), L, _ptr(out),
-                                           _ptr(lse), _ptr(workspace), nbytes, _stream(stream)))
+                                           _ptr(lse), _ptr(workspace), nbytes, _gate(gate, out),
+                                           _stream(stream)))
 
 
 def duo_decode_workspace_bytes(params: DuoParams, max_seq_len: int) -> int:
@@ -228,23 +257,25 @@ def duo_decode_workspace_bytes(params: DuoParams, max_seq_len: int) -> int:
 
 def duo_attn_decode(params: DuoParams, cache: DuoCache, q: torch.Tensor, max_seq_len: int,
                     out: torch.Tensor, lse: Optional[torch.Tensor], workspace: torch.Tensor,
-                    stream=None) -> None:
+                    stream=None, gate: Optional[torch.Tensor] = None) -> None:
+    """gate: None, or bf16 gate pre-activations [B][Hq][D] or [B][Hq]."""
     p, c = params.as_c(), cache.as_c()
     nbytes = workspace.numel() * workspace.element_size()
     _check(load_library().duo_attn_decode(ctypes.byref(p), ctypes.byref(c), _ptr(q), int(max_seq_len),
                                           _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
-                                          _stream(stream)))
+                                          _gate(gate, out), _stream(stream)))
 
 
 def duo_attn_decode_static(params: DuoParams, cache: DuoCache, q: torch.Tensor, max_seq_len: int,
-                           out: torch.Tensor, lse: Optional[torch.Tensor], stream=None) -> None:
+                           out: torch.Tensor, lse: Optional[torch.Tensor], stream=None,
+                           gate: Optional[torch.Tensor] = None) -> None:
     """duo_attn_decode with the library's built-in 16 MiB scratch instead of a
     caller workspace, for callers that cannot allocate device memory when they
     decode.  Calls that may overlap on the GPU share that scratch and race."""
     p, c = params.as_c(), cache.as_c()
     _check(load_library().duo_attn_decode_static(ctypes.byref(p), ctypes.byref(c), _ptr(q),
                                                  int(max_seq_len), _ptr(out), _ptr(lse),
-                                                 _stream(stream)))
+                                                 _gate(gate, out), _stream(stream)))
 
 
 def duo_cache_bytes(params: DuoParams, capacity: int, seq_len: int) -> CacheStats:

@@ -62,6 +62,8 @@ struct DecodeArgs {
     int32_t sink, ring, slots;
     int32_t chunk_full, splits_full, chunk_ring, splits_ring, max_splits, n_items;
     float scale_log2;               // softmax_scale * log2(e)
+    const __nv_bfloat16 *gate;      // output gate pre-activations or null
+    int32_t gate_mode;              // 0 none, 1 per (head, channel) [B][Hq][D], 2 per head [B][Hq]
     int32_t withhold_tile;          // test hook: CTA 0 issues no load from this tile on (-1: off)
     int8_t full_head[64];           // full rank -> KV head
     int8_t ring_head_of[64];        // ring rank -> KV head
@@ -497,7 +499,12 @@ __global__ void __launch_bounds__(kD) decode_merge(const __grid_constant__ Decod
         }
         if (has_sink) den += ex2_approx(sig - M);
     }
-    const float o = den > 0.f ? num / den : 0.f;
+    float o = den > 0.f ? num / den : 0.f;
+    if (a.gate_mode != 0) {
+        // output gate: o * sigmoid(g), g per channel or per head
+        const float g = __bfloat162float(a.gate[a.gate_mode == 1 ? (size_t)bh * kD + threadIdx.x : (size_t)bh]);
+        o = o / (1.f + ex2_approx(-g * kLog2eF));
+    }
     a.out[(size_t)bh * kD + threadIdx.x] = __float2bfloat16_rn(o);
     if (a.lse != nullptr && threadIdx.x == 0)
         a.lse[bh] = den > 0.f ? (M + log2f(den)) * kLn2F : -INFINITY;

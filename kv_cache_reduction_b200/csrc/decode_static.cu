@@ -60,12 +60,13 @@ extern "C" {
 // workspace check: DUO_ERR_WORKSPACE, nothing launched, and duo_last_error()
 // gives the bytes needed and available.
 DUO_API int duo_attn_decode_static(const duo_params *params, const duo_cache *cache, const void *q,
-                                   int32_t max_seq_len, void *out, float *lse, void *stream) {
+                                   int32_t max_seq_len, void *out, float *lse,
+                                   const duo_gate *gate, void *stream) {
     void *scratch = nullptr;
     const int rc = scratch_for_current_device(&scratch);
     if (rc != DUO_OK) return rc;
     return duo_attn_decode(params, cache, q, max_seq_len, out, lse, scratch, kStaticScratchBytes,
-                           stream);
+                           gate, stream);
 }
 
 }  // extern "C"

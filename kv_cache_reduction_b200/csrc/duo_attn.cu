@@ -27,6 +27,21 @@ int fail(int code, const char *fmt, ...) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// The output gate, if any: mode in range, values present and 16-byte aligned.
+int check_gate(const duo_gate *g, int *mode, const void **values) {
+    *mode = DUO_GATE_NONE;
+    *values = nullptr;
+    if (g == nullptr || g->mode == DUO_GATE_NONE) return DUO_OK;
+    if (g->mode != DUO_GATE_PER_ELEMENT && g->mode != DUO_GATE_PER_HEAD)
+        return fail(DUO_ERR_INVALID_ARG, "gate mode %d is not DUO_GATE_NONE / PER_ELEMENT / PER_HEAD",
+                    (int)g->mode);
+    if (g->values == nullptr || !aligned16(g->values))
+        return fail(DUO_ERR_INVALID_ARG, "gate values must be a 16-byte aligned device pointer");
+    *mode = g->mode;
+    *values = g->values;
+    return DUO_OK;
+}
+
 constexpr int kMaxHkv = 64;
 constexpr int kMaxWindow = 8192;
 constexpr int kMaxRing = 8192;
@@ -283,10 +298,13 @@ size_t duo_decode_workspace_bytes(const duo_params *params, int32_t max_seq_len)
 
 int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void *q,
                     int32_t max_seq_len, void *out, float *lse, void *workspace,
-                    size_t workspace_size, void *stream) {
+                    size_t workspace_size, const duo_gate *gate, void *stream) {
     Layout L;
     int rc = check_params(params, &L);
     if (rc) return rc;
+    int gate_mode = 0;
+    const void *gate_values = nullptr;
+    if ((rc = check_gate(gate, &gate_mode, &gate_values))) return rc;
     if ((rc = check_cache(cache, L))) return rc;
     if (max_seq_len < 0 || max_seq_len > kMaxPos)
         return fail(DUO_ERR_INVALID_ARG, "max_seq_len must be in [0, 2^30]");
@@ -338,6 +356,8 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     a.max_splits = d.max_splits;
     a.n_items = (int32_t)d.items;
     a.scale_log2 = params->softmax_scale * duo::kLog2eF;
+    a.gate = (const __nv_bfloat16 *)gate_values;
+    a.gate_mode = gate_mode;
     // Test hook for the failure-detection path: DUO_TEST_WITHHOLD_TILE=t makes
     // the first CTA's producer stop before tile t; its consumers then time out
     // and the call reports DUO_ERR_TIMEOUT through duo_get_device_status().
@@ -374,10 +394,13 @@ size_t duo_prefill_workspace_bytes(void) { return kPrefillWorkspaceBytes; }
 
 int duo_attn_prefill(const duo_params *params, const void *q, const void *k, const void *v,
                      int32_t seq_len, void *out, float *lse, void *workspace, size_t workspace_bytes,
-                     void *stream) {
+                     const duo_gate *gate, void *stream) {
     Layout L;
     int rc = check_params(params, &L);
     if (rc) return rc;
+    int gate_mode = 0;
+    const void *gate_values = nullptr;
+    if ((rc = check_gate(gate, &gate_mode, &gate_values))) return rc;
     if (workspace && (workspace_bytes < kPrefillWorkspaceBytes || !aligned16(workspace)))
         return fail(DUO_ERR_WORKSPACE, "prefill workspace: need %zu bytes, 16-byte aligned (got %zu)",
                     kPrefillWorkspaceBytes, workspace_bytes);
@@ -388,7 +411,8 @@ int duo_attn_prefill(const duo_params *params, const void *q, const void *k, con
         return fail(DUO_ERR_INVALID_ARG, "q / k / v / out / lse must be 16-byte aligned");
     if ((rc = check_device(nullptr))) return rc;
     return duo::launch_prefill(params, L.sliding, L.heads.is_full, L.sink, L.ring, q, k, v, seq_len,
-                               out, lse, (int32_t *)workspace, (cudaStream_t)stream, g_err, sizeof g_err);
+                               out, lse, (int32_t *)workspace, gate_mode, gate_values, (cudaStream_t)stream,
+                               g_err, sizeof g_err);
 }
 
 int duo_cache_bytes(const duo_params *params, int64_t capacity, int64_t seq_len,

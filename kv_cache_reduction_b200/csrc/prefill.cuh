@@ -63,6 +63,8 @@ struct PrefillArgs {
     float *lse;            // [B][Hq][L] or null
     const float *sink_logit;
     int32_t *work_counter; // zeroed before the launch, or null for the static order
+    const __nv_bfloat16 *gate;  // output gate pre-activations or null
+    // gate layout: kGate 1 [B][L][Hq][128], kGate 2 [B][L][Hq]
     int32_t L, hq, hkv, n_qtiles, n_work, batch_pairs;
     int32_t sink, recent, window;
     float scale_log2;
@@ -125,6 +127,8 @@ __device__ __forceinline__ PfWork work_of(const PrefillArgs &a, int w) {
     return wk;
 }
 
+// kGate: 0 no output gate, 1 one gate per (head, channel), 2 one gate per head
+template <int kGate>
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_constant__ PrefillArgs a) {
     extern __shared__ __align__(16) char psmem_base[];
     char *smem = psmem_base + ((1024u - (smem_u32(psmem_base) & 1023u)) & 1023u);
@@ -415,6 +419,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             }
             if (!ok) break;
             // ------------------------------------------------------------ work-tile epilogue
+            // the output gate of this row's 64 channels (16 at a time, one chunk
+            // ahead) or of its head; the first loads overlap the waits below
+            const uint4 *gp = reinterpret_cast<const uint4 *>(
+                a.gate + (((size_t)wk.b * a.L + i) * a.hq + hq) * 128 + half * 64);
+            uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
+            float g_head = 0.f;
+            if (kGate == 1 && i < a.L) {
+                g0 = __ldg(gp);
+                g1 = __ldg(gp + 1);
+            } else if (kGate == 2 && i < a.L) {
+                g_head = __bfloat162float(a.gate[((size_t)wk.b * a.L + i) * a.hq + hq]);
+            }
             red_sum[h][half][r] = l_run;
             __syncwarp();
             if (lane == 0) mbar_arrive(&xsum[h]);
@@ -424,6 +440,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             tc_fence_after();
             const float l_row = red_sum[h][0][r] + red_sum[h][1][r];
             const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+            // o * sigmoid(g): one factor per row, or one per channel below
+            const float row_mul = kGate == 2 ? inv_l / (1.f + ex2_approx(-g_head * kLog2eF)) : inv_l;
             // O / l leaves through this warp's 1 KB staging buffer as 32-row x
             // 16-column TMA stores (rows past L are clipped by the tensor map):
             // coalesced by the copy engine instead of 32 scattered rows per store
@@ -437,11 +455,24 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 reg_fence32(orr);
 #pragma unroll
                 for (int c16 = 0; c16 < 32; c16 += 16) {
+                    uint4 n0 = g0, n1 = g1;                // the next chunk's gates
+                    if (kGate == 1 && cb + c16 + 16 < 64 && i < a.L) {
+                        n0 = __ldg(gp + (cb + c16 + 16) / 8);
+                        n1 = __ldg(gp + (cb + c16 + 16) / 8 + 1);
+                    }
                     if (lane == 0) bulk_wait_read_all();   // the previous chunk has left the buffer
                     __syncwarp();
                     auto nb = [&](int e) {
-                        return pack_bf16x2(__uint_as_float(orr[c16 + e]) * inv_l,
-                                           __uint_as_float(orr[c16 + e + 1]) * inv_l);
+                        float m0 = row_mul, m1 = row_mul;
+                        if (kGate == 1) {
+                            // channels e, e + 1 of the chunk: one bf16 pair of its gates
+                            const uint4 q4 = e < 8 ? g0 : g1;
+                            const uint32_t w = (e & 7) < 2 ? q4.x : (e & 7) < 4 ? q4.y : (e & 7) < 6 ? q4.z : q4.w;
+                            m0 = inv_l / (1.f + ex2_approx(-__uint_as_float(w << 16) * kLog2eF));
+                            m1 = inv_l / (1.f + ex2_approx(-__uint_as_float(w & 0xffff0000u) * kLog2eF));
+                        }
+                        return pack_bf16x2(__uint_as_float(orr[c16 + e]) * m0,
+                                           __uint_as_float(orr[c16 + e + 1]) * m1);
                     };
                     const uint4 v0 = make_uint4(nb(0), nb(2), nb(4), nb(6));
                     const uint4 v1 = make_uint4(nb(8), nb(10), nb(12), nb(14));
@@ -454,6 +485,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                         tma_store_4d(&a.tm_o, stage, half * 64 + cb + c16, hq, row0, wk.b);
                         bulk_commit_group();
                     }
+                    g0 = n0;
+                    g1 = n1;
                 }
             }
             if (a.lse != nullptr && i < a.L && half == 0)
@@ -523,8 +556,8 @@ inline bool make_tmap(CUtensorMap *m, const void *base, int B, int L, int H, int
 
 inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_full, int sink,
                           int ring, const void *q, const void *k, const void *v, int32_t L, void *out,
-                          float *lse, int32_t *work_counter, cudaStream_t stream, char *err,
-                          size_t err_len) {
+                          float *lse, int32_t *work_counter, int gate_mode, const void *gate,
+                          cudaStream_t stream, char *err, size_t err_len) {
     PrefillArgs a;
     memset(&a, 0, sizeof a);
     const int B = p->batch;
@@ -537,6 +570,7 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     }
     a.lse = lse;
     a.sink_logit = p->sink_logit;
+    a.gate = (const __nv_bfloat16 *)gate;
     a.L = L;
     a.hq = p->num_q_heads;
     a.hkv = p->num_kv_heads;
@@ -547,16 +581,17 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     a.scale_log2 = p->softmax_scale * kLog2eF;
     for (int g = 0; g < p->num_kv_heads; ++g)
         a.kind[g] = sliding ? kKindSliding : (is_full[g] ? kKindFull : kKindStreaming);
-    static bool smem_set[64] = {};
+    void (*kernel)(PrefillArgs) = gate_mode == 1 ? prefill_fwd<1> : gate_mode == 2 ? prefill_fwd<2> : prefill_fwd<0>;
+    static bool smem_set[3][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !smem_set[dev]) {
-        if (cudaFuncSetAttribute(prefill_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kPfSmem) != cudaSuccess) {
+    if (dev < 0 || dev >= 64 || !smem_set[gate_mode][dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmem) !=
+            cudaSuccess) {
             snprintf(err, err_len, "cudaFuncSetAttribute(prefill_fwd) failed");
             return DUO_ERR_CUDA;
         }
-        if (dev >= 0 && dev < 64) smem_set[dev] = true;
+        if (dev >= 0 && dev < 64) smem_set[gate_mode][dev] = true;
     }
     a.batch_pairs = B * (p->num_q_heads / 2);
     const int64_t n_work = (int64_t)a.batch_pairs * a.n_qtiles;
@@ -574,7 +609,7 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
         snprintf(err, err_len, "zeroing the prefill work counter failed");
         return DUO_ERR_CUDA;
     }
-    prefill_fwd<<<grid, kPfThreads, kPfSmem, stream>>>(a);
+    kernel<<<grid, kPfThreads, kPfSmem, stream>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(err, err_len, "prefill_fwd launch: %s", cudaGetErrorString(e));

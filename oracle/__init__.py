@@ -211,6 +211,53 @@ def attn_decode(layer: Layer, cache: Cache, q, rows=None):
     return out, lse
 
 
+# ------------------------------------------------------------------ output gate
+# Laguna's optional attention output gate (the Laguna attention article
+# "深入理解Laguna的注意力机制", section on attention output gating: one gate per
+# (head, channel) or one per head broadcast over the channels; the Laguna XS
+# 2.1 sliding-window article: the g_proj gate on the attention output).  The
+# pages do not name the activation; the reading taken is the logistic sigmoid,
+# applied to the normalised attention output: out * 1 / (1 + exp(-g)).
+
+GATE_NONE, GATE_PER_ELEMENT, GATE_PER_HEAD = 0, 1, 2
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def sigmoid(x: np.ndarray) -> np.ndarray:
+    """The logistic function in float64 (exp overflow for very negative x gives 0)."""
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-x))
+
+
+def gate_prefill(out: np.ndarray, gate, mode: int, L: int, Hq: int, rows=None) -> np.ndarray:
+    """Gated prefill output.  out: [n][D] float64 rows as attn_prefill returns
+    them (ids (b*Hq + h)*L + i); gate: bf16 bits [B][L][Hq][D] (per element) or
+    [B][L][Hq] (per head)."""
+    if mode == GATE_NONE:
+        return out
+    g = bf16_bits_to_f64(gate)
+    r = np.arange(out.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
+    i, h, b = r % L, (r // L) % Hq, r // (L * Hq)
+    gv = g[b, i, h, :] if mode == GATE_PER_ELEMENT else g[b, i, h][:, None]
+    return out * sigmoid(gv)
+
+
+def gate_decode(out: np.ndarray, gate, mode: int, Hq: int, rows=None) -> np.ndarray:
+    """Gated decode output.  out: [n][D] rows with ids b*Hq + h; gate: bf16 bits
+    [B][Hq][D] (per element) or [B][Hq] (per head)."""
+    if mode == GATE_NONE:
+        return out
+    g = bf16_bits_to_f64(gate)
+    r = np.arange(out.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
+    h, b = r % Hq, r // Hq
+    gv = g[b, h, :] if mode == GATE_PER_ELEMENT else g[b, h][:, None]
+    return out * sigmoid(gv)
+
+
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
 

@@ -129,7 +129,7 @@ def test_decode_argument_checks(lib):
     pc = p.as_c()
     c = duo._Cache(0x1000, 0x1000, 64, 0x1000, 0x1000, 0x1000, 0x1000)
     call = lambda msl, q=0x1000, out=0x1000, ws=0x1000, wsb=1 << 30: lib.duo_attn_decode(
-        ctypes.byref(pc), ctypes.byref(c), q, msl, out, None, ws, wsb, None)
+        ctypes.byref(pc), ctypes.byref(c), q, msl, out, None, ws, wsb, None, None)
     assert call(65) == duo.DUO_ERR_INVALID_ARG      # longer than the capacity
     assert call(-1) == duo.DUO_ERR_INVALID_ARG
     assert call(10, q=0) == duo.DUO_ERR_INVALID_ARG
@@ -141,15 +141,34 @@ def test_prefill_argument_checks(lib):
     pc = p.as_c()
     f = lib.duo_attn_prefill
     a = 0x1000
-    assert f(ctypes.byref(pc), a, a, a, -5, a, None, None, 0, None) == duo.DUO_ERR_INVALID_ARG
-    assert f(ctypes.byref(pc), a, 0, a, 16, a, None, None, 0, None) == duo.DUO_ERR_INVALID_ARG
-    assert f(ctypes.byref(pc), a, a, a, 16, a, 0x1004, None, 0, None) == duo.DUO_ERR_INVALID_ARG
-    assert f(ctypes.byref(pc), 0, 0, 0, 0, 0, None, None, 0, None) == duo.DUO_OK   # empty prefill
+    assert f(ctypes.byref(pc), a, a, a, -5, a, None, None, 0, None, None) == duo.DUO_ERR_INVALID_ARG
+    assert f(ctypes.byref(pc), a, 0, a, 16, a, None, None, 0, None, None) == duo.DUO_ERR_INVALID_ARG
+    assert f(ctypes.byref(pc), a, a, a, 16, a, 0x1004, None, 0, None, None) == duo.DUO_ERR_INVALID_ARG
+    assert f(ctypes.byref(pc), 0, 0, 0, 0, 0, None, None, 0, None, None) == duo.DUO_OK   # empty prefill
     need = duo.duo_prefill_workspace_bytes()
     assert need >= 4
     # a workspace that is too small or misaligned is refused before anything runs
-    assert f(ctypes.byref(pc), a, a, a, 16, a, None, 0x2000, need - 1, None) == duo.DUO_ERR_WORKSPACE
-    assert f(ctypes.byref(pc), a, a, a, 16, a, None, 0x2008, need, None) == duo.DUO_ERR_WORKSPACE
+    assert f(ctypes.byref(pc), a, a, a, 16, a, None, 0x2000, need - 1, None, None) == duo.DUO_ERR_WORKSPACE
+    assert f(ctypes.byref(pc), a, a, a, 16, a, None, 0x2008, need, None, None) == duo.DUO_ERR_WORKSPACE
+
+
+def test_gate_argument_checks(lib):
+    """A bad output gate is refused on the host before anything runs."""
+    p = _params()
+    pc = p.as_c()
+    a = 0x1000
+    f = lib.duo_attn_prefill
+    for mode, values in ((3, a), (-1, a), (duo.DUO_GATE_PER_ELEMENT, None),
+                         (duo.DUO_GATE_PER_HEAD, 0x1008)):
+        g = duo._Gate(mode, values)
+        assert f(ctypes.byref(pc), a, a, a, 16, a, None, None, 0, ctypes.byref(g), None) == \
+            duo.DUO_ERR_INVALID_ARG, (mode, values)
+        c = duo._Cache(a, a, 64, a, a, a, a)
+        assert lib.duo_attn_decode(ctypes.byref(pc), ctypes.byref(c), a, 10, a, None, a, 1 << 30,
+                                   ctypes.byref(g), None) == duo.DUO_ERR_INVALID_ARG
+    # mode NONE ignores the values pointer: the empty prefill still succeeds
+    g = duo._Gate(duo.DUO_GATE_NONE, None)
+    assert f(ctypes.byref(pc), 0, 0, 0, 0, 0, None, None, 0, ctypes.byref(g), None) == duo.DUO_OK
 
 
 def test_workspace_size_is_host_arithmetic(lib):

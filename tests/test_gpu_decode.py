@@ -160,3 +160,24 @@ def test_decode_b32_workload_full_size(cuda_device):
     rh = rng.integers(0, 256, size=w.batch).tolist()
     cache = random_cache(p, w.seq_len, [w.seq_len] * w.batch, rh, seed=w.seed)
     check_decode(p, o, cache, seed=w.seed + 5, max_seq_len=w.seq_len)
+
+
+@pytest.mark.parametrize("mode", ["per_element", "per_head"])
+def test_decode_output_gate(cuda_device, mode):
+    """out * sigmoid(g) applied in the split merge, against the oracle's gate."""
+    B = 3
+    p, o = layers(B, full_mask=(1, 0, 0, 1, 0, 1, 1, 0))
+    seq = [5, 700, 3000]
+    cache = random_cache(p, 3000, seq, [0, 11, 200], seed=60)
+    q = inputs.randn_bf16((B, 48, 128), 61, "cuda")
+    shape = (B, 48, 128) if mode == "per_element" else (B, 48)
+    g = (inputs.randn_f32(shape, 62) * 2.5).to("cuda", torch.bfloat16)
+    out = torch.empty((B, 48, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, 48), dtype=torch.float32, device="cuda")
+    duo.duo_attn_decode(p, cache, q, 3000, out, lse, duo.workspace_for(p, 3000), gate=g)
+    torch.cuda.synchronize()
+    assert duo.duo_get_device_status() == duo.DUO_OK
+    ref_o, ref_l = oracle.attn_decode(o, host_cache(o, cache), inputs.bits(q))
+    gm = oracle.GATE_PER_ELEMENT if mode == "per_element" else oracle.GATE_PER_HEAD
+    ref_g = oracle.gate_decode(ref_o, inputs.bits(g), gm, 48)
+    assert_close(out, ref_g.reshape(B, 48, 128), lse, ref_l.reshape(B, 48), mode)

@@ -181,3 +181,24 @@ def test_sliding_32k_workload_sampled(cuda_device):
     ref_o, ref_l = oracle.attn_prefill(o, inputs.bits(q), inputs.bits(k), inputs.bits(v), rows=rows)
     compare_rows(out, lse, ref_o, ref_l, rows, w.batch, 48, w.seq_len, "sliding_32k")
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("mode", ["per_element", "per_head"])
+@pytest.mark.parametrize("L", [129, 300])
+def test_prefill_output_gate(cuda_device, mode, L):
+    """out * sigmoid(g) fused into the epilogue, against the oracle's gate."""
+    B = 2
+    p, o = layers(B, full_mask=(1, 0, 0, 1, 0, 1, 1, 0))
+    q, k, v = make_qkv(B, L, 48)
+    shape = (B, L, 48, 128) if mode == "per_element" else (B, L, 48)
+    g = (inputs.randn_f32(shape, 49) * 2.5).to("cuda", torch.bfloat16)
+    out = torch.full((B, L, 48, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, 48, L), dtype=torch.float32, device="cuda")
+    ws = torch.empty(duo.duo_prefill_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    duo.duo_attn_prefill(p, q, k, v, out, lse, workspace=ws, gate=g)
+    torch.cuda.synchronize()
+    assert duo.duo_get_device_status() == duo.DUO_OK
+    ref_o, ref_l = oracle.attn_prefill(o, inputs.bits(q), inputs.bits(k), inputs.bits(v))
+    gm = oracle.GATE_PER_ELEMENT if mode == "per_element" else oracle.GATE_PER_HEAD
+    ref_g = oracle.gate_prefill(ref_o, inputs.bits(g), gm, L, 48)
+    assert_close(out.permute(0, 2, 1, 3).reshape(-1, 128), ref_g, lse.reshape(-1), ref_l, mode)

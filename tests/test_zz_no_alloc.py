@@ -78,6 +78,6 @@ def test_static_scratch_rejects_layers_that_do_not_fit(cuda_device):
     lib = duo.load_library()
     pc = p.as_c()
     rc = lib.duo_attn_decode_static(ctypes.byref(pc), ctypes.byref(fake), 0x10000, 4096, 0x10000,
-                                    None, None)
+                                    None, None, None)
     assert rc == duo.DUO_ERR_WORKSPACE
     assert str(need) in duo.duo_last_error()
