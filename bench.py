@@ -403,6 +403,48 @@ class Prefill:
                 "window": self.w.window, "full_mask": list(self.w.full_mask)}
 
 
+class Prep:
+    """The fused query/key preparation + append of a 16384-token prompt on the
+    prefill_16k layer (2 of 8 KV heads full): RMSNorm + YaRN RoPE of q and k in
+    place, prepared k and v appended to the cache.  HBM-bound: GB/s of the
+    bytes it must move (q and k read and written, the surviving K/V rows
+    written, their v rows read)."""
+
+    APPENDS = 64                      # capacity in prompts; the cache is reset when full
+
+    def __init__(self, rank: int):
+        w = self.w = inputs.workload("prefill_16k")
+        B, L = w.batch, w.seq_len
+        seed = rank_seed(w.seed, rank)
+        self.params = duo.DuoParams(B, 48, 8, 128, inputs.SINK, inputs.RECENT, 0, 128 ** -0.5,
+                                    w.full_mask, None)
+        self.cache = duo.DuoCache.allocate(self.params, L * self.APPENDS)
+        self.q = inputs.randn_bf16((B, L, 48, 128), seed, "cuda")
+        self.k = inputs.randn_bf16((B, L, 8, 128), seed + 1, "cuda")
+        self.v = inputs.randn_bf16((B, L, 8, 128), seed + 2, "cuda")
+        self.prep = duo.DuoQKPrep(
+            q_norm_weight=(1 + 0.1 * inputs.randn_f32((128,), seed + 3)).to("cuda", torch.bfloat16),
+            k_norm_weight=(1 + 0.1 * inputs.randn_f32((128,), seed + 4)).to("cuda", torch.bfloat16))
+        self.appends = 0
+        n_full, n_ring = self.params.n_full, self.params.n_ring
+        kept = B * (n_full * L + n_ring * inputs.RECENT)   # rows each later append keeps
+        self.bytes = 2 * (self.q.numel() + self.k.numel()) * 2 + 3 * kept * 256
+        self.launches_per_step = 2      # qk_prep_append + kv_append_commit
+        self.unit = "GB/s"
+        self.kernel = "qk_prep_append"
+
+    def step(self):
+        if self.appends == self.APPENDS:
+            self.cache.seq_len.zero_()
+            self.cache.ring_head.zero_()
+            self.appends = 0
+        duo.duo_kv_append_prep(self.params, self.cache, self.prep, self.q, self.k, self.v)
+        self.appends += 1
+
+    def config(self):
+        return {"workload": "prep_16k: RMSNorm + YaRN RoPE of q/k in place + append, B=1, 16384 tokens"}
+
+
 class DecodeSmall:
     """B=1: a 1024-token prompt is prefilled and appended, then each step
     appends one token and decodes it (full heads {0,3,5,6}).  Latency-bound:
@@ -441,7 +483,7 @@ class DecodeSmall:
         return {"workload": "decode_small: B=1, 1024-token prompt, then append one token + decode per step"}
 
 
-WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40, "decode_small": DecodeSmall,
+WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40, "decode_small": DecodeSmall, "prep_16k": Prep,
              "prefill_16k": lambda rank: Prefill(rank, "prefill_16k"),
              "sliding_32k": lambda rank: Prefill(rank, "sliding_32k")}
 
@@ -578,7 +620,7 @@ def run_ours(args, world, rank):
         del wl
         torch.cuda.empty_cache()
         sec = {}
-        for name in ("stack40", "prefill_16k", "sliding_32k", "decode_small"):
+        for name in ("stack40", "prefill_16k", "sliding_32k", "prep_16k", "decode_small"):
             w2 = WORKLOADS[name](rank)
             st = max(3, min(args.steps, 10))
             ps, ck = measure(w2, st, args.warmup, world)

@@ -146,6 +146,51 @@ DUO_API int duo_kv_append(const duo_params *params, const duo_cache *cache, cons
  * scheduling (the same for every layer). */
 DUO_API size_t duo_prefill_workspace_bytes(void);
 
+/* Query/key preparation fused into the append (Laguna attention article
+ * "深入理解Laguna的注意力机制", section on YaRN dynamic RoPE: the
+ * full-attention layers' rope parameters; Laguna XS 2.1 sliding-window
+ * article, section on its attention optimisations: RMSNorm of the queries and
+ * keys before the rotary embedding).  Per head row x of D = 128 channels:
+ *   y = x / sqrt(mean(x^2) + rms_eps) * w        (w: the norm weight, or 1)
+ *   then the rotary embedding at the token's cache position p, rotating the
+ *   pairs (y[i], y[i + 64]), i < 64, by the angle p * inv_freq[i]:
+ *   out[i]      = (y[i] cos a - y[i + 64] sin a) * attention_factor
+ *   out[i + 64] = (y[i + 64] cos a + y[i] sin a) * attention_factor
+ * inv_freq follows YaRN ("NTK-by-parts"): with base theta and D = 128,
+ * f_i = theta^(-2i/D); dimensions that turn more than beta_fast times over
+ * original_max_position keep f_i, those that turn fewer than beta_slow times
+ * use f_i / rope_factor, and a linear ramp over the dimension index blends the
+ * two in between (bounds floor / ceil of D ln(original_max_position /
+ * (2 pi beta)) / (2 ln theta)).  rope_factor = 1 gives plain RoPE.  The
+ * pages' full-attention values: theta 500000, factor 64, original 4096,
+ * beta_fast 64, beta_slow 1, attention_factor 1.  Which half-pairing the
+ * rotation uses, and the norm epsilon, are not on the pages: the (i, i + 64)
+ * pairing and eps 1e-6 are this library's readings. */
+typedef struct {
+    float rope_theta;
+    float rope_factor;
+    int32_t original_max_position;
+    float beta_fast;
+    float beta_slow;
+    float attention_factor;
+    float rms_eps;
+    const void *q_norm_weight;  /* device bf16 [D], or NULL for unit weight */
+    const void *k_norm_weight;  /* device bf16 [D], or NULL for unit weight */
+} duo_qk_prep;
+
+/* duo_kv_append with the query/key preparation above fused in: for each
+ * sequence b and token t (position p = seq_len[b] + t), every head row of q
+ * [B][n_new][Hq][D] and k [B][n_new][Hkv][D] is normalised and rotated IN
+ * PLACE (so that duo_attn_prefill / duo_attn_decode read the prepared
+ * tensors), and the prepared k with v is appended exactly as duo_kv_append
+ * appends it.  Results are rounded to bf16 once, after the rotation.  Errors
+ * as duo_kv_append; a NULL prep, a non-positive theta, rope_factor < 1,
+ * original_max_position < 1, beta_slow <= 0, beta_fast < beta_slow or
+ * rms_eps < 0 is DUO_ERR_INVALID_ARG. */
+DUO_API int duo_kv_append_prep(const duo_params *params, const duo_cache *cache,
+                               const duo_qk_prep *prep, void *q, void *k, const void *v,
+                               int32_t n_new, void *stream);
+
 /* Prefill attention over a sequence that starts at position 0 (empty cache).
  * q: device bf16 [B][L][Hq][D]; k, v: device bf16 [B][L][Hkv][D]; L = seq_len.
  * out: device bf16 [B][L][Hq][D].  lse: device fp32 [B][Hq][L] (natural-log

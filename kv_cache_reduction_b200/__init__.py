@@ -35,7 +35,7 @@ DUO_ERR_TIMEOUT = -5
 DUO_ERR_CAPACITY = -6
 DUO_ERR_DEVICE = -7
 
-EXPORTED = ("duo_kv_append", "duo_prefill_workspace_bytes", "duo_attn_prefill",
+EXPORTED = ("duo_kv_append", "duo_kv_append_prep", "duo_prefill_workspace_bytes", "duo_attn_prefill",
             "duo_decode_workspace_bytes", "duo_attn_decode",
             "duo_attn_decode_static", "duo_cache_bytes", "duo_get_device_status",
             "duo_status_string", "duo_last_error")
@@ -75,6 +75,36 @@ def _gate(gate: Optional[torch.Tensor], out: torch.Tensor):
     return ctypes.byref(_Gate(mode, _ptr(gate)))
 
 
+class _Prep(ctypes.Structure):
+    _fields_ = [("rope_theta", ctypes.c_float), ("rope_factor", ctypes.c_float),
+                ("original_max_position", ctypes.c_int32), ("beta_fast", ctypes.c_float),
+                ("beta_slow", ctypes.c_float), ("attention_factor", ctypes.c_float),
+                ("rms_eps", ctypes.c_float), ("q_norm_weight", ctypes.c_void_p),
+                ("k_norm_weight", ctypes.c_void_p)]
+
+
+@dataclass
+class DuoQKPrep:
+    """RMSNorm + YaRN RoPE of the new queries and keys (duo_qk_prep).  The
+    defaults are the full-attention layers' rope parameters printed on the
+    Laguna attention page; eps 1e-6 is a reading.  Norm weights: device bf16
+    [128] tensors or None (unit weight)."""
+    rope_theta: float = 500000.0
+    rope_factor: float = 64.0
+    original_max_position: int = 4096
+    beta_fast: float = 64.0
+    beta_slow: float = 1.0
+    attention_factor: float = 1.0
+    rms_eps: float = 1e-6
+    q_norm_weight: Optional[torch.Tensor] = None
+    k_norm_weight: Optional[torch.Tensor] = None
+
+    def as_c(self) -> _Prep:
+        return _Prep(self.rope_theta, self.rope_factor, self.original_max_position, self.beta_fast,
+                     self.beta_slow, self.attention_factor, self.rms_eps,
+                     _ptr(self.q_norm_weight), _ptr(self.k_norm_weight))
+
+
 class _Params(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
@@ -110,6 +140,8 @@ def load_library(path: str = LIBRARY_PATH) -> ctypes.CDLL:
     P, C, vp = ctypes.POINTER(_Params), ctypes.POINTER(_Cache), ctypes.c_void_p
     lib.duo_kv_append.argtypes = [P, C, vp, vp, ctypes.c_int32, vp]
     lib.duo_kv_append.restype = ctypes.c_int
+    lib.duo_kv_append_prep.argtypes = [P, C, ctypes.POINTER(_Prep), vp, vp, vp, ctypes.c_int32, vp]
+    lib.duo_kv_append_prep.restype = ctypes.c_int
     lib.duo_prefill_workspace_bytes.argtypes = []
     lib.duo_prefill_workspace_bytes.restype = ctypes.c_size_t
     G = ctypes.POINTER(_Gate)
@@ -227,6 +259,17 @@ def duo_kv_append(params: DuoParams, cache: DuoCache, k: torch.Tensor, v: torch.
     p, c = params.as_c(), cache.as_c()
     _check(load_library().duo_kv_append(ctypes.byref(p), ctypes.byref(c), _ptr(k), _ptr(v), n_new,
                                         _stream(stream)))
+
+
+def duo_kv_append_prep(params: DuoParams, cache: DuoCache, prep: DuoQKPrep, q: torch.Tensor,
+                       k: torch.Tensor, v: torch.Tensor, n_new: Optional[int] = None,
+                       stream=None) -> None:
+    """RMSNorm + YaRN RoPE of q [B][n][Hq][D] and k [B][n][Hkv][D] in place at
+    positions seq_len[b] + t, then the append of the prepared k with v."""
+    n_new = int(k.shape[1]) if n_new is None else int(n_new)
+    p, c, pr = params.as_c(), cache.as_c(), prep.as_c()
+    _check(load_library().duo_kv_append_prep(ctypes.byref(p), ctypes.byref(c), ctypes.byref(pr),
+                                             _ptr(q), _ptr(k), _ptr(v), n_new, _stream(stream)))
 
 
 def duo_prefill_workspace_bytes() -> int:

@@ -12,6 +12,7 @@
 #include "kv_append.cuh"
 #include "prefill.cuh"
 #include "ptx.cuh"
+#include "qk_prep.cuh"
 
 namespace {
 
@@ -223,6 +224,39 @@ bool cache_tmap(CUtensorMap *m, void *base, int64_t rows) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Checks an append's arguments and fills the scatter arguments (nothing is
+// launched); DUO_OK with n_new == 0 means there is nothing to do.
+int append_args(const duo_params *params, const duo_cache *cache, const void *k, const void *v,
+                int32_t n_new, Layout *L, duo::AppendArgs *a) {
+    int rc = check_params(params, L);
+    if (rc) return rc;
+    if ((rc = check_cache(cache, *L))) return rc;
+    if (n_new < 0 || n_new > kMaxPos) return fail(DUO_ERR_INVALID_ARG, "n_new must be in [0, 2^30]");
+    if (n_new == 0) return DUO_OK;
+    if (!k || !v) return fail(DUO_ERR_INVALID_ARG, "k / v is NULL");
+    if (!aligned16(k) || !aligned16(v)) return fail(DUO_ERR_INVALID_ARG, "k / v must be 16-byte aligned");
+    if ((rc = check_device(nullptr))) return rc;
+    a->k = (const uint4 *)k;
+    a->v = (const uint4 *)v;
+    a->full_k = (uint4 *)cache->full_k;
+    a->full_v = (uint4 *)cache->full_v;
+    a->strm_k = (uint4 *)cache->strm_k;
+    a->strm_v = (uint4 *)cache->strm_v;
+    a->seq_len = cache->seq_len;
+    a->ring_head = cache->ring_head;
+    a->capacity = L->n_full > 0 ? cache->capacity : 0;
+    a->batch = params->batch;
+    a->n_new = n_new;
+    a->hkv = params->num_kv_heads;
+    a->n_full = L->n_full;
+    a->n_ring = L->n_ring;
+    a->sink = L->sink;
+    a->ring = L->ring;
+    a->slots = L->slots;
+    a->heads = L->heads;
+    return DUO_OK;
+}
+
 size_t workspace_bytes(const duo_params *p, const DecodePlan &d) {
     return (size_t)p->batch * p->num_kv_heads * d.max_splits * duo::kPartFloats * sizeof(float);
 }
@@ -250,39 +284,69 @@ const char *duo_status_string(int code) {
 int duo_kv_append(const duo_params *params, const duo_cache *cache, const void *k, const void *v,
                   int32_t n_new, void *stream) {
     Layout L;
-    int rc = check_params(params, &L);
-    if (rc) return rc;
-    if ((rc = check_cache(cache, L))) return rc;
-    if (n_new < 0 || n_new > kMaxPos) return fail(DUO_ERR_INVALID_ARG, "n_new must be in [0, 2^30]");
-    if (n_new == 0) return DUO_OK;
-    if (!k || !v) return fail(DUO_ERR_INVALID_ARG, "k / v is NULL");
-    if (!aligned16(k) || !aligned16(v)) return fail(DUO_ERR_INVALID_ARG, "k / v must be 16-byte aligned");
-    if ((rc = check_device(nullptr))) return rc;
     duo::AppendArgs a{};
-    a.k = (const uint4 *)k;
-    a.v = (const uint4 *)v;
-    a.full_k = (uint4 *)cache->full_k;
-    a.full_v = (uint4 *)cache->full_v;
-    a.strm_k = (uint4 *)cache->strm_k;
-    a.strm_v = (uint4 *)cache->strm_v;
-    a.seq_len = cache->seq_len;
-    a.ring_head = cache->ring_head;
-    a.capacity = L.n_full > 0 ? cache->capacity : 0;
-    a.batch = params->batch;
-    a.n_new = n_new;
-    a.hkv = params->num_kv_heads;
-    a.n_full = L.n_full;
-    a.n_ring = L.n_ring;
-    a.sink = L.sink;
-    a.ring = L.ring;
-    a.slots = L.slots;
-    a.heads = L.heads;
+    int rc = append_args(params, cache, k, v, n_new, &L, &a);
+    if (rc || n_new == 0) return rc;
     cudaStream_t st = (cudaStream_t)stream;
     const int64_t vecs = (int64_t)params->batch * n_new * params->num_kv_heads * duo::kVecPerRow;
     const int64_t blocks = (vecs + 255) / 256;
     if (blocks > INT32_MAX) return fail(DUO_ERR_INVALID_ARG, "append too large for one launch");
     duo::kv_append_scatter<<<(unsigned)blocks, 256, 0, st>>>(a);
     if ((rc = launch_status("kv_append_scatter"))) return rc;
+    duo::kv_append_commit<<<(params->batch + 127) / 128, 128, 0, st>>>(
+        cache->seq_len, cache->ring_head, params->batch, n_new, L.sink, L.ring);
+    return launch_status("kv_append_commit");
+}
+
+// YaRN inverse frequencies ("NTK-by-parts"), in double: f_i = theta^(-2i/D);
+// the dimensions between the correction bounds of beta_fast and beta_slow blend
+// f_i (extrapolation) and f_i / factor (interpolation) along a linear ramp.
+static void yarn_inv_freq(const duo_qk_prep *p, double *inv) {
+    const double d = duo::kD, theta = p->rope_theta, s = p->rope_factor;
+    const double orig = p->original_max_position;
+    const double two_pi = 6.283185307179586476925286766559;
+    auto bound = [&](double beta) { return d * std::log(orig / (beta * two_pi)) / (2.0 * std::log(theta)); };
+    double low = std::floor(bound(p->beta_fast)), high = std::ceil(bound(p->beta_slow));
+    low = std::max(low, 0.0);
+    high = std::min(high, d - 1.0);
+    if (high == low) high += 0.001;
+    for (int i = 0; i < duo::kD / 2; ++i) {
+        const double f = std::pow(theta, -2.0 * i / d);
+        const double ramp = std::min(1.0, std::max(0.0, (i - low) / (high - low)));
+        const double keep = 1.0 - ramp;             // share of the unscaled frequency
+        inv[i] = f / s * (1.0 - keep) + f * keep;
+    }
+}
+
+int duo_kv_append_prep(const duo_params *params, const duo_cache *cache, const duo_qk_prep *prep,
+                       void *q, void *k, const void *v, int32_t n_new, void *stream) {
+    if (!prep) return fail(DUO_ERR_INVALID_ARG, "prep is NULL");
+    if (!(prep->rope_theta > 1.f) || !(prep->rope_factor >= 1.f) || prep->original_max_position < 1 ||
+        !(prep->beta_slow > 0.f) || !(prep->beta_fast >= prep->beta_slow) || !(prep->rms_eps >= 0.f) ||
+        !std::isfinite(prep->attention_factor) || !std::isfinite(prep->rope_theta) ||
+        !std::isfinite(prep->rope_factor) || !std::isfinite(prep->beta_fast))
+        return fail(DUO_ERR_INVALID_ARG, "rope / norm parameters out of range");
+    if ((prep->q_norm_weight && !aligned16(prep->q_norm_weight)) ||
+        (prep->k_norm_weight && !aligned16(prep->k_norm_weight)))
+        return fail(DUO_ERR_INVALID_ARG, "norm weights must be 16-byte aligned");
+    Layout L;
+    duo::PrepArgs a{};
+    int rc = append_args(params, cache, k, v, n_new, &L, &a.app);
+    if (rc || n_new == 0) return rc;
+    if (!q || !aligned16(q)) return fail(DUO_ERR_INVALID_ARG, "q must be a 16-byte aligned pointer");
+    const int64_t blocks = (int64_t)params->batch * n_new;
+    if (blocks > INT32_MAX) return fail(DUO_ERR_INVALID_ARG, "append too large for one launch");
+    a.q = (uint4 *)q;
+    a.kw = (uint4 *)k;
+    a.q_w = (const __nv_bfloat16 *)prep->q_norm_weight;
+    a.k_w = (const __nv_bfloat16 *)prep->k_norm_weight;
+    yarn_inv_freq(prep, a.inv_freq);
+    a.attention_factor = prep->attention_factor;
+    a.rms_eps = prep->rms_eps;
+    a.hq = params->num_q_heads;
+    cudaStream_t st = (cudaStream_t)stream;
+    duo::qk_prep_append<<<(unsigned)blocks, duo::kPrepThreads, 0, st>>>(a);
+    if ((rc = launch_status("qk_prep_append"))) return rc;
     duo::kv_append_commit<<<(params->batch + 127) / 128, 128, 0, st>>>(
         cache->seq_len, cache->ring_head, params->batch, n_new, L.sink, L.ring);
     return launch_status("kv_append_commit");
