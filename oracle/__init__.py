@@ -67,6 +67,8 @@ def _load():
         lib.oracle_kv_append.restype = ctypes.c_int
         lib.oracle_attn_decode.argtypes = [P, C, vp, vp, i64, vp, vp]
         lib.oracle_attn_decode.restype = ctypes.c_int
+        lib.oracle_attn_decode_block.argtypes = [P, C, vp, vp, vp, ctypes.c_int32, vp, i64, vp, vp]
+        lib.oracle_attn_decode_block.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
@@ -208,6 +210,28 @@ def attn_decode(layer: Layer, cache: Cache, q, rows=None):
                                     out.ctypes.data, lse.ctypes.data)
     if rc != 0:
         raise ValueError(f"oracle_attn_decode failed ({rc})")
+    return out, lse
+
+
+def attn_decode_block(layer: Layer, cache: Cache, q, kb, vb, rows=None):
+    """Block (verify) decode against the cache before the block is appended.
+    q: [B][k][Hq][D], kb/vb: [B][k][Hkv][D] uint16 bits; query t of sequence b
+    is at position seq_len[b] + t.  rows: flat ids (b*k + t)*Hq + h.  Returns
+    (out [n][D], lse [n]) in float64."""
+    q, kb, vb = _u16(q), _u16(kb), _u16(vb)
+    B, k, Hq, D = q.shape
+    n = B * k * Hq if rows is None else len(rows)
+    r = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    p, keep = layer._c()
+    c = cache._c()
+    rc = _load().oracle_attn_decode_block(ctypes.byref(p), ctypes.byref(c), q.ctypes.data,
+                                          kb.ctypes.data, vb.ctypes.data, int(k),
+                                          None if r is None else r.ctypes.data, n,
+                                          out.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_attn_decode_block failed ({rc})")
     return out, lse
 
 

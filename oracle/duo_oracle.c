@@ -299,6 +299,86 @@ int oracle_attn_decode(const oracle_params *p, const oracle_cache *c, const uint
     return bad ? -2 : 0;
 }
 
+/* Block decode: a block of qlen query tokens (a verify block) against the
+ * cache as it stands BEFORE the block is appended.  Query t of sequence b sits
+ * at position i = n + t, n = seq_len[b], and attends to the keys its head's
+ * rule allows at i: the cached ones (a full head: rows 0..n-1; a ring head:
+ * its sink slots, and the ring slots holding a position j > i - recent, where
+ * the ring slot written d-th to last holds position n - 1 - d) and the block's
+ * own keys u <= t (positions n..i) that the same rule allows, given in kb, vb
+ * [B][qlen][Hkv][D].
+ * q: [B][qlen][Hq][D].  rows: flat ids (b*qlen + t)*Hq + h, or NULL for all. */
+int oracle_attn_decode_block(const oracle_params *p, const oracle_cache *c, const uint16_t *q,
+                             const uint16_t *kb, const uint16_t *vb, int32_t qlen,
+                             const int64_t *rows, int64_t n_rows, double *out, double *lse) {
+    const int Hq = p->num_q_heads, Hkv = p->num_kv_heads, D = p->head_dim;
+    if (Hq % Hkv || qlen < 1) return -1;
+    const int group = Hq / Hkv;
+    const int32_t n_full = count_full(p), n_ring = Hkv - n_full;
+    const int32_t S = ring_sink(p), R = ring_recent(p), slots = S + R;
+    const int64_t total = (int64_t)p->batch * qlen * Hq;
+    if (!rows) n_rows = total;
+    int64_t max_keys = 1;
+    for (int32_t b = 0; b < p->batch; ++b)
+        if (c->seq_len[b] + qlen > max_keys) max_keys = c->seq_len[b] + qlen;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)max_keys);
+        const uint16_t **vr = (const uint16_t **)malloc(sizeof(void *) * (size_t)max_keys);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t x = 0; x < n_rows; ++x) {
+            const int64_t r = rows ? rows[x] : x;
+            if (r < 0 || r >= total) { bad = 1; continue; }
+            const int h = (int)(r % Hq);
+            const int64_t t = (r / Hq) % qlen;
+            const int64_t b = r / Hq / qlen;
+            const int g = h / group;
+            const int64_t n = c->seq_len[b];
+            const int64_t i = n + t;                   /* the query's position */
+            const uint16_t *qh = q + ((b * qlen + t) * Hq + h) * D;
+            int m = 0;
+            if (oracle_head_kind(p, g) == KIND_FULL) {
+                const int64_t base = ((b * n_full + full_rank(p, g)) * c->capacity) * D;
+                for (int64_t j = 0; j < n; ++j) {
+                    s[m] = p->softmax_scale * dot_bf16(qh, c->full_k + base + j * D, D);
+                    vr[m++] = c->full_v + base + j * D;
+                }
+            } else {
+                const int64_t base = ((b * n_ring + ring_rank(p, g)) * slots) * D;
+                const int64_t n_sink = n < S ? n : S;
+                int64_t cnt = n - S;
+                if (cnt < 0) cnt = 0;
+                if (cnt > R) cnt = R;
+                for (int64_t j = 0; j < n_sink; ++j) {
+                    s[m] = p->softmax_scale * dot_bf16(qh, c->strm_k + base + j * D, D);
+                    vr[m++] = c->strm_v + base + j * D;
+                }
+                for (int64_t d = 0; d < cnt; ++d) {    /* d-th to last written: position n-1-d */
+                    const int64_t pos = n - 1 - d;
+                    if (pos <= i - R) continue;        /* outside the query's recent window */
+                    const int64_t slot = S + (((int64_t)c->ring_head[b] - 1 - d) % R + R) % R;
+                    s[m] = p->softmax_scale * dot_bf16(qh, c->strm_k + base + slot * D, D);
+                    vr[m++] = c->strm_v + base + slot * D;
+                }
+            }
+            for (int64_t u = 0; u <= t; ++u) {         /* the block's keys up to the query */
+                const int64_t j = n + u;
+                if (oracle_head_kind(p, g) != KIND_FULL && !(j < S || j > i - R)) continue;
+                const int64_t kr = ((b * qlen + u) * Hkv + g) * D;
+                s[m] = p->softmax_scale * dot_bf16(qh, kb + kr, D);
+                vr[m++] = vb + kr;
+            }
+            const int has_sink = p->sink_logit != NULL;
+            const double sigma = has_sink ? (double)p->sink_logit[h] : 0.0;
+            lse[x] = softmax_row(m, s, vr, D, has_sink, sigma, out + x * D);
+        }
+        free(s);
+        free((void *)vr);
+    }
+    return bad ? -2 : 0;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
