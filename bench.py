@@ -403,6 +403,42 @@ class Prefill:
                 "window": self.w.window, "full_mask": list(self.w.full_mask)}
 
 
+class VerifyB32(DecodeB32):
+    """Verify-block decode on decode_b32's caches: a block of 8 query tokens per
+    sequence (the DFlash verify shape) against 32768 cached tokens plus the
+    block's own keys, cache untouched.  GB/s of the bytes it must read: the
+    cached K/V rows the block's queries attend to (each read once for all 8
+    queries), the block's K/V, q and out."""
+
+    Q_LEN = 8
+    e2e_step = None          # the end-to-end and CPU legs belong to the main line
+    oracle_sample = None
+
+    def __init__(self, rank: int):
+        super().__init__(rank)
+        B, n, k = self.w.batch, self.w.seq_len, self.Q_LEN
+        seed = rank_seed(self.w.seed, rank)
+        self.qb = inputs.randn_bf16((B, k, 48, 128), seed + 6, "cuda")
+        self.kb = inputs.randn_bf16((B, k, 8, 128), seed + 7, "cuda")
+        self.vb = inputs.randn_bf16((B, k, 8, 128), seed + 8, "cuda")
+        self.outb = torch.empty_like(self.qb)
+        self.lseb = torch.empty((B, k, 48), dtype=torch.float32, device="cuda")
+        nb = duo.duo_decode_block_workspace_bytes(self.params, k, n)
+        self.wsb = torch.zeros((nb + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+        n_full, n_ring = self.params.n_full, self.params.n_ring
+        rows = B * (n_full * n + n_ring * min(n, inputs.SINK + inputs.RECENT)) + B * 8 * k
+        self.bytes = rows * 2 * 128 * 2 + 2 * self.qb.numel() * 2
+        self.kernel = "decode_block_split + decode_block_merge (one duo_attn_decode_block call)"
+
+    def step(self):
+        duo.duo_attn_decode_block(self.params, self.cache, self.qb, self.kb, self.vb, self.w.seq_len,
+                                  self.outb, self.lseb, self.wsb)
+
+    def config(self):
+        return {"workload": "verify_b32: block of 8 query tokens, B=32, context 32768, "
+                            "2 of 8 KV heads full"}
+
+
 class Prep:
     """The fused query/key preparation + append of a 16384-token prompt on the
     prefill_16k layer (2 of 8 KV heads full): RMSNorm + YaRN RoPE of q and k in
@@ -484,6 +520,7 @@ class DecodeSmall:
 
 
 WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40, "decode_small": DecodeSmall, "prep_16k": Prep,
+             "verify_b32": VerifyB32,
              "prefill_16k": lambda rank: Prefill(rank, "prefill_16k"),
              "sliding_32k": lambda rank: Prefill(rank, "sliding_32k")}
 
@@ -603,7 +640,7 @@ def run_ours(args, world, rank):
            "config": {**wl.config(), "parallelism": f"dp{world} (independent batches, no collective)"},
            "roofline": rf, "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks}
     # end to end through the public API: pinned host inputs, copies in the timed region
-    if hasattr(wl, "e2e_step"):
+    if getattr(wl, "e2e_step", None) is not None:
         h2d, d2h = wl.e2e_buffers()
         for _ in range(args.warmup):
             wl.e2e_step()
@@ -613,14 +650,14 @@ def run_ours(args, world, rank):
         res["e2e"] = {"value": round(aggregate(units(wl), world, t_e2e), 2), "unit": wl.unit,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                       "ms_per_step": round(t_e2e * 1e3, 4)}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(wl, "oracle_sample"):
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and getattr(wl, "oracle_sample", None) is not None:
         res["cpu_baseline"] = wl.oracle_sample(args.cpu_budget)
     # the other workloads of the path, on this GPU, as context for the main line
     if args.secondary and args.workload == "decode_b32":
         del wl
         torch.cuda.empty_cache()
         sec = {}
-        for name in ("stack40", "prefill_16k", "sliding_32k", "prep_16k", "decode_small"):
+        for name in ("stack40", "verify_b32", "prefill_16k", "sliding_32k", "prep_16k", "decode_small"):
             w2 = WORKLOADS[name](rank)
             st = max(3, min(args.steps, 10))
             ps, ck = measure(w2, st, args.warmup, world)

@@ -36,7 +36,8 @@ DUO_ERR_CAPACITY = -6
 DUO_ERR_DEVICE = -7
 
 EXPORTED = ("duo_kv_append", "duo_kv_append_prep", "duo_prefill_workspace_bytes", "duo_attn_prefill",
-            "duo_decode_workspace_bytes", "duo_attn_decode",
+            "duo_decode_workspace_bytes", "duo_attn_decode", "duo_decode_block_workspace_bytes",
+            "duo_attn_decode_block",
             "duo_attn_decode_static", "duo_cache_bytes", "duo_get_device_status",
             "duo_status_string", "duo_last_error")
 
@@ -152,6 +153,11 @@ def load_library(path: str = LIBRARY_PATH) -> ctypes.CDLL:
     lib.duo_attn_decode.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, vp, ctypes.c_size_t, G, vp]
     lib.duo_attn_decode.restype = ctypes.c_int
     lib.duo_attn_decode_static.argtypes = [P, C, vp, ctypes.c_int32, vp, vp, G, vp]
+    lib.duo_decode_block_workspace_bytes.argtypes = [P, ctypes.c_int32, ctypes.c_int32]
+    lib.duo_decode_block_workspace_bytes.restype = ctypes.c_size_t
+    lib.duo_attn_decode_block.argtypes = [P, C, vp, vp, vp, ctypes.c_int32, ctypes.c_int32, vp, vp, vp,
+                                          ctypes.c_size_t, G, vp]
+    lib.duo_attn_decode_block.restype = ctypes.c_int
     lib.duo_attn_decode_static.restype = ctypes.c_int
     lib.duo_cache_bytes.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(CacheStats)]
     lib.duo_cache_bytes.restype = ctypes.c_int
@@ -307,6 +313,27 @@ def duo_attn_decode(params: DuoParams, cache: DuoCache, q: torch.Tensor, max_seq
     _check(load_library().duo_attn_decode(ctypes.byref(p), ctypes.byref(c), _ptr(q), int(max_seq_len),
                                           _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
                                           _gate(gate, out), _stream(stream)))
+
+
+def duo_decode_block_workspace_bytes(params: DuoParams, q_len: int, max_seq_len: int) -> int:
+    p = params.as_c()
+    return int(load_library().duo_decode_block_workspace_bytes(ctypes.byref(p), int(q_len),
+                                                               int(max_seq_len)))
+
+
+def duo_attn_decode_block(params: DuoParams, cache: DuoCache, q: torch.Tensor, k_new: torch.Tensor,
+                          v_new: torch.Tensor, max_seq_len: int, out: torch.Tensor,
+                          lse: Optional[torch.Tensor], workspace: torch.Tensor, stream=None,
+                          gate: Optional[torch.Tensor] = None) -> None:
+    """Verify-block decode: q [B][k][Hq][D] at positions seq_len[b] + t against
+    the cache plus the block's own k_new / v_new [B][k][Hkv][D]; the cache is
+    not modified."""
+    p, c = params.as_c(), cache.as_c()
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load_library().duo_attn_decode_block(ctypes.byref(p), ctypes.byref(c), _ptr(q), _ptr(k_new),
+                                                _ptr(v_new), int(q.shape[1]), int(max_seq_len), _ptr(out),
+                                                _ptr(lse), _ptr(workspace), nbytes, _gate(gate, out),
+                                                _stream(stream)))
 
 
 def duo_attn_decode_static(params: DuoParams, cache: DuoCache, q: torch.Tensor, max_seq_len: int,

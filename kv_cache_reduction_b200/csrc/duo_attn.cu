@@ -9,6 +9,7 @@
 
 #include "duo_attn.h"
 #include "decode.cuh"
+#include "decode_block.cuh"
 #include "kv_append.cuh"
 #include "prefill.cuh"
 #include "ptx.cuh"
@@ -261,6 +262,31 @@ size_t workspace_bytes(const duo_params *p, const DecodePlan &d) {
     return (size_t)p->batch * p->num_kv_heads * d.max_splits * duo::kPartFloats * sizeof(float);
 }
 
+constexpr int kMaxBlock = 8;     // block decode: query tokens per call
+
+template <int kQ>
+int launch_block(duo::BlockArgs &a, int grid, cudaStream_t st, int64_t merge_blocks) {
+    static bool smem_set[64] = {};
+    int rc;
+    if ((rc = set_smem_once(duo::decode_block_split<kQ>, duo::BlockCfg<kQ>::Smem, "decode_block_split",
+                            smem_set)))
+        return rc;
+    duo::decode_block_split<kQ><<<(unsigned)grid, duo::kBlkThreads, duo::BlockCfg<kQ>::Smem, st>>>(a);
+    if ((rc = launch_status("decode_block_split"))) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)merge_blocks);
+    cfg.blockDim = dim3(duo::kD);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, duo::decode_block_merge<kQ>, a) != cudaSuccess)
+        return fail(DUO_ERR_CUDA, "decode_block_merge launch: %s", cudaGetErrorString(cudaGetLastError()));
+    return launch_status("decode_block_merge");
+}
+
 }  // namespace
 
 extern "C" {
@@ -497,6 +523,112 @@ int duo_cache_bytes(const duo_params *params, int64_t capacity, int64_t seq_len,
     out->active_bytes = B * (act_full + act_ring) * row;
     out->utilization = out->duo_bytes ? (double)out->active_bytes / (double)out->duo_bytes : 0.0;
     return DUO_OK;
+}
+
+// ------------------------------------------------------------------ block decode
+size_t duo_decode_block_workspace_bytes(const duo_params *params, int32_t q_len, int32_t max_seq_len) {
+    Layout L;
+    if (check_params(params, &L) || q_len < 1 || q_len > kMaxBlock || max_seq_len < 0 ||
+        max_seq_len > kMaxPos)
+        return 0;
+    int sms = 148;
+    if (check_device(&sms)) sms = 148;
+    const DecodePlan d = plan_decode(params, L, max_seq_len, sms);
+    const size_t slots = (size_t)std::max(d.splits_full, d.splits_ring) + 1;
+    return (size_t)params->batch * params->num_kv_heads * slots * (size_t)(duo::kGroup * q_len) *
+           (duo::kD + 2) * sizeof(float);
+}
+
+int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, const void *q,
+                          const void *k_new, const void *v_new, int32_t q_len, int32_t max_seq_len,
+                          void *out, float *lse, void *workspace, size_t workspace_size,
+                          const duo_gate *gate, void *stream) {
+    Layout L;
+    int rc = check_params(params, &L);
+    if (rc) return rc;
+    if ((rc = check_cache(cache, L))) return rc;
+    if (q_len < 1 || q_len > kMaxBlock)
+        return fail(DUO_ERR_UNSUPPORTED, "q_len must be in [1, %d] (got %d)", kMaxBlock, q_len);
+    int gate_mode = 0;
+    const void *gate_values = nullptr;
+    if ((rc = check_gate(gate, &gate_mode, &gate_values))) return rc;
+    if (max_seq_len < 0 || max_seq_len > kMaxPos)
+        return fail(DUO_ERR_INVALID_ARG, "max_seq_len must be in [0, 2^30]");
+    if (L.n_full > 0 && max_seq_len > cache->capacity)
+        return fail(DUO_ERR_INVALID_ARG, "max_seq_len %d exceeds capacity %lld", max_seq_len,
+                    (long long)cache->capacity);
+    if (!q || !out || !k_new || !v_new) return fail(DUO_ERR_INVALID_ARG, "q / k_new / v_new / out is NULL");
+    if (!aligned16(q) || !aligned16(out) || !aligned16(k_new) || !aligned16(v_new) || (lse && !aligned16(lse)))
+        return fail(DUO_ERR_INVALID_ARG, "q / k_new / v_new / out / lse must be 16-byte aligned");
+    if ((int64_t)params->batch * L.n_full * (L.n_full ? cache->capacity : 0) > INT32_MAX ||
+        (int64_t)params->batch * L.n_ring * L.slots > INT32_MAX)
+        return fail(DUO_ERR_UNSUPPORTED, "cache rows exceed 2^31 (tensor-map coordinates are 32-bit)");
+    int sms = 148;
+    if ((rc = check_device(&sms))) return rc;
+    const DecodePlan d = plan_decode(params, L, max_seq_len, sms);
+    const size_t need = duo_decode_block_workspace_bytes(params, q_len, max_seq_len);
+    if (!workspace || workspace_size < need || ((uintptr_t)workspace & 255u))
+        return fail(DUO_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
+                    workspace_size);
+    duo::BlockArgs a;
+    memset(&a, 0, sizeof a);
+    duo::DecodeArgs &da = a.d;
+    if (L.n_full > 0 &&
+        (!cache_tmap(&da.tm_fk, cache->full_k, (int64_t)params->batch * L.n_full * cache->capacity) ||
+         !cache_tmap(&da.tm_fv, cache->full_v, (int64_t)params->batch * L.n_full * cache->capacity)))
+        return fail(DUO_ERR_CUDA, "cuTensorMapEncodeTiled failed for the full cache");
+    if (L.n_ring > 0 &&
+        (!cache_tmap(&da.tm_rk, cache->strm_k, (int64_t)params->batch * L.n_ring * L.slots) ||
+         !cache_tmap(&da.tm_rv, cache->strm_v, (int64_t)params->batch * L.n_ring * L.slots)))
+        return fail(DUO_ERR_CUDA, "cuTensorMapEncodeTiled failed for the ring cache");
+    if (!duo::make_tmap(&a.tm_bk, k_new, params->batch, q_len, params->num_kv_heads, duo::kTok) ||
+        !duo::make_tmap(&a.tm_bv, v_new, params->batch, q_len, params->num_kv_heads, duo::kTok))
+        return fail(DUO_ERR_CUDA, "cuTensorMapEncodeTiled failed for the block keys");
+    da.seq_len = cache->seq_len;
+    da.ring_head = cache->ring_head;
+    da.sink_logit = params->sink_logit;
+    da.part = (float *)workspace;
+    da.capacity = L.n_full > 0 ? cache->capacity : 0;
+    da.batch = params->batch;
+    da.hkv = params->num_kv_heads;
+    da.n_full = L.n_full;
+    da.n_ring = L.n_ring;
+    da.sink = L.sink;
+    da.ring = L.ring;
+    da.slots = L.slots;
+    da.chunk_full = d.chunk_full;
+    da.splits_full = d.splits_full;
+    da.chunk_ring = d.chunk_ring;
+    da.splits_ring = d.splits_ring;
+    da.max_splits = std::max(d.splits_full, d.splits_ring) + 1;
+    da.n_items = (int32_t)d.items;
+    da.scale_log2 = params->softmax_scale * duo::kLog2eF;
+    da.gate = (const __nv_bfloat16 *)gate_values;
+    da.gate_mode = gate_mode;
+    da.withhold_tile = -1;
+    memcpy(da.full_head, L.full_head, sizeof da.full_head);
+    memcpy(da.ring_head_of, L.ring_head_of, sizeof da.ring_head_of);
+    da.heads = L.heads;
+    a.q = (const __nv_bfloat16 *)q;
+    a.out = (__nv_bfloat16 *)out;
+    a.lse = lse;
+    a.q_len = q_len;
+    a.n_cache_items = (int32_t)d.items;
+    a.part_slots = da.max_splits;
+    const int64_t items = d.items + (int64_t)params->batch * params->num_kv_heads;
+    const int grid = (int)std::min<int64_t>(items, sms);
+    const int64_t merge_blocks = (int64_t)params->batch * q_len * params->num_q_heads;
+    cudaStream_t st = (cudaStream_t)stream;
+    switch (q_len) {
+        case 1: return launch_block<1>(a, grid, st, merge_blocks);
+        case 2: return launch_block<2>(a, grid, st, merge_blocks);
+        case 3: return launch_block<3>(a, grid, st, merge_blocks);
+        case 4: return launch_block<4>(a, grid, st, merge_blocks);
+        case 5: return launch_block<5>(a, grid, st, merge_blocks);
+        case 6: return launch_block<6>(a, grid, st, merge_blocks);
+        case 7: return launch_block<7>(a, grid, st, merge_blocks);
+        default: return launch_block<8>(a, grid, st, merge_blocks);
+    }
 }
 
 int duo_get_device_status(void *stream) {

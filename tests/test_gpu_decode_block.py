@@ -1,0 +1,97 @@
+"""duo_attn_decode_block (verify-block decode) on the GPU against the float64
+oracle's block decode, which is pinned to the prefill oracle over the full
+token history.
+
+Every q_len from 1 to 8 (three operand widths: 16, 32 and 48 query rows),
+sequences that are empty, below the sink, filling the ring and past it, a
+sliding layer with sink logits, an output gate, and a 32768-token context.
+The cache must be left untouched.  Tolerances as the one-token decode.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import kv_cache_reduction_b200 as duo
+from kv_cache_reduction_b200 import inputs
+
+from gpu_helpers import assert_close, host_cache, layers, random_cache
+
+pytestmark = pytest.mark.gpu
+
+
+def block_case(p, o, cache, q_len, seed, max_seq_len, gate=None, gate_mode=0):
+    B = p.batch
+    q = inputs.randn_bf16((B, q_len, 48, 128), seed, "cuda")
+    kn = inputs.randn_bf16((B, q_len, 8, 128), seed + 1, "cuda")
+    vn = inputs.randn_bf16((B, q_len, 8, 128), seed + 2, "cuda")
+    out = torch.full((B, q_len, 48, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, q_len, 48), float("nan"), dtype=torch.float32, device="cuda")
+    n = max(duo.duo_decode_block_workspace_bytes(p, q_len, max_seq_len), 256)
+    ws = torch.full(((n + 255) // 256 * 256,), 0x7f, dtype=torch.uint8, device="cuda")
+    before = [t.clone() for t in (cache.seq_len, cache.ring_head)]
+    snap = host_cache(o, cache)
+    duo.duo_attn_decode_block(p, cache, q, kn, vn, max_seq_len, out, lse, ws, gate=gate)
+    torch.cuda.synchronize()
+    assert duo.duo_get_device_status() == duo.DUO_OK
+    assert torch.equal(before[0], cache.seq_len) and torch.equal(before[1], cache.ring_head)
+    after = host_cache(o, cache)
+    for name in ("full_k", "full_v", "strm_k", "strm_v"):
+        assert np.array_equal(getattr(after, name), getattr(snap, name)), name
+    ref_o, ref_l = oracle.attn_decode_block(o, snap, inputs.bits(q), inputs.bits(kn), inputs.bits(vn))
+    if gate is not None:
+        ref_o = oracle.gate_decode(ref_o, inputs.bits(gate).reshape(B * q_len, 48, -1).squeeze(-1)
+                                   if gate_mode == oracle.GATE_PER_HEAD else
+                                   inputs.bits(gate).reshape(B * q_len, 48, 128), gate_mode, 48)
+    return assert_close(out, ref_o.reshape(B, q_len, 48, 128), lse, ref_l.reshape(B, q_len, 48),
+                        f"q_len={q_len}")
+
+
+@pytest.mark.parametrize("q_len", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_block_decode_duo_layer(cuda_device, q_len):
+    p, o = layers(6, full_mask=(1, 0, 0, 1, 0, 1, 1, 0))
+    seq = [0, 5, 64, 200, 320, 3000]
+    rh = [0, 0, 0, 136, 0, 77]
+    cache = random_cache(p, 3000, seq, rh, seed=80 + q_len)
+    block_case(p, o, cache, q_len, seed=90 + q_len, max_seq_len=3000)
+
+
+@pytest.mark.parametrize("q_len", [4, 8])
+def test_block_decode_sliding_layer_with_sink(cuda_device, q_len):
+    sig = inputs.randn_f32((48,), 100)
+    p, o = layers(3, window=512, sink_logit=sig)
+    seq = [3, 511, 9000]
+    cache = random_cache(p, 64, seq, [0, 0, 300], seed=101)
+    block_case(p, o, cache, q_len, seed=102, max_seq_len=9000)
+
+
+@pytest.mark.parametrize("mode", ["per_element", "per_head"])
+def test_block_decode_output_gate(cuda_device, mode):
+    p, o = layers(2, full_mask=(0, 1, 0, 0, 0, 0, 1, 0))
+    cache = random_cache(p, 700, [700, 33], [10, 0], seed=103)
+    shape = (2, 3, 48, 128) if mode == "per_element" else (2, 3, 48)
+    g = (inputs.randn_f32(shape, 104) * 2.0).to("cuda", torch.bfloat16)
+    gm = oracle.GATE_PER_ELEMENT if mode == "per_element" else oracle.GATE_PER_HEAD
+    block_case(p, o, cache, 3, seed=105, max_seq_len=700, gate=g, gate_mode=gm)
+
+
+@pytest.mark.slow
+def test_block_decode_long_context(cuda_device):
+    """B=8, context 32768, a block of 8: the verify shape at the decode_b32 context."""
+    p, o = layers(8, full_mask=inputs.seeded_full_mask(2002, 2))
+    rng = np.random.default_rng(106)
+    cache = random_cache(p, 32768, [32768] * 8, rng.integers(0, 256, size=8).tolist(), seed=107)
+    block_case(p, o, cache, 8, seed=108, max_seq_len=32768)
+
+
+def test_block_decode_rejects_long_blocks(cuda_device):
+    p, o = layers(1, full_mask=(1,) * 8)
+    cache = random_cache(p, 64, [10], [0], seed=109)
+    q = torch.zeros((1, 9, 48, 128), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((1, 9, 8, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros_like(q)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(duo.DuoError) as e:
+        duo.duo_attn_decode_block(p, cache, q, kv, kv, 64, out, None, ws)
+    assert e.value.code == duo.DUO_ERR_UNSUPPORTED
+    assert duo.duo_decode_block_workspace_bytes(p, 9, 64) == 0
