@@ -55,8 +55,13 @@ struct BlockCfg {
     static constexpr int NP = (NR + 15) / 16 * 16;               // MMA N
     static constexpr uint32_t OpBytes = NP * kD * 2;             // Q or P^T operand
     static constexpr uint32_t OpHalf = NP * 128;                 // one 64-column half of it
-    static constexpr int Stages = NP <= 16 ? 3 : 2;
-    static constexpr size_t Smem = 1024 + Stages * kDecStageBytes + 4 * OpBytes;   // Q x2, P^T x2
+    // three K/V stages keep two tiles in flight behind the one being scored;
+    // the operand buffers give way when the query rows grow
+    static constexpr int Stages = 3;
+    static constexpr int QB = NP <= 32 ? 2 : 1;                  // Q buffers (next item's Q staged early)
+    static constexpr int PB = NP <= 16 ? 2 : 1;                  // P^T buffers
+    static constexpr size_t Smem = 1024 + Stages * kDecStageBytes + (QB + PB) * OpBytes;
+    static_assert(Smem + 4096 <= 232448, "shared memory");
     static constexpr int PartFloats = NR * (kD + 2);             // m[NR], l[NR], acc[NR][D]
     static constexpr uint32_t TmemCols = 3 * NP <= 64 ? 64 : 3 * NP <= 128 ? 128 : 256;
     static constexpr int NH = NP / 2;                            // query rows per softmax warp
@@ -94,6 +99,20 @@ __device__ __forceinline__ float lane_row_reduce(float (&v)[RP], int lane) {
         }
     }
     return v[0];
+}
+
+// OR of a predicate over the 256 softmax threads (named barrier 1).
+__device__ __forceinline__ bool softmax_vote_any(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, 1, 256, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
 }
 
 template <int RP>
@@ -193,7 +212,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
     char *smem = bsmem_base + ((1024u - (smem_u32(bsmem_base) & 1023u)) & 1023u);
     char *sKV = smem;                                         // [stages][K 32 KB | V 32 KB]
     char *sQ = smem + ST * kDecStageBytes;                    // [2 items][OpBytes]
-    char *sP = sQ + 2 * C::OpBytes;                           // [2 tiles][OpBytes]
+    char *sP = sQ + C::QB * C::OpBytes;                       // [PB tiles][OpBytes]
     __shared__ uint64_t kv_full[ST], kv_empty[ST];
     // P^T is double-buffered: PV of tile j commits o_done[j & 1]
     __shared__ uint64_t s_full[2], p_full, o_done[2], q_ready[2];
@@ -219,7 +238,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
     }
     if (warp < 8) {
         // operand rows NR..NP-1 stay zero for the whole kernel
-        for (int i = threadIdx.x; i < 4 * (int)C::OpBytes / 16; i += 256)
+        for (int i = threadIdx.x; i < (C::QB + C::PB) * (int)C::OpBytes / 16; i += 256)
             reinterpret_cast<uint4 *>(sQ)[i] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
     }
@@ -288,8 +307,9 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
                 for (int k = 0; k < 8; ++k)
                     mma_ss(o_tmem, smem_desc_sw128(kv_addr + st * kDecStageBytes + kDecTileBytes + k * 2048,
                                                    kDecHalfBytes, 1024),
-                           smem_desc_sw128(p_addr + pbuf * C::OpBytes + (k >> 2) * C::OpHalf + (k & 3) * 32, 16,
-                                           1024),
+                           smem_desc_sw128(p_addr + (C::PB == 2 ? pbuf : 0) * C::OpBytes + (k >> 2) * C::OpHalf +
+                                               (k & 3) * 32,
+                                           16, 1024),
                            id_pv, (first && k == 0) ? 0u : 1u);
             };
             int jg = 0, ic = 0;
@@ -307,7 +327,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const uint32_t off = (k >> 2) * kDecHalfBytes + (k & 3) * 32;
-                        const uint32_t qoff = (ic & 1) * C::OpBytes + (k >> 2) * C::OpHalf + (k & 3) * 32;
+                        const uint32_t qoff = (C::QB == 2 ? (ic & 1) : 0) * C::OpBytes + (k >> 2) * C::OpHalf + (k & 3) * 32;
                         mma_ss(tmem + (jg & 1) * NP, smem_desc_sw128(kv_addr + st * kDecStageBytes + off, 16, 1024),
                                smem_desc_sw128(q_addr + qoff, 16, 1024), id_qk, k > 0);
                     }
@@ -354,7 +374,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
                     const int t = row / kGroup, h = row % kGroup;
                     const uint4 v = reinterpret_cast<const uint4 *>(
                         a.q + (((size_t)nx.it.b * kQ + t) * d.hkv * kGroup + nx.it.g * kGroup + h) * kD)[ch];
-                    *reinterpret_cast<uint4 *>(sQ + buf * C::OpBytes + blk_op_offset<NP>(row, ch * 8)) = v;
+                    *reinterpret_cast<uint4 *>(sQ + (C::QB == 2 ? buf : 0) * C::OpBytes + blk_op_offset<NP>(row, ch * 8)) = v;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -389,75 +409,86 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
                 const int32_t e = it.e_begin + t * kTok + r;
                 int t_lo, t_hi;
                 key_query_range(a, bi, e, &t_lo, &t_hi);
-                float s[NH], mx[RP];
+                // a full head's tile inside the cached length: every key for every query
+                const bool dense = !bi.block && !it.ring && it.e_begin + (t + 1) * kTok <= it.e_end;
+                float s[NH];
+                bool exceed = false;
 #pragma unroll
                 for (int q = 0; q < NH; ++q) {
                     const int tq = (q0 + q) / kGroup;
-                    s[q] = (q0 + q < NR && tq >= t_lo && tq <= t_hi) ? __uint_as_float(sr[q]) : -INFINITY;
-                    mx[q] = s[q];
+                    const bool keep = q0 + q < NR && (dense || (tq >= t_lo && tq <= t_hi));
+                    s[q] = keep ? __uint_as_float(sr[q]) : -INFINITY;
+                    exceed |= s[q] * c > m_run[q] + 8.f;
                 }
+                // The running max of a row moves only when some score exceeds it by
+                // more than 2^8.  One vote over the eight warps settles whether any
+                // row of this tile does; if none does, the tile's max is not needed
+                // and every row keeps its max (the same result as computing it).
+                if (softmax_vote_any(exceed)) {
+                    float mx[RP];
 #pragma unroll
-                for (int q = NH; q < RP; ++q) mx[q] = -INFINITY;
-                const float mrow = lane_row_reduce<RP, 0>(mx, lane);
-                if (lane == (lane_row<RP>(lane) << (5 - (RP == 8 ? 3 : RP == 16 ? 4 : 5))) && lane_row<RP>(lane) < NH)
-                    red_max[jg & 1][quarter][q0 + lane_row<RP>(lane)] = mrow;
-                sm_sync();
-                float alpha[NH], m_sub[NH];
-                bool rescale = false;
-                float m_join[NH];
+                    for (int q = 0; q < RP; ++q) mx[q] = q < NH ? s[q] : -INFINITY;
+                    const float mrow = lane_row_reduce<RP, 0>(mx, lane);
+                    if (lane == (lane_row<RP>(lane) << (5 - (RP == 8 ? 3 : RP == 16 ? 4 : 5))) &&
+                        lane_row<RP>(lane) < NH)
+                        red_max[jg & 1][quarter][q0 + lane_row<RP>(lane)] = mrow;
+                    sm_sync();
+                    float alpha[NH];
+                    bool rescale = false;
 #pragma unroll
-                for (int q = 0; q < NH; q += 4) {
-                    float4 v4[4];
+                    for (int q = 0; q < NH; q += 4) {
+                        float4 v4[4];
 #pragma unroll
-                    for (int w4 = 0; w4 < 4; ++w4)
-                        v4[w4] = *reinterpret_cast<const float4 *>(&red_max[jg & 1][w4][q0 + q]);
-                    m_join[q] = fmaxf(fmaxf(v4[0].x, v4[1].x), fmaxf(v4[2].x, v4[3].x));
-                    m_join[q + 1] = fmaxf(fmaxf(v4[0].y, v4[1].y), fmaxf(v4[2].y, v4[3].y));
-                    m_join[q + 2] = fmaxf(fmaxf(v4[0].z, v4[1].z), fmaxf(v4[2].z, v4[3].z));
-                    m_join[q + 3] = fmaxf(fmaxf(v4[0].w, v4[1].w), fmaxf(v4[2].w, v4[3].w));
-                }
+                        for (int w4 = 0; w4 < 4; ++w4)
+                            v4[w4] = *reinterpret_cast<const float4 *>(&red_max[jg & 1][w4][q0 + q]);
+                        const float mj[4] = {fmaxf(fmaxf(v4[0].x, v4[1].x), fmaxf(v4[2].x, v4[3].x)),
+                                             fmaxf(fmaxf(v4[0].y, v4[1].y), fmaxf(v4[2].y, v4[3].y)),
+                                             fmaxf(fmaxf(v4[0].z, v4[1].z), fmaxf(v4[2].z, v4[3].z)),
+                                             fmaxf(fmaxf(v4[0].w, v4[1].w), fmaxf(v4[2].w, v4[3].w))};
 #pragma unroll
-                for (int q = 0; q < NH; ++q) {
-                    const float m_tile = m_join[q] * c;
-                    alpha[q] = 1.f;
-                    if (m_tile > m_run[q] + 8.f) {
-                        alpha[q] = (m_run[q] == -INFINITY) ? 0.f : ex2_approx(m_run[q] - m_tile);
-                        m_run[q] = m_tile;
-                        rescale = true;
+                        for (int u = 0; u < 4; ++u) {
+                            const float m_tile = mj[u] * c;
+                            alpha[q + u] = 1.f;
+                            if (m_tile > m_run[q + u] + 8.f) {
+                                alpha[q + u] = (m_run[q + u] == -INFINITY) ? 0.f : ex2_approx(m_run[q + u] - m_tile);
+                                m_run[q + u] = m_tile;
+                                l_part[q + u] *= alpha[q + u];
+                                rescale = true;
+                            }
+                        }
                     }
-                    m_sub[q] = (m_run[q] == -INFINITY) ? 0.f : m_run[q];
+                    if (t > 0 && __any_sync(0xffffffffu, rescale)) {
+                        // O^T must hold every earlier tile's product before it is scaled
+                        const bool prev = mbar_wait(&o_done[(jg - 1) & 1], ((jg - 1) >> 1) & 1);
+                        __syncwarp();
+                        if (!__all_sync(0xffffffffu, prev)) { ok = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int cb = 0; cb < NH; cb += 8) {
+                            uint32_t orr[8];
+                            tmem_ld8(o_tmem + cb, orr);
+                            tmem_ld_wait();
+                            reg_fence8(orr);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * alpha[cb + q]);
+                            tmem_st8(o_tmem + cb, orr);
+                        }
+                        tmem_st_wait();
+                    }
                 }
                 float p[NH];
 #pragma unroll
                 for (int q = 0; q < NH; ++q) {
-                    p[q] = ex2_approx(fmaf(s[q], c, -m_sub[q]));
-                    l_part[q] = fmaf(l_part[q], alpha[q], p[q]);
+                    p[q] = ex2_approx(fmaf(s[q], c, m_run[q] == -INFINITY ? 0.f : -m_run[q]));
+                    l_part[q] += p[q];
                 }
-                // P^T buffer jg & 1 was last read by the PV of tile jg - 2
-                if (jg >= 2) {
-                    const bool prev = mbar_wait(&o_done[jg & 1], ((jg - 2) >> 1) & 1);
+                // the P^T buffer was last read by the PV of tile jg - PB
+                if (jg >= C::PB) {
+                    const int pj = jg - C::PB;
+                    const bool prev = mbar_wait(&o_done[pj & 1], (pj >> 1) & 1);
                     __syncwarp();
                     if (!__all_sync(0xffffffffu, prev)) { ok = false; break; }
                     tc_fence_after();
-                }
-                const bool do_rescale = t > 0 && __any_sync(0xffffffffu, rescale);
-                if (do_rescale) {
-                    // O^T must hold every earlier tile's product before it is scaled
-                    const bool prev = mbar_wait(&o_done[(jg - 1) & 1], ((jg - 1) >> 1) & 1);
-                    __syncwarp();
-                    if (!__all_sync(0xffffffffu, prev)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int cb = 0; cb < NH; cb += 8) {
-                        uint32_t orr[8];
-                        tmem_ld8(o_tmem + cb, orr);
-                        tmem_ld_wait();
-                        reg_fence8(orr);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * alpha[cb + q]);
-                        tmem_st8(o_tmem + cb, orr);
-                    }
-                    tmem_st_wait();
                 }
                 if (t_lo > t_hi && half == 0) {
                     // a key no query keeps: its V row must not reach the PV product
@@ -471,7 +502,8 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
 #pragma unroll
                 for (int q = 0; q < NH; ++q)
                     if (q0 + q < NR)
-                        *reinterpret_cast<__nv_bfloat16 *>(sP + (jg & 1) * C::OpBytes + blk_op_offset<NP>(q0 + q, r)) =
+                        *reinterpret_cast<__nv_bfloat16 *>(sP + (C::PB == 2 ? (jg & 1) : 0) * C::OpBytes +
+                                                           blk_op_offset<NP>(q0 + q, r)) =
                             __float2bfloat16_rn(p[q]);
                 fence_proxy_async_smem();
                 tc_fence_before();
