@@ -106,3 +106,44 @@ def test_prep_rejects_bad_parameters(cuda_device):
             duo.duo_kv_append_prep(p, cache, duo.DuoQKPrep(**bad), q, k, k)
         assert e.value.code == duo.DUO_ERR_INVALID_ARG, bad
     assert int(cache.seq_len[0]) == 0
+
+
+@pytest.mark.slow
+def test_prep_bench_shape_sampled(cuda_device):
+    """The bench's prep_16k call: a 16384-token prompt on the prefill_16k layer
+    (positions 0..16383), every prepared q/k row checked; the cache's full
+    heads checked in a seeded sample of rows, its ring heads completely."""
+    w = inputs.workload("prefill_16k")
+    p, o = layers(w.batch, full_mask=w.full_mask)
+    L = w.seq_len
+    cache = duo.DuoCache.allocate(p, L)
+    q = inputs.randn_bf16((1, L, 48, 128), 110, "cuda")
+    k = inputs.randn_bf16((1, L, 8, 128), 111, "cuda")
+    v = inputs.randn_bf16((1, L, 8, 128), 112, "cuda")
+    pr = duo.DuoQKPrep(q_norm_weight=(1 + 0.1 * inputs.randn_f32((128,), 113)).to("cuda", torch.bfloat16),
+                       k_norm_weight=(1 + 0.1 * inputs.randn_f32((128,), 114)).to("cuda", torch.bfloat16))
+    q0, k0 = f64(q), f64(k)
+    duo.duo_kv_append_prep(p, cache, pr, q, k, v)
+    torch.cuda.synchronize()
+    assert duo.duo_get_device_status() == duo.DUO_OK
+    inv = oprep.yarn_inv_freq(pr.rope_theta, pr.rope_factor, pr.original_max_position, pr.beta_fast,
+                              pr.beta_slow)
+    pos = np.arange(L, dtype=np.float64)[None, :]
+    q_ref = oprep.prep_rows(q0, f64(pr.q_norm_weight), pos, inv, 1.0, pr.rms_eps)
+    k_ref = oprep.prep_rows(k0, f64(pr.k_norm_weight), pos, inv, 1.0, pr.rms_eps)
+    within_half_ulp(f64(q), q_ref, "q")
+    within_half_ulp(f64(k), k_ref, "k")
+    # the cache holds the prepared keys: full heads at their positions, ring heads the kept tokens
+    kb = oprep.f64_to_bf16_bits(k_ref)
+    ref = oracle.Cache(o, L)
+    oracle.kv_append(o, ref, kb, inputs.bits(v))
+    got = host_cache(o, cache)
+    rows = np.random.default_rng(115).integers(0, L, size=512)
+    to_f = lambda b: (np.asarray(b, np.uint32) << 16).view(np.float32).astype(np.float64)
+    g, r = to_f(got.full_k[:, :, rows]), to_f(ref.full_k[:, :, rows])
+    assert np.all(np.abs(g - r) <= np.ldexp(1.0, np.frexp(r)[1] - 8) + 1e-6)
+    assert np.array_equal(got.full_v[:, :, rows], ref.full_v[:, :, rows])
+    g, r = to_f(got.strm_k), to_f(ref.strm_k)
+    assert np.all(np.abs(g - r) <= np.ldexp(1.0, np.frexp(r)[1] - 8) + 1e-6)
+    assert np.array_equal(got.strm_v, ref.strm_v)
+    assert np.array_equal(got.seq_len, ref.seq_len) and np.array_equal(got.ring_head, ref.ring_head)
