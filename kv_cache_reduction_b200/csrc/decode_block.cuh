@@ -64,13 +64,31 @@ struct BlockCfg {
     static_assert(Smem + 4096 <= 232448, "shared memory");
     static constexpr int PartFloats = NR * (kD + 2);             // m[NR], l[NR], acc[NR][D]
     static constexpr uint32_t TmemCols = 3 * NP <= 64 ? 64 : 3 * NP <= 128 ? 128 : 256;
-    static constexpr int NH = NP / 2;                            // query rows per softmax warp
-    static constexpr int RP = NH <= 8 ? 8 : NH <= 16 ? 16 : 32;  // NH padded to a power of two
+    // softmax warps per TMEM lane quarter, each with NH of the query rows: more
+    // of them for wide blocks, so that no thread holds more than 16 rows
+    static constexpr int NPART = NP == 48 ? 3 : 2;
+    static constexpr int NH = NP / NPART;                        // 8 or 16 rows
+    static constexpr int RP = NH <= 4 ? 4 : NH <= 8 ? 8 : NH <= 16 ? 16 : 32;   // NH padded to 2^k
+    static constexpr int SoftmaxThreads = 128 * NPART;
+    // softmax warps 0 .. 4*NPART-1, then the producer warp and the MMA warp
+    static constexpr int Threads = SoftmaxThreads + 64;
 };
 
-// Softmax warps 0-7 (two per TMEM lane quarter, each with half of the query
-// rows), producer warp 8, MMA warp 9.
-constexpr int kBlkThreads = 320;
+__device__ __forceinline__ void blk_tmem_ld4(uint32_t taddr, uint32_t *r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void blk_tmem_st4(uint32_t taddr, const uint32_t *r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+
+__device__ __forceinline__ void blk_reg_fence4(uint32_t *r) {
+    asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]));
+}
 
 // Per-row reduction of v[RP] over the 32 lanes of a warp that leaves row
 // (lane >> (5 - log2 RP)) with each lane: at every step a lane keeps half of
@@ -101,25 +119,25 @@ __device__ __forceinline__ float lane_row_reduce(float (&v)[RP], int lane) {
     return v[0];
 }
 
-// OR of a predicate over the 256 softmax threads (named barrier 1).
-__device__ __forceinline__ bool softmax_vote_any(bool v) {
+// OR of a predicate over the `nthreads` softmax threads (named barrier 1).
+__device__ __forceinline__ bool softmax_vote_any(bool v, int nthreads) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, 1, 256, q;\n\t"
+        "bar.red.or.pred p, 1, %2, q;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)v)
+        : "r"((uint32_t)v), "r"(nthreads)
         : "memory");
     return r != 0;
 }
 
 template <int RP>
-__device__ __forceinline__ int lane_row(int lane) {
-    constexpr int bits = RP == 8 ? 3 : RP == 16 ? 4 : 5;
-    return lane >> (5 - bits);
-}
+__host__ __device__ constexpr int rp_bits() { return RP == 4 ? 2 : RP == 8 ? 3 : RP == 16 ? 4 : 5; }
+
+template <int RP>
+__device__ __forceinline__ int lane_row(int lane) { return lane >> (5 - rp_bits<RP>()); }
 
 struct BlockArgs {
     DecodeArgs d;                   // cache maps, geometry, splits (d.q, d.out, d.lse unused)
@@ -204,9 +222,11 @@ __device__ __forceinline__ void key_query_range(const BlockArgs &a, const BlockI
 }
 
 template <int kQ>
-__global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __grid_constant__ BlockArgs a) {
+__global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(const __grid_constant__ BlockArgs a) {
     using C = BlockCfg<kQ>;
     constexpr int NR = C::NR, NP = C::NP, ST = C::Stages, NH = C::NH, RP = C::RP;
+    constexpr int NSM = C::SoftmaxThreads, NSW = NSM / 32;    // softmax threads / warps
+    constexpr int kProducer = NSW, kMma = NSW + 1;
     const DecodeArgs &d = a.d;
     extern __shared__ __align__(16) char bsmem_base[];
     char *smem = bsmem_base + ((1024u - (smem_u32(bsmem_base) & 1023u)) & 1023u);
@@ -229,20 +249,20 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&q_ready[i], 8);
+            mbar_init(&q_ready[i], NSW);
         }
-        mbar_init(&p_full, 8);
+        mbar_init(&p_full, NSW);
         mbar_init(&o_done[0], 1);
         mbar_init(&o_done[1], 1);
         fence_mbar_init();
     }
-    if (warp < 8) {
+    if (warp < NSW) {
         // operand rows NR..NP-1 stay zero for the whole kernel
-        for (int i = threadIdx.x; i < (C::QB + C::PB) * (int)C::OpBytes / 16; i += 256)
+        for (int i = threadIdx.x; i < (C::QB + C::PB) * (int)C::OpBytes / 16; i += NSM)
             reinterpret_cast<uint4 *>(sQ)[i] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
     }
-    if (warp == 9) {
+    if (warp == kMma) {
         tmem_alloc(&tmem_base, C::TmemCols);
         tmem_relinquish();
     }
@@ -252,7 +272,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
     tc_fence_after();
     const uint32_t tmem = tmem_base;
 
-    if (warp == 8) {
+    if (warp == kProducer) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             if (d.n_full > 0) {
@@ -295,7 +315,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
             }
         }
         __syncwarp();
-    } else if (warp == 9) {
+    } else if (warp == kMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(kTok, NP, 0, 0);
@@ -356,20 +376,20 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
     } else {
         // ------------------------------------------------------------ softmax + epilogue
         const int quarter = warp & 3;                        // TMEM lane quarter: tokens / dims
-        const int half = warp >> 2;                          // query rows [half * NH, half * NH + NH)
+        const int part = warp >> 2;                          // query rows [part * NH, part * NH + NH)
         const int r = quarter * 32 + lane;                   // token row / output dimension
-        const int q0 = half * NH;
+        const int q0 = part * NH;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t o_tmem = tmem + 2 * NP + q0 + lane_base;
         const float c = d.scale_log2;
-        const int tid = threadIdx.x;                         // 0..255
-        auto sm_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+        const int tid = threadIdx.x;                         // 0 .. NSM - 1
+        auto sm_sync = [] { asm volatile("bar.sync 1, %0;" ::"r"(NSM) : "memory"); };
         // Stages the NR query rows of the first non-empty item at or after w.
         auto stage_q = [&](int w, int buf) {
             for (; w < n_items; w += gridDim.x) {
                 const BlockItem nx = block_item_of(a, w);
                 if (nx.it.n_tiles == 0) continue;
-                for (int i = tid; i < NR * 16; i += 256) {
+                for (int i = tid; i < NR * 16; i += NSM) {
                     const int row = i >> 4, ch = i & 15;
                     const int t = row / kGroup, h = row % kGroup;
                     const uint4 v = reinterpret_cast<const uint4 *>(
@@ -401,11 +421,10 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
                 tc_fence_after();
                 uint32_t sr[NH];
 #pragma unroll
-                for (int cb = 0; cb < NH; cb += 8)
-                    tmem_ld8(tmem + (jg & 1) * NP + q0 + cb + lane_base, *reinterpret_cast<uint32_t(*)[8]>(&sr[cb]));
+                for (int cb = 0; cb < NH; cb += 4) blk_tmem_ld4(tmem + (jg & 1) * NP + q0 + cb + lane_base, &sr[cb]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int cb = 0; cb < NH; cb += 8) reg_fence8(*reinterpret_cast<uint32_t(*)[8]>(&sr[cb]));
+                for (int cb = 0; cb < NH; cb += 4) blk_reg_fence4(&sr[cb]);
                 const int32_t e = it.e_begin + t * kTok + r;
                 int t_lo, t_hi;
                 key_query_range(a, bi, e, &t_lo, &t_hi);
@@ -424,13 +443,12 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
                 // more than 2^8.  One vote over the eight warps settles whether any
                 // row of this tile does; if none does, the tile's max is not needed
                 // and every row keeps its max (the same result as computing it).
-                if (softmax_vote_any(exceed)) {
+                if (softmax_vote_any(exceed, NSM)) {
                     float mx[RP];
 #pragma unroll
                     for (int q = 0; q < RP; ++q) mx[q] = q < NH ? s[q] : -INFINITY;
                     const float mrow = lane_row_reduce<RP, 0>(mx, lane);
-                    if (lane == (lane_row<RP>(lane) << (5 - (RP == 8 ? 3 : RP == 16 ? 4 : 5))) &&
-                        lane_row<RP>(lane) < NH)
+                    if (lane == (lane_row<RP>(lane) << (5 - rp_bits<RP>())) && lane_row<RP>(lane) < NH)
                         red_max[jg & 1][quarter][q0 + lane_row<RP>(lane)] = mrow;
                     sm_sync();
                     float alpha[NH];
@@ -464,14 +482,14 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
                         if (!__all_sync(0xffffffffu, prev)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
-                        for (int cb = 0; cb < NH; cb += 8) {
-                            uint32_t orr[8];
-                            tmem_ld8(o_tmem + cb, orr);
+                        for (int cb = 0; cb < NH; cb += 4) {
+                            uint32_t orr[4];
+                            blk_tmem_ld4(o_tmem + cb, orr);
                             tmem_ld_wait();
-                            reg_fence8(orr);
+                            blk_reg_fence4(orr);
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * alpha[cb + q]);
-                            tmem_st8(o_tmem + cb, orr);
+                            for (int q = 0; q < 4; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * alpha[cb + q]);
+                            blk_tmem_st4(o_tmem + cb, orr);
                         }
                         tmem_st_wait();
                     }
@@ -490,7 +508,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
                     if (!__all_sync(0xffffffffu, prev)) { ok = false; break; }
                     tc_fence_after();
                 }
-                if (t_lo > t_hi && half == 0) {
+                if (t_lo > t_hi && part == 0) {
                     // a key no query keeps: its V row must not reach the PV product
                     char *vrow = sKV + (jg % ST) * kDecStageBytes + kDecTileBytes + r * 128;
 #pragma unroll
@@ -525,13 +543,13 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
                 if (!__all_sync(0xffffffffu, done)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
-                for (int cb = 0; cb < NH; cb += 8) {
-                    uint32_t orr[8];
-                    tmem_ld8(o_tmem + cb, orr);
+                for (int cb = 0; cb < NH; cb += 4) {
+                    uint32_t orr[4];
+                    blk_tmem_ld4(o_tmem + cb, orr);
                     tmem_ld_wait();
-                    reg_fence8(orr);
+                    blk_reg_fence4(orr);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) acc[cb + q] = __uint_as_float(orr[q]);
+                    for (int q = 0; q < 4; ++q) acc[cb + q] = __uint_as_float(orr[q]);
                 }
             }
             // l: this warp's 32 tokens per row, then the four quarters in a fixed order
@@ -540,7 +558,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
             for (int q = 0; q < RP; ++q) lsum[q] = q < NH ? l_part[q] : 0.f;
             const float lrow = lane_row_reduce<RP, 1>(lsum, lane);
             const int my_row = lane_row<RP>(lane);
-            const bool row_writer = lane == (my_row << (5 - (RP == 8 ? 3 : RP == 16 ? 4 : 5)));
+            const bool row_writer = lane == (my_row << (5 - rp_bits<RP>()));
             if (row_writer && my_row < NH) red_sum[quarter][q0 + my_row] = lrow;
             sm_sync();
             float *part = d.part + (((size_t)it.b * d.hkv + it.g) * a.part_slots + it.split) * C::PartFloats;
@@ -563,7 +581,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1) decode_block_split(const __gri
     tc_fence_before();
     __syncthreads();
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (warp == 9) {
+    if (warp == kMma) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TmemCols);
     }

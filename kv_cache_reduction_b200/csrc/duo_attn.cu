@@ -271,7 +271,7 @@ int launch_block(duo::BlockArgs &a, int grid, cudaStream_t st, int64_t merge_blo
     if ((rc = set_smem_once(duo::decode_block_split<kQ>, duo::BlockCfg<kQ>::Smem, "decode_block_split",
                             smem_set)))
         return rc;
-    duo::decode_block_split<kQ><<<(unsigned)grid, duo::kBlkThreads, duo::BlockCfg<kQ>::Smem, st>>>(a);
+    duo::decode_block_split<kQ><<<(unsigned)grid, duo::BlockCfg<kQ>::Threads, duo::BlockCfg<kQ>::Smem, st>>>(a);
     if ((rc = launch_status("decode_block_split"))) return rc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)merge_blocks);
