@@ -30,6 +30,8 @@
 //              O_h += P_h V (P_h read from tensor memory).  S_h(j+1) overwrites
 //              the columns PV_h(j) reads; the tcgen05 MMAs of one thread execute
 //              in issue order, so it is issued right behind it without a wait.
+//              The same holds across work tiles: the next work tile's first
+//              S_h follows this one's last PV_h.
 // TMEM: S0 | S1 | O0 | O1, 128 fp32 columns each (512 in total).  Key tiles
 // that no row of a query tile attends to are never loaded.
 #pragma once
@@ -94,11 +96,13 @@ __device__ __forceinline__ TileList tile_list(int kind, int t, int L, int sink, 
     return tl;
 }
 
-__device__ __forceinline__ bool key_attended(int kind, int i, int j, int sink, int recent, int window) {
-    if (j > i) return false;
-    if (kind == kKindFull) return true;
-    if (kind == kKindStreaming) return j < sink || j > i - recent;
-    return j > i - window;
+// Bits lo..hi of a 64-bit column mask (clamped to 0..63; empty when lo > hi).
+__device__ __forceinline__ uint64_t col_range_bits(int lo, int hi) {
+    lo = max(lo, 0);
+    hi = min(hi, 63);
+    if (lo > hi) return 0ull;
+    const uint64_t upto = hi == 63 ? ~0ull : ((1ull << (hi + 1)) - 1ull);
+    return upto & (~0ull << lo);
 }
 
 // True when every (row, key) pair of the tile is attended.
@@ -254,41 +258,67 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                            id_pv, (first && k == 0) ? 0u : 1u);
                 mma_commit(&o_done[h]);
             };
-            int jg = 0;
-            bool ok = true;
-            for (int wc = 0; ok; ++wc) {
-                const int sl = wc % kPfSlots;
-                if (!(ok = mbar_wait(&work_full[sl], (wc / kPfSlots) & 1))) break;
-                const int w = work_slot[sl];
+            // the work tile index of slot wc (an index >= n_work ends the list)
+            auto fetch = [&](int wcx, int *wout) -> bool {
+                const int sl = wcx % kPfSlots;
+                if (!mbar_wait(&work_full[sl], (wcx / kPfSlots) & 1)) return false;
+                *wout = work_slot[sl];
                 mbar_arrive(&work_empty[sl]);
-                if (w >= a.n_work) break;
+                return true;
+            };
+            auto kv_count = [&](int w) {
                 const PfWork wk = work_of(a, w);
-                const TileList tl = tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window);
-                const int n_kv = tl.count();
-                if (!(ok = mbar_wait(&q_full, wc & 1))) break;
-                if (!(ok = mbar_wait(&kv_full[jg % kPfStages], (jg / kPfStages) & 1))) break;
-                tc_fence_after();
-                issue_qk(0, jg % kPfStages);
-                issue_qk(1, jg % kPfStages);
-                if (n_kv == 1) mma_commit(&q_empty);
+                return tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window).count();
+            };
+            int jg = 0, wc = 0, w = 0;
+            bool ok = fetch(0, &w);
+            int n_kv = 0;
+            if (ok && w < a.n_work) {
+                n_kv = kv_count(w);
+                ok = mbar_wait(&q_full, 0) && mbar_wait(&kv_full[0], 0);
+                if (ok) {
+                    tc_fence_after();
+                    issue_qk(0, 0);
+                    issue_qk(1, 0);
+                    if (n_kv == 1) mma_commit(&q_empty);
+                }
+            }
+            // Each work tile's first S products are issued right behind the previous
+            // work tile's last PV of the same head, so that the tensor core has them
+            // while the softmax warps run that work tile's epilogue.
+            while (ok && w < a.n_work) {
+                int w_next = a.n_work, n_kv_next = 0;
                 for (int j = 0; j < n_kv && ok; ++j, ++jg) {
                     const int st = jg % kPfStages;
-                    const bool more = j + 1 < n_kv;
                     const int st1 = (jg + 1) % kPfStages;
+                    const bool last = j + 1 == n_kv;
+                    if (last) {
+                        if (!(ok = fetch(wc + 1, &w_next))) break;
+                        if (w_next < a.n_work) n_kv_next = kv_count(w_next);
+                    }
+                    const bool more = !last || w_next < a.n_work;
                     for (int h = 0; h < 2 && ok; ++h) {
                         if (!(ok = mbar_wait(&p_full[h], jg & 1))) break;
                         tc_fence_after();
                         issue_pv(h, st, j == 0);
                         if (more) {
-                            if (h == 0 && !(ok = mbar_wait(&kv_full[st1], ((jg + 1) / kPfStages) & 1))) break;
+                            if (h == 0) {
+                                if (last && !(ok = mbar_wait(&q_full, (wc + 1) & 1))) break;   // next Q
+                                if (!(ok = mbar_wait(&kv_full[st1], ((jg + 1) / kPfStages) & 1))) break;
+                            }
                             tc_fence_after();
                             issue_qk(h, st1);
                         }
                     }
                     if (!ok) break;
                     mma_commit(&kv_empty[st]);
-                    if (j + 2 == n_kv) mma_commit(&q_empty);   // the work tile's last S products are issued
+                    // Q of a work tile is free once its last S products are issued
+                    if (!last && j + 2 == n_kv) mma_commit(&q_empty);
+                    if (last && more && n_kv_next == 1) mma_commit(&q_empty);
                 }
+                w = w_next;
+                n_kv = n_kv_next;
+                ++wc;
             }
         }
         __syncwarp();  // lanes 1..31 wait for the MMA lane before the CTA barrier
@@ -340,10 +370,21 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 const int c0 = tl.at(j) * kPfN;
                 const bool dense = tile_dense(kind, wk.t * kPfM, c0, a.sink, a.recent, a.window);
                 if (!dense) {
+                    // the row's attended keys among this half's 64 columns as a bit
+                    // mask built from their one or two ranges
+                    const int cb0 = c0 + half * 64;
+                    const int di = i - cb0;                    // the diagonal's column
+                    uint64_t m;
+                    if (kind == kKindFull)
+                        m = col_range_bits(0, di);
+                    else if (kind == kKindStreaming)
+                        m = col_range_bits(0, min(di, a.sink - 1 - cb0)) | col_range_bits(di - a.recent + 1, di);
+                    else
+                        m = col_range_bits(di - a.window + 1, di);
+                    const uint32_t mlo = (uint32_t)m, mhi = (uint32_t)(m >> 32);
 #pragma unroll
                     for (int cc = 0; cc < 64; ++cc)
-                        if (!key_attended(kind, i, c0 + half * 64 + cc, a.sink, a.recent, a.window))
-                            sr[cc] = __float_as_uint(-INFINITY);
+                        if (!((((cc < 32) ? mlo : mhi) >> (cc & 31)) & 1u)) sr[cc] = __float_as_uint(-INFINITY);
                 }
                 float mx8[8];
 #pragma unroll
