@@ -25,6 +25,10 @@
 // extra item for the block's keys: one 128-row tile of the block's K/V (rows
 // past q_len are zero-filled by the tensor map and masked).  Every key token
 // carries the range [t_lo, t_hi] of block queries that may attend to it.
+// The softmax of a tile is split over two or three warps per TMEM lane
+// quarter (at most 16 query rows per thread), and one vote across them
+// (bar.red.or) skips the row-max reduction on tiles where no score exceeds its
+// row's running max by more than 2^8 -- the same result as reducing.
 #pragma once
 
 #include <cuda.h>
