@@ -211,6 +211,52 @@ DecodePlan plan_decode(const duo_params *p, const Layout &L, int64_t max_n, int 
     return d;
 }
 
+// The block decode's plan.  Each item (split of a full head, ring head, the
+// block's own keys) carries a fixed cost that grows with the query rows it
+// holds (staging their Q, filling the pipeline, writing their partials), so
+// the full heads' split count is chosen on the makespan of the persistent
+// CTAs' round-robin share of ALL the items, in tiles plus that cost.
+DecodePlan plan_block(const duo_params *p, const Layout &L, int64_t max_n, int sms, int rows) {
+    DecodePlan d = plan_decode(p, L, max_n, sms);
+    const double item = 1.0 + rows / 10.0;          // per-item cost in tiles (measured ~6 at 48 rows)
+    const int64_t full_units = (int64_t)p->batch * L.n_full;
+    const int64_t ring_items = (int64_t)p->batch * L.n_ring * d.splits_ring;
+    const int64_t block_items = (int64_t)p->batch * p->num_kv_heads;
+    if (full_units > 0) {
+        const int64_t tiles = cdiv(std::max<int64_t>(max_n, 1), duo::kTok);
+        const double c_ring = (double)cdiv(d.chunk_ring, duo::kTok) + item, c_block = 1.0 + item;
+        double best = 1e300;
+        for (int64_t s = 1; s <= std::min<int64_t>(tiles, 64); ++s) {
+            const int64_t chunk = cdiv(tiles, s), splits = cdiv(tiles, chunk);
+            const int64_t nf = full_units * splits, total = nf + ring_items + block_items;
+            const int64_t g = std::min<int64_t>(total, sms);
+            // items of [start, start + n) that CTA b takes: b, b + g, b + 2g, ...
+            auto count = [g](int64_t b, int64_t start, int64_t n) -> int64_t {
+                if (n <= 0) return 0;
+                const int64_t k0 = start > b ? cdiv(start - b, g) : 0;
+                const int64_t last = start + n - 1;
+                if (last < b) return 0;
+                const int64_t k1 = (last - b) / g;
+                return k1 >= k0 ? k1 - k0 + 1 : 0;
+            };
+            double span = 0.0;
+            for (int64_t b = 0; b < g; ++b)
+                span = std::max(span, count(b, 0, nf) * ((double)chunk + item) +
+                                          count(b, nf, ring_items) * c_ring +
+                                          count(b, nf + ring_items, block_items) * c_block);
+            if (span < best - 1e-9) {
+                best = span;
+                d.chunk_full = (int)(chunk * duo::kTok);
+                d.splits_full = (int)splits;
+            }
+        }
+        d.max_splits = std::max(1, std::max(d.splits_full, d.splits_ring));
+        d.items = full_units * d.splits_full + ring_items;
+        d.grid = (int)std::min<int64_t>(d.items, sms);
+    }
+    return d;
+}
+
 // A cache viewed as a 2-D tensor (128 columns, rows) loaded in 64-column x
 // 128-row boxes with the 128-byte swizzle.
 bool cache_tmap(CUtensorMap *m, void *base, int64_t rows) {
@@ -533,7 +579,7 @@ size_t duo_decode_block_workspace_bytes(const duo_params *params, int32_t q_len,
         return 0;
     int sms = 148;
     if (check_device(&sms)) sms = 148;
-    const DecodePlan d = plan_decode(params, L, max_seq_len, sms);
+    const DecodePlan d = plan_block(params, L, max_seq_len, sms, duo::kGroup * q_len);
     const size_t slots = (size_t)std::max(d.splits_full, d.splits_ring) + 1;
     return (size_t)params->batch * params->num_kv_heads * slots * (size_t)(duo::kGroup * q_len) *
            (duo::kD + 2) * sizeof(float);
@@ -565,7 +611,7 @@ int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, cons
         return fail(DUO_ERR_UNSUPPORTED, "cache rows exceed 2^31 (tensor-map coordinates are 32-bit)");
     int sms = 148;
     if ((rc = check_device(&sms))) return rc;
-    const DecodePlan d = plan_decode(params, L, max_seq_len, sms);
+    const DecodePlan d = plan_block(params, L, max_seq_len, sms, duo::kGroup * q_len);
     const size_t need = duo_decode_block_workspace_bytes(params, q_len, max_seq_len);
     if (!workspace || workspace_size < need || ((uintptr_t)workspace & 255u))
         return fail(DUO_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
