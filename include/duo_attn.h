@@ -254,7 +254,9 @@ DUO_API size_t duo_decode_block_workspace_bytes(const duo_params *params, int32_
  * out: [B][q_len][Hq][D]; lse: fp32 [B][q_len][Hq] or NULL.  max_seq_len
  * bounds every seq_len[b] (the cached length, without the block).
  * workspace: >= duo_decode_block_workspace_bytes(params, q_len, max_seq_len)
- * bytes, 256-byte aligned, contents need not be initialised.  gate: NULL or an
+ * bytes, 256-byte aligned, contents need not be initialised (it holds the
+ * split partials and a work-item counter that the call zeroes on the stream;
+ * calls that may run at the same time need separate workspaces).  gate: NULL or an
  * output gate (values [B][q_len][Hq][D] or [B][q_len][Hq]).  q_len outside
  * [1, 8] is DUO_ERR_UNSUPPORTED; other errors as duo_attn_decode. */
 DUO_API int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, const void *q,

@@ -150,6 +150,7 @@ struct BlockArgs {
     __nv_bfloat16 *out;             // [B][q_len][Hq][D]
     float *lse;                     // [B][q_len][Hq] or null
     int32_t q_len, n_cache_items, part_slots;   // part_slots = splits + 1 (the block item last)
+    int32_t *work_counter;          // zeroed before the launch: items claimed so far
 };
 
 // Byte offset of element (row, k) in an [NP rows][128] bf16 K-major operand
@@ -240,6 +241,10 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
     __shared__ uint64_t kv_full[ST], kv_empty[ST];
     // P^T is double-buffered: PV of tile j commits o_done[j & 1]
     __shared__ uint64_t s_full[2], p_full, o_done[2], q_ready[2];
+    // items claimed by the producer, read by the MMA issuer and the softmax warps
+    constexpr int kSlots = 4;
+    __shared__ uint64_t work_full[kSlots], work_empty[kSlots];
+    __shared__ int work_slot[kSlots];
     __shared__ uint32_t tmem_base;
     __shared__ __align__(16) float red_max[2][4][NP];
     __shared__ float red_sum[4][NP];
@@ -258,6 +263,10 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         mbar_init(&p_full, NSW);
         mbar_init(&o_done[0], 1);
         mbar_init(&o_done[1], 1);
+        for (int i = 0; i < kSlots; ++i) {
+            mbar_init(&work_full[i], 1);
+            mbar_init(&work_empty[i], 1 + NSW);        // the MMA issuer and every softmax warp
+        }
         fence_mbar_init();
     }
     if (warp < NSW) {
@@ -291,7 +300,17 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
             prefetch_tmap(&a.tm_bv);
             int jg = 0;
             bool ok = true;
-            for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+            int w = blockIdx.x;
+            for (int ic = 0; ok; ++ic) {
+                // publish the item (an index >= n_items tells the consumers to stop)
+                const int sl = ic % kSlots;
+                if (ic >= kSlots && !(ok = mbar_wait(&work_empty[sl], ((ic / kSlots) - 1) & 1))) break;
+                work_slot[sl] = w;
+                mbar_arrive(&work_full[sl]);
+                if (w >= n_items) break;
+                // the next claim, heaviest items first: a CTA takes the next one when it
+                // is ready for it, so unequal items do not pile up on a few CTAs
+                const int w_next = (int)gridDim.x + atomicAdd(a.work_counter, 1);
                 const BlockItem bi = block_item_of(a, w);
                 const Item &it = bi.it;
                 for (int t = 0; t < it.n_tiles; ++t, ++jg) {
@@ -316,6 +335,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                         tma_load_2d(ks + kDecTileBytes + kDecHalfBytes, tv, 64, row, &kv_full[st]);
                     }
                 }
+                w = w_next;
             }
         }
         __syncwarp();
@@ -339,11 +359,18 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
             int jg = 0, ic = 0;
             bool ok = true, pend = false, pend_first = false;
             int pend_st = 0;
-            for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+            for (; ok; ++ic) {
+                const int sl = ic % kSlots;
+                if (!(ok = mbar_wait(&work_full[sl], (ic / kSlots) & 1))) break;
+                const int w = work_slot[sl];
+                mbar_arrive(&work_empty[sl]);
+                if (w >= n_items) break;
                 const BlockItem bi = block_item_of(a, w);
                 const Item &it = bi.it;
-                if (it.n_tiles == 0) continue;
+                // every item's Q is staged (an empty item's only signals), so the
+                // staging and this wait pair up item by item
                 if (!(ok = mbar_wait(&q_ready[ic & 1], (ic >> 1) & 1))) break;
+                if (it.n_tiles == 0) continue;
                 for (int t = 0; t < it.n_tiles && ok; ++t, ++jg) {
                     const int st = jg % ST;
                     if (!(ok = mbar_wait(&kv_full[st], (jg / ST) & 1))) break;
@@ -367,7 +394,6 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                     pend_st = st;
                     pend_first = (t == 0);
                 }
-                ++ic;
             }
             if (ok && pend && mbar_wait(&p_full, (jg - 1) & 1)) {
                 tc_fence_after();
@@ -388,11 +414,24 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         const float c = d.scale_log2;
         const int tid = threadIdx.x;                         // 0 .. NSM - 1
         auto sm_sync = [] { asm volatile("bar.sync 1, %0;" ::"r"(NSM) : "memory"); };
-        // Stages the NR query rows of the first non-empty item at or after w.
+        // Reads item slot icx (each softmax warp once per slot).
+        auto read_slot = [&](int icx, int *wout) -> bool {
+            const int sl = icx % kSlots;
+            const bool got = mbar_wait(&work_full[sl], (icx / kSlots) & 1);
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, got)) return false;
+            *wout = work_slot[sl];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&work_empty[sl]);
+            return true;
+        };
+        // Stages the NR query rows of item w as the Q operand in buffer `buf`
+        // (nothing to copy for an empty item, but the MMA warp is still told).
         auto stage_q = [&](int w, int buf) {
-            for (; w < n_items; w += gridDim.x) {
+            if (w >= n_items) return;
+            {
                 const BlockItem nx = block_item_of(a, w);
-                if (nx.it.n_tiles == 0) continue;
+                if (nx.it.n_tiles > 0)
                 for (int i = tid; i < NR * 16; i += NSM) {
                     const int row = i >> 4, ch = i & 15;
                     const int t = row / kGroup, h = row % kGroup;
@@ -403,13 +442,12 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&q_ready[buf]);
-                return;
             }
         };
-        int jg = 0, ic = 0;
-        bool ok = true;
-        stage_q(blockIdx.x, 0);
-        for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        int jg = 0, ic = 0, w = 0;
+        bool ok = read_slot(0, &w);
+        if (ok) stage_q(w, 0);
+        for (; ok && w < n_items; ++ic) {
             const BlockItem bi = block_item_of(a, w);
             const Item &it = bi.it;
             float m_run[NH], l_part[NH];
@@ -533,10 +571,10 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 if (lane == 0) mbar_arrive(&p_full);
             }
             if (!ok) break;
-            if (it.n_tiles > 0) {
-                ++ic;
-                stage_q(w + gridDim.x, ic & 1);
-            }
+            // the next item: its Q may be staged now (this item's S products are all read)
+            int w_next = n_items;
+            if (!(ok = read_slot(ic + 1, &w_next))) break;
+            stage_q(w_next, (ic + 1) & 1);
             // ------------------------------------------------------------ item epilogue
             float acc[NH];
 #pragma unroll
@@ -579,6 +617,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 part[NR + q] = (red_sum[0][q] + red_sum[1][q]) + (red_sum[2][q] + red_sum[3][q]);
             }
             sm_sync();
+            w = w_next;
         }
         __syncwarp();
     }

@@ -581,8 +581,9 @@ size_t duo_decode_block_workspace_bytes(const duo_params *params, int32_t q_len,
     if (check_device(&sms)) sms = 148;
     const DecodePlan d = plan_block(params, L, max_seq_len, sms, duo::kGroup * q_len);
     const size_t slots = (size_t)std::max(d.splits_full, d.splits_ring) + 1;
-    return (size_t)params->batch * params->num_kv_heads * slots * (size_t)(duo::kGroup * q_len) *
-           (duo::kD + 2) * sizeof(float);
+    const size_t partials = (size_t)params->batch * params->num_kv_heads * slots *
+                            (size_t)(duo::kGroup * q_len) * (duo::kD + 2) * sizeof(float);
+    return (partials + 255) / 256 * 256 + 256;       // + the work-item counter
 }
 
 int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, const void *q,
@@ -661,6 +662,10 @@ int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, cons
     a.q_len = q_len;
     a.n_cache_items = (int32_t)d.items;
     a.part_slots = da.max_splits;
+    // the work-item counter sits behind the partials, zeroed on the stream
+    a.work_counter = (int32_t *)((char *)workspace + (need - 256));
+    if (cudaMemsetAsync(a.work_counter, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess)
+        return fail(DUO_ERR_CUDA, "zeroing the block decode's work counter failed");
     const int64_t items = d.items + (int64_t)params->batch * params->num_kv_heads;
     const int grid = (int)std::min<int64_t>(items, sms);
     const int64_t merge_blocks = (int64_t)params->batch * q_len * params->num_q_heads;
