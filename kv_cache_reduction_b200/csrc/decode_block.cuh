@@ -21,9 +21,10 @@
 // 128-token tile in M and the query rows in N:
 //   S^T[128 tok x NP] = K_tile . Q^T,   O^T[128 d x NP] += V_tile^T . P^T
 // with NR = 6 * q_len query rows (row t*6 + h: block token t, head h of the
-// group) padded to NP = 16, 32 or 48.  Each (sequence, KV head) gets one
-// extra item for the block's keys: one 128-row tile of the block's K/V (rows
-// past q_len are zero-filled by the tensor map and masked).  Every key token
+// group) padded to NP = 16, 32 or 48.  Each (sequence, KV head) has one
+// more tile for the block's keys: one 128-row tile of the block's K/V (rows
+// past q_len are zero-filled by the tensor map and masked), the last tile of
+// that head's last split item.  Every key token
 // carries the range [t_lo, t_hi] of block queries that may attend to it.
 // The softmax of a tile is split over two or three warps per TMEM lane
 // quarter (at most 16 query rows per thread), and one vote across them
@@ -149,7 +150,7 @@ struct BlockArgs {
     const __nv_bfloat16 *q;         // [B][q_len][Hq][D]
     __nv_bfloat16 *out;             // [B][q_len][Hq][D]
     float *lse;                     // [B][q_len][Hq] or null
-    int32_t q_len, n_cache_items, part_slots;   // part_slots = splits + 1 (the block item last)
+    int32_t q_len, n_cache_items, part_slots;   // part_slots = the most splits of a head
     int32_t *work_counter;          // zeroed before the launch: items claimed so far
 };
 
@@ -163,52 +164,39 @@ __device__ __forceinline__ uint32_t blk_op_offset(int row, int k) {
 }
 
 struct BlockItem {
-    Item it;                        // the cache item (it.n_tiles = 1 for the block item)
-    bool block;
+    Item it;                        // the cache item; n_tiles includes the block's tile
+    int cache_tiles;                // tiles of cached keys; the block's tile, if any, follows
+    bool has_block;                 // the last split of its (sequence, KV head): carries the block's keys
 };
 
 __device__ __forceinline__ BlockItem block_item_of(const BlockArgs &a, int w) {
     BlockItem bi;
-    if (w < a.n_cache_items) {
-        bi.it = item_of(a.d, w);
-        bi.block = false;
-        return bi;
-    }
-    w -= a.n_cache_items;                           // one per (sequence, KV head)
-    bi.block = true;
-    Item &it = bi.it;
-    it.b = w / a.d.hkv;
-    it.g = w % a.d.hkv;
-    it.split = a.part_slots - 1;
-    it.ring = !a.d.heads.is_full[it.g];
-    it.row0 = 0;
-    it.e_begin = 0;
-    it.e_end = a.q_len;
-    const int32_t n = a.d.seq_len[it.b];
-    it.n_sink = min(n, a.d.sink);
-    it.cnt = 0;
-    it.ring_base = 0;
-    it.n_tiles = 1;
+    bi.it = item_of(a.d, w);
+    bi.cache_tiles = bi.it.n_tiles;
+    const int splits = bi.it.ring ? a.d.splits_ring : a.d.splits_full;
+    bi.has_block = bi.it.split == splits - 1;
+    if (bi.has_block) bi.it.n_tiles += 1;
     return bi;
 }
 
 // The block queries [t_lo, t_hi] that may attend to key e of the item (empty
-// when t_lo > t_hi).
-__device__ __forceinline__ void key_query_range(const BlockArgs &a, const BlockItem &bi, int32_t e,
-                                                int *t_lo, int *t_hi) {
+// when t_lo > t_hi); on the block's tile e is the block token u.
+__device__ __forceinline__ void key_query_range(const BlockArgs &a, const BlockItem &bi, bool block_tile,
+                                                int32_t e, int *t_lo, int *t_hi) {
     const Item &it = bi.it;
     const int never_lo = 1, never_hi = 0, all = 1 << 20;
     *t_lo = never_lo;
     *t_hi = never_hi;
-    if (e >= it.e_end) return;
-    if (bi.block) {
+    if (block_tile) {
         // block key u = e at position n + u: causal from query u on; a ring
         // head keeps it while it is within `ring` of the query (or a sink key)
+        if (e >= a.q_len) return;
         const int32_t n = a.d.seq_len[it.b];
         *t_lo = e;
         *t_hi = (!it.ring || n + e < a.d.sink) ? all : e + a.d.ring - 1;
         return;
     }
+    if (e >= it.e_end) return;
     if (!it.ring || e < a.d.sink) {
         // full head rows, sink slots: every query (sink slots only once written)
         if (!it.ring || e < it.n_sink) {
@@ -250,7 +238,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
     __shared__ float red_sum[4][NP];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = a.n_cache_items + d.batch * d.hkv;
+    const int n_items = a.n_cache_items;
     if (threadIdx.x == 0) {
         for (int i = 0; i < ST; ++i) {
             mbar_init(&kv_full[i], 1);
@@ -318,8 +306,8 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                     if (jg >= ST && !(ok = mbar_wait(&kv_empty[st], ((jg / ST) - 1) & 1))) break;
                     char *ks = sKV + st * kDecStageBytes;
                     mbar_expect_tx(&kv_full[st], kDecStageBytes);
-                    if (bi.block) {
-                        // rows u >= q_len are outside the tensor: zero-filled
+                    if (t == bi.cache_tiles) {
+                        // the block's keys; rows u >= q_len are outside the tensor: zero-filled
                         tma_load_4d(ks, &a.tm_bk, 0, it.g, 0, it.b, &kv_full[st]);
                         tma_load_4d(ks + kDecHalfBytes, &a.tm_bk, 64, it.g, 0, it.b, &kv_full[st]);
                         tma_load_4d(ks + kDecTileBytes, &a.tm_bv, 0, it.g, 0, it.b, &kv_full[st]);
@@ -467,11 +455,12 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 tmem_ld_wait();
 #pragma unroll
                 for (int cb = 0; cb < NH; cb += 4) blk_reg_fence4(&sr[cb]);
-                const int32_t e = it.e_begin + t * kTok + r;
+                const bool block_tile = t == bi.cache_tiles;
+                const int32_t e = block_tile ? r : it.e_begin + t * kTok + r;
                 int t_lo, t_hi;
-                key_query_range(a, bi, e, &t_lo, &t_hi);
+                key_query_range(a, bi, block_tile, e, &t_lo, &t_hi);
                 // a full head's tile inside the cached length: every key for every query
-                const bool dense = !bi.block && !it.ring && it.e_begin + (t + 1) * kTok <= it.e_end;
+                const bool dense = !block_tile && !it.ring && it.e_begin + (t + 1) * kTok <= it.e_end;
                 float s[NH];
                 bool exceed = false;
 #pragma unroll
@@ -630,8 +619,8 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
     }
 }
 
-// Folds the cache splits, the block item and the sink logit of every
-// (sequence, block token, query head).
+// Folds the splits (the last one holds the block's keys too) and the sink
+// logit of every (sequence, block token, query head).
 template <int kQ>
 __global__ void __launch_bounds__(kD) decode_block_merge(const __grid_constant__ BlockArgs a) {
     using C = BlockCfg<kQ>;
@@ -648,13 +637,12 @@ __global__ void __launch_bounds__(kD) decode_block_merge(const __grid_constant__
     const float *part = d.part + ((size_t)b * d.hkv + g) * a.part_slots * C::PartFloats;
     const bool has_sink = d.sink_logit != nullptr;
     const float sig = has_sink ? d.sink_logit[h] * kLog2eF : -INFINITY;
-    auto slot = [&](int i) { return i < splits ? i : a.part_slots - 1; };   // cache splits, then the block
     float M = sig;
-    for (int i = 0; i <= splits; ++i) M = fmaxf(M, part[slot(i) * C::PartFloats + row]);
+    for (int i = 0; i < splits; ++i) M = fmaxf(M, part[i * C::PartFloats + row]);
     float den = 0.f, num = 0.f;
     if (M != -INFINITY) {
-        for (int i = 0; i <= splits; ++i) {
-            const float *ps = part + slot(i) * C::PartFloats;
+        for (int i = 0; i < splits; ++i) {
+            const float *ps = part + i * C::PartFloats;
             const float ms = ps[row];
             if (ms == -INFINITY) continue;
             const float f = ex2_approx(ms - M);

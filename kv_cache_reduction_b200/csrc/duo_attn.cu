@@ -211,17 +211,18 @@ DecodePlan plan_decode(const duo_params *p, const Layout &L, int64_t max_n, int 
     return d;
 }
 
-// The block decode's plan.  Each item (split of a full head, ring head, the
-// block's own keys) carries a fixed cost that grows with the query rows it
-// holds (staging their Q, filling the pipeline, writing their partials), so
-// the full heads' split count is chosen on the makespan of the persistent
-// CTAs' round-robin share of ALL the items, in tiles plus that cost.
+// The block decode's plan.  Each item (split of a full head, ring head; the
+// last split of each also takes the block's own tile) carries a fixed cost
+// that grows with the query rows it holds (staging their Q, filling the
+// pipeline, writing their partials), so the full heads' split count is chosen
+// on the makespan of the persistent CTAs' round-robin share of all the items,
+// in tiles plus that cost.
 DecodePlan plan_block(const duo_params *p, const Layout &L, int64_t max_n, int sms, int rows) {
     DecodePlan d = plan_decode(p, L, max_n, sms);
     const double item = 1.0 + rows / 10.0;          // per-item cost in tiles (measured ~6 at 48 rows)
     const int64_t full_units = (int64_t)p->batch * L.n_full;
     const int64_t ring_items = (int64_t)p->batch * L.n_ring * d.splits_ring;
-    const int64_t block_items = (int64_t)p->batch * p->num_kv_heads;
+    const int64_t block_items = 0;                  // the block's tiles ride on the last splits
     if (full_units > 0) {
         const int64_t tiles = cdiv(std::max<int64_t>(max_n, 1), duo::kTok);
         const double c_ring = (double)cdiv(d.chunk_ring, duo::kTok) + item, c_block = 1.0 + item;
@@ -580,7 +581,7 @@ size_t duo_decode_block_workspace_bytes(const duo_params *params, int32_t q_len,
     int sms = 148;
     if (check_device(&sms)) sms = 148;
     const DecodePlan d = plan_block(params, L, max_seq_len, sms, duo::kGroup * q_len);
-    const size_t slots = (size_t)std::max(d.splits_full, d.splits_ring) + 1;
+    const size_t slots = (size_t)std::max(d.splits_full, d.splits_ring);
     const size_t partials = (size_t)params->batch * params->num_kv_heads * slots *
                             (size_t)(duo::kGroup * q_len) * (duo::kD + 2) * sizeof(float);
     return (partials + 255) / 256 * 256 + 256;       // + the work-item counter
@@ -647,7 +648,7 @@ int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, cons
     da.splits_full = d.splits_full;
     da.chunk_ring = d.chunk_ring;
     da.splits_ring = d.splits_ring;
-    da.max_splits = std::max(d.splits_full, d.splits_ring) + 1;
+    da.max_splits = std::max(d.splits_full, d.splits_ring);
     da.n_items = (int32_t)d.items;
     da.scale_log2 = params->softmax_scale * duo::kLog2eF;
     da.gate = (const __nv_bfloat16 *)gate_values;
@@ -666,7 +667,7 @@ int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, cons
     a.work_counter = (int32_t *)((char *)workspace + (need - 256));
     if (cudaMemsetAsync(a.work_counter, 0, sizeof(int32_t), (cudaStream_t)stream) != cudaSuccess)
         return fail(DUO_ERR_CUDA, "zeroing the block decode's work counter failed");
-    const int64_t items = d.items + (int64_t)params->batch * params->num_kv_heads;
+    const int64_t items = d.items;
     const int grid = (int)std::min<int64_t>(items, sms);
     const int64_t merge_blocks = (int64_t)params->batch * q_len * params->num_q_heads;
     cudaStream_t st = (cudaStream_t)stream;
