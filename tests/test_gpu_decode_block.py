@@ -76,12 +76,38 @@ def test_block_decode_output_gate(cuda_device, mode):
 
 
 @pytest.mark.slow
-def test_block_decode_long_context(cuda_device):
-    """B=8, context 32768, a block of 8: the verify shape at the decode_b32 context."""
-    p, o = layers(8, full_mask=inputs.seeded_full_mask(2002, 2))
+def test_block_decode_bench_shape_sampled(cuda_device):
+    """The verify_b32 line's call: B=32, context 32768, decode_b32's head mask, a
+    block of 8; every row of three sequences against the oracle, the cache
+    untouched, every output finite."""
+    w = inputs.workload("decode_b32")
+    B, n, k = w.batch, w.seq_len, 8
+    p, o = layers(B, full_mask=w.full_mask)
     rng = np.random.default_rng(106)
-    cache = random_cache(p, 32768, [32768] * 8, rng.integers(0, 256, size=8).tolist(), seed=107)
-    block_case(p, o, cache, 8, seed=108, max_seq_len=32768)
+    cache = random_cache(p, n, [n] * B, rng.integers(0, 256, size=B).tolist(), seed=107)
+    q = inputs.randn_bf16((B, k, 48, 128), 108, "cuda")
+    kn = inputs.randn_bf16((B, k, 8, 128), 109, "cuda")
+    vn = inputs.randn_bf16((B, k, 8, 128), 110, "cuda")
+    out = torch.full((B, k, 48, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, k, 48), float("nan"), dtype=torch.float32, device="cuda")
+    nb = duo.duo_decode_block_workspace_bytes(p, k, n)
+    ws = torch.full(((nb + 255) // 256 * 256,), 0x7f, dtype=torch.uint8, device="cuda")
+    before = (cache.seq_len.clone(), cache.ring_head.clone(), cache.full_k[0, 0, :64].clone(),
+              cache.strm_v[B - 1, 0].clone())
+    duo.duo_attn_decode_block(p, cache, q, kn, vn, n, out, lse, ws)
+    torch.cuda.synchronize()
+    assert duo.duo_get_device_status() == duo.DUO_OK
+    assert torch.equal(before[0], cache.seq_len) and torch.equal(before[1], cache.ring_head)
+    assert torch.equal(before[2], cache.full_k[0, 0, :64]) and torch.equal(before[3], cache.strm_v[B - 1, 0])
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    snap = host_cache(o, cache)
+    seqs = (0, 17, 31)
+    rows = [(b * k + t) * 48 + h for b in seqs for t in range(k) for h in range(48)]
+    ref_o, ref_l = oracle.attn_decode_block(o, snap, inputs.bits(q), inputs.bits(kn), inputs.bits(vn),
+                                            rows=rows)
+    got_o = out[list(seqs)].reshape(-1, 128)
+    got_l = lse[list(seqs)].reshape(-1)
+    assert_close(got_o, ref_o, got_l, ref_l, "verify_b32 shape")
 
 
 def test_block_decode_rejects_long_blocks(cuda_device):
