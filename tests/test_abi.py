@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import kv_cache_reduction_b200 as duo
 from kv_cache_reduction_b200 import build as duo_build
@@ -177,3 +178,18 @@ def test_workspace_size_is_host_arithmetic(lib):
     assert n > 0 and n % 4 == 0
     assert duo.duo_decode_workspace_bytes(p, 64) <= n
     assert duo.duo_decode_workspace_bytes(_params(head_dim=64), 128) == 0
+
+
+def test_gate_shape_picks_the_mode():
+    """The binding reads the gate mode from the gate's shape: out's shape is one
+    gate per channel, out's shape without the channel dimension one per head."""
+    out = torch.zeros((2, 3, 48, 128), dtype=torch.bfloat16)
+    g = duo._gate(torch.zeros_like(out), out)
+    assert g._obj.mode == duo.DUO_GATE_PER_ELEMENT
+    g = duo._gate(torch.zeros((2, 3, 48), dtype=torch.bfloat16), out)
+    assert g._obj.mode == duo.DUO_GATE_PER_HEAD
+    assert duo._gate(None, out) is None
+    with pytest.raises(ValueError):
+        duo._gate(torch.zeros((2, 3, 48, 64), dtype=torch.bfloat16), out)
+    with pytest.raises(ValueError):
+        duo._gate(torch.zeros((2, 3, 48), dtype=torch.float32), out)
