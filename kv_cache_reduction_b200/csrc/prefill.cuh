@@ -9,14 +9,16 @@
 //
 // A CTA computes 128-row query tiles for two query heads of one GQA group,
 // so both heads share every K/V tile in shared memory.  CTAs are persistent
-// (one per SM) and walk a static list of (sequence, head pair, query tile)
-// work tiles, heaviest query tiles first.  Keys come in 128-key tiles.
+// (one per SM) and take (sequence, head pair, query tile) work tiles from a
+// list ordered heaviest first: each claims its next one from an atomic
+// counter when it is ready for it.  Keys come in 128-key tiles.
 //   warps 0-7  softmax of head 0, warps 8-15 softmax of head 1: each query
 //              row is split over two warps (64 keys each, the row max joined
 //              through shared memory); they read S from TMEM, write P (bf16)
 //              back over the first 64 columns of S, rescale O in TMEM only when
-//              the running max grew by more than 2^8, and write O / l and the
-//              log-sum-exp at the end of each work tile.  The two heads take
+//              the running max grew by more than 2^8, and write O / l (times
+//              the output gate, if any) by TMA stores and the log-sum-exp at
+//              the end of each work tile.  The two heads take
 //              turns for the exponentials, so that the MUFU units serve one head
 //              while the tensor core runs the other head's PV and next S
 //   warp 16    TMA producer: claims the work tiles (an atomic counter in the
