@@ -131,23 +131,33 @@ __global__ void __launch_bounds__(kPrepThreads) qk_prep_append(const __grid_cons
             const bool is_q = r < a.hq;
             float x[8];
             unpack8(xin[u], x);
-            float ss = 0.f;
+            // pairs of channels through the packed f32x2 pipe
+            f2 ss2 = f2_mul(f2_make(x[0], x[1]), f2_make(x[0], x[1]));
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+            for (int e = 2; e < 8; e += 2) ss2 = f2_fma(f2_make(x[e], x[e + 1]), f2_make(x[e], x[e + 1]), ss2);
+            float ss = f2_sum(ss2);
             // the 16 threads of a row are 16 consecutive lanes: reduce within them
 #pragma unroll
             for (int m = 1; m < 16; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-            const float inv = rsqrtf(ss * (1.f / 128.f) + a.rms_eps);
-            float y[8], p[8];
+            const f2 inv2 = f2_splat(rsqrtf(ss * (1.f / 128.f) + a.rms_eps));
+            f2 y2[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = x[e] * inv * (is_q ? wq[e] : wk[e]);
+            for (int e = 0; e < 4; ++e)
+                y2[e] = f2_mul(f2_mul(f2_make(x[2 * e], x[2 * e + 1]), inv2),
+                               is_q ? f2_make(wq[2 * e], wq[2 * e + 1]) : f2_make(wk[2 * e], wk[2 * e + 1]));
+            f2 p2[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) p[e] = __shfl_xor_sync(0xffffffffu, y[e], 8);   // channel +-64
+            for (int e = 0; e < 4; ++e) {
+                p2[e].x = __shfl_xor_sync(0xffffffffu, y2[e].x, 8);   // channel +-64
+                p2[e].y = __shfl_xor_sync(0xffffffffu, y2[e].y, 8);
+            }
             uint32_t o[4];
 #pragma unroll
-            for (int e = 0; e < 8; e += 2)
-                o[e / 2] = pack_bf16x2(fmaf(p[e], s8[e], y[e] * c8[e]),
-                                       fmaf(p[e + 1], s8[e + 1], y[e + 1] * c8[e + 1]));
+            for (int e = 0; e < 4; ++e) {
+                const f2 r2 = f2_fma(p2[e], f2_make(s8[2 * e], s8[2 * e + 1]),
+                                     f2_mul(y2[e], f2_make(c8[2 * e], c8[2 * e + 1])));
+                o[e] = pack_bf16x2(r2.x, r2.y);
+            }
             if (!active) continue;
             const uint4 out = make_uint4(o[0], o[1], o[2], o[3]);
             row_ptr(r)[j] = out;
