@@ -415,21 +415,21 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 const bool my_turn = mbar_wait(&turn[h], jg & 1);
                 __syncwarp();
                 if (!__all_sync(0xffffffffu, my_turn)) { ok = false; break; }
-                float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+                // score * c - max on the packed f32x2 pipe, two columns per instruction
+                const f2 c2 = f2_splat(c), ms2 = f2_splat(-m_sub);
+                f2 ls01 = f2_splat(0.f), ls23 = f2_splat(0.f);
 #pragma unroll
                 for (int ch = 0; ch < 2; ++ch) {
                     uint32_t pw[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
                         const int cc = ch * 32 + e;
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[cc]), c, -m_sub));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[cc + 1]), c, -m_sub));
-                        const float p2 = ex2_approx(fmaf(__uint_as_float(sr[cc + 2]), c, -m_sub));
-                        const float p3 = ex2_approx(fmaf(__uint_as_float(sr[cc + 3]), c, -m_sub));
-                        ls0 += p0;
-                        ls1 += p1;
-                        ls2 += p2;
-                        ls3 += p3;
+                        const f2 a01 = f2_fma(f2_make(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), c2, ms2);
+                        const f2 a23 = f2_fma(f2_make(__uint_as_float(sr[cc + 2]), __uint_as_float(sr[cc + 3])), c2, ms2);
+                        const float p0 = ex2_approx(a01.x), p1 = ex2_approx(a01.y);
+                        const float p2 = ex2_approx(a23.x), p3 = ex2_approx(a23.y);
+                        ls01 = f2_add(ls01, f2_make(p0, p1));
+                        ls23 = f2_add(ls23, f2_make(p2, p3));
                         pw[e / 2] = pack_bf16x2(p0, p1);
                         pw[e / 2 + 1] = pack_bf16x2(p2, p3);
                     }
@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&turn[h ^ 1]);
-                l_run = l_run * alpha + ((ls0 + ls1) + (ls2 + ls3));
+                l_run = l_run * alpha + ((ls01.x + ls01.y) + (ls23.x + ls23.y));
                 m_run = m_use;
                 // O holds the previous key tiles' sum (its PV is complete: this S
                 // was computed after it); rescale this half's 64 columns when the
