@@ -652,6 +652,16 @@ def run_ours(args, world, rank):
                       "ms_per_step": round(t_e2e * 1e3, 4)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline and getattr(wl, "oracle_sample", None) is not None:
         res["cpu_baseline"] = wl.oracle_sample(args.cpu_budget)
+        # the same oracle on one host thread, on a shorter bounded sample
+        import oracle
+        n_threads = oracle.num_threads()
+        oracle.set_num_threads(1)
+        try:
+            one = wl.oracle_sample(max(1.0, args.cpu_budget / 3))
+        finally:
+            oracle.set_num_threads(n_threads)
+        res["cpu_baseline"]["single_thread"] = {"value": one["value"], "unit": one["unit"],
+                                                "cores": 1, "sample": one["sample"]}
     # the other workloads of the path, on this GPU, as context for the main line
     if args.secondary and args.workload == "decode_b32":
         del wl
