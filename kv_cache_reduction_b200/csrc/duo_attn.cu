@@ -1,6 +1,7 @@
 // duo_attn.cu -- the C ABI of libduoattn.so: argument checks, work
 // planning and kernel launches.  Every check runs on the host before the
 // first launch, so a call that returns an error has launched nothing.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -144,16 +145,18 @@ int launch_status(const char *what) {
     return DUO_OK;
 }
 
-// Raises a kernel's dynamic shared-memory limit once per device.
+// Raises a kernel's dynamic shared-memory limit once per device.  The flags
+// are atomic because host threads may launch concurrently; two threads that
+// both see a flag clear both set the attribute, which is harmless.
 template <typename Kernel>
-int set_smem_once(Kernel kernel, size_t bytes, const char *name, bool (&done)[64]) {
+int set_smem_once(Kernel kernel, size_t bytes, const char *name, std::atomic<bool> (&done)[64]) {
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && done[dev]) return DUO_OK;
+    if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire)) return DUO_OK;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
         cudaSuccess)
         return fail(DUO_ERR_CUDA, "cudaFuncSetAttribute(%s) failed", name);
-    if (dev >= 0 && dev < 64) done[dev] = true;
+    if (dev >= 0 && dev < 64) done[dev].store(true, std::memory_order_release);
     return DUO_OK;
 }
 
@@ -313,7 +316,7 @@ constexpr int kMaxBlock = 8;     // block decode: query tokens per call
 
 template <int kQ>
 int launch_block(duo::BlockArgs &a, int grid, cudaStream_t st, int64_t merge_blocks) {
-    static bool smem_set[64] = {};
+    static std::atomic<bool> smem_set[64] = {};
     int rc;
     if ((rc = set_smem_once(duo::decode_block_split<kQ>, duo::BlockCfg<kQ>::Smem, "decode_block_split",
                             smem_set)))
@@ -504,7 +507,7 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     memcpy(a.ring_head_of, L.ring_head_of, sizeof a.ring_head_of);
     a.heads = L.heads;
     cudaStream_t st = (cudaStream_t)stream;
-    static bool smem_set[64] = {};
+    static std::atomic<bool> smem_set[64] = {};
     if ((rc = set_smem_once(duo::decode_split, duo::kDecSmem, "decode_split", smem_set))) return rc;
     if (d.items > 0) {
         duo::decode_split<<<(unsigned)d.grid, duo::kDecThreads, duo::kDecSmem, st>>>(a);

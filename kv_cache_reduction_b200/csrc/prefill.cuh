@@ -40,6 +40,8 @@
 
 #include <cuda.h>
 
+#include <atomic>
+
 #include "ptx.cuh"
 
 namespace duo {
@@ -625,16 +627,17 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     for (int g = 0; g < p->num_kv_heads; ++g)
         a.kind[g] = sliding ? kKindSliding : (is_full[g] ? kKindFull : kKindStreaming);
     void (*kernel)(PrefillArgs) = gate_mode == 1 ? prefill_fwd<1> : gate_mode == 2 ? prefill_fwd<2> : prefill_fwd<0>;
-    static bool smem_set[3][64] = {};
+    // set once per device and instantiation (atomic: host threads may launch concurrently)
+    static std::atomic<bool> smem_set[3][64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !smem_set[gate_mode][dev]) {
+    if (dev < 0 || dev >= 64 || !smem_set[gate_mode][dev].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmem) !=
             cudaSuccess) {
             snprintf(err, err_len, "cudaFuncSetAttribute(prefill_fwd) failed");
             return DUO_ERR_CUDA;
         }
-        if (dev >= 0 && dev < 64) smem_set[gate_mode][dev] = true;
+        if (dev >= 0 && dev < 64) smem_set[gate_mode][dev].store(true, std::memory_order_release);
     }
     a.batch_pairs = B * (p->num_q_heads / 2);
     const int64_t n_work = (int64_t)a.batch_pairs * a.n_qtiles;
