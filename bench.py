@@ -172,10 +172,7 @@ class DecodeB32:
         self.out = torch.empty((B, 48, 128), dtype=torch.bfloat16, device="cuda")
         self.lse = torch.empty((B, 48), dtype=torch.float32, device="cuda")
         self.ws = duo.workspace_for(self.params, n)
-        # algorithmic bytes: K and V rows each head reads, plus q and out
-        n_full, n_ring = self.params.n_full, self.params.n_ring
-        rows = B * (n_full * n + n_ring * min(n, inputs.SINK + inputs.RECENT))
-        self.bytes = rows * 2 * 128 * 2 + 2 * self.q.numel() * 2
+        self.bytes = decode_bytes(B, n, self.params.n_full, self.params.n_ring)
         self.launches_per_step = 2
         self.unit = "GB/s"
         self.kernel = "decode_split + decode_merge (one duo_attn_decode call)"
@@ -243,6 +240,25 @@ def attended_pairs(L: int, span):
         return L * (L + 1) // 2
     m = min(L, span)
     return m * (m + 1) // 2 + (L - m) * span
+
+
+def prefill_flops(w) -> int:
+    """Algorithmic FLOPs of one prefill of workload w (48 query heads, 6 per KV
+    head): 4 * 128 per attended (query, key) pair and query head (QK^T and PV,
+    2 * 128 each); masked tile area, padding and the sink term are not counted."""
+    pairs = 0
+    for g in range(8):
+        span = w.window if w.window else (None if w.full_mask[g] else inputs.SINK + inputs.RECENT)
+        pairs += 6 * attended_pairs(w.seq_len, span)
+    return 4 * 128 * pairs * w.batch
+
+
+def decode_bytes(batch: int, n: int, n_full: int, n_ring: int) -> int:
+    """Algorithmic bytes of one one-token decode at context n: the K and V rows
+    (2 x 128 bf16 each) every KV head attends to, read once for its 6 query
+    heads, plus q and out (48 x 128 bf16 each per sequence)."""
+    rows = batch * (n_full * n + n_ring * min(n, inputs.SINK + inputs.RECENT))
+    return rows * 2 * 128 * 2 + 2 * batch * 48 * 128 * 2
 
 
 class Stack40:
@@ -384,11 +400,7 @@ class Prefill:
             self.q, self.k = inputs.rmsnorm_bf16(self.q), inputs.rmsnorm_bf16(self.k)
         self.out = torch.empty_like(self.q)
         self.lse = torch.empty((B, 48, L), dtype=torch.float32, device="cuda")
-        pairs = 0
-        for g in range(8):
-            span = w.window if w.window else (None if w.full_mask[g] else inputs.SINK + inputs.RECENT)
-            pairs += 6 * attended_pairs(L, span)
-        self.flops = 4 * 128 * pairs * B
+        self.flops = prefill_flops(w)
         self.ws = torch.empty(duo.duo_prefill_workspace_bytes(), dtype=torch.uint8, device="cuda")
         self.launches_per_step = 1      # prefill_fwd (plus a 4-byte memset of its work counter)
         self.unit = "TFLOP/s"

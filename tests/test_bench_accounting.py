@@ -1,0 +1,84 @@
+"""The roofline numerators bench.py reports, pinned to the oracle's attended-set
+rule: prefill FLOPs count 4 * 128 per attended (query, key) pair and query head,
+decode bytes count each attended K/V row once per KV head.  The pair counts come
+from the oracle (brute force over its per-pair rule for small L, its cumulative
+count for large L), never from the closed form under test."""
+import pytest
+
+import bench
+import oracle
+from kv_cache_reduction_b200 import inputs
+
+
+def _layer(kind: str) -> oracle.Layer:
+    if kind == "full":
+        return oracle.Layer(1, 6, 1, 128, inputs.SINK, inputs.RECENT, 0, full_mask=(1,))
+    if kind == "streaming":
+        return oracle.Layer(1, 6, 1, 128, inputs.SINK, inputs.RECENT, 0, full_mask=(0,))
+    return oracle.Layer(1, 6, 1, 128, 0, 0, inputs.WINDOW, full_mask=(0,))
+
+
+def _span(kind: str):
+    return {"full": None, "streaming": inputs.SINK + inputs.RECENT, "sliding": inputs.WINDOW}[kind]
+
+
+@pytest.mark.parametrize("kind", ["full", "streaming", "sliding"])
+@pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 255, 256, 319, 320, 321, 511, 512, 513, 700])
+def test_pair_count_matches_brute_force_over_the_oracle_rule(kind, L):
+    layer = _layer(kind)
+    if L <= 321:
+        brute = sum(oracle.attended(layer, 0, i, j) for i in range(L) for j in range(L))
+    else:
+        brute = oracle.count_pairs(layer, 0, L)
+    assert bench.attended_pairs(L, _span(kind)) == brute
+
+
+@pytest.mark.parametrize("kind", ["full", "streaming", "sliding"])
+@pytest.mark.parametrize("L", [16384, 32768])
+def test_pair_count_matches_the_oracle_at_workload_lengths(kind, L):
+    assert bench.attended_pairs(L, _span(kind)) == oracle.count_pairs(_layer(kind), 0, L)
+
+
+def test_prefill_flops_of_the_two_prefill_workloads():
+    # prefill_16k: 12 query heads on full KV heads, 36 on streaming ones, B=1
+    w = inputs.workload("prefill_16k")
+    assert sum(w.full_mask) == 2
+    full = oracle.count_pairs(_layer("full"), 0, w.seq_len)
+    strm = oracle.count_pairs(_layer("streaming"), 0, w.seq_len)
+    assert bench.prefill_flops(w) == 4 * 128 * (12 * full + 36 * strm) * w.batch
+    assert bench.prefill_flops(w) == pytest.approx(920.38e9, rel=1e-5)
+    # sliding_32k: all 48 query heads on the 512-key band, B=2
+    w = inputs.workload("sliding_32k")
+    band = oracle.count_pairs(_layer("sliding"), 0, w.seq_len)
+    assert bench.prefill_flops(w) == 4 * 128 * 48 * band * w.batch
+    assert bench.prefill_flops(w) == pytest.approx(818.20e9, rel=1e-5)
+
+
+@pytest.mark.parametrize("n", [1, 63, 64, 320, 321, 1000, 32768])
+def test_decode_bytes_count_the_last_rows_attended_keys(n):
+    # keys the decode query (position n - 1) attends: the oracle's cumulative
+    # pair count at n minus the one at n - 1
+    def last_row(kind):
+        layer = _layer(kind)
+        return oracle.count_pairs(layer, 0, n) - (oracle.count_pairs(layer, 0, n - 1) if n > 1 else 0)
+
+    B, n_full, n_ring = 3, 2, 6
+    rows = B * (n_full * last_row("full") + n_ring * last_row("streaming"))
+    q_out = 2 * B * 48 * 128 * 2
+    assert bench.decode_bytes(B, n, n_full, n_ring) == rows * 512 + q_out
+
+
+def test_decode_bytes_of_the_main_workload():
+    w = inputs.workload("decode_b32")
+    assert sum(w.full_mask) == 2
+    assert bench.decode_bytes(w.batch, w.seq_len, 2, 6) == 1_105_985_536
+
+
+@pytest.mark.parametrize("L", range(1, 14))
+@pytest.mark.parametrize("sink,recent,window", [(2, 3, 0), (0, 1, 0), (3, 1, 0), (0, 0, 4), (0, 0, 1)])
+def test_pair_count_matches_brute_force_with_small_spans(L, sink, recent, window):
+    # every band edge is crossed within L <= 13
+    layer = oracle.Layer(1, 6, 1, 128, sink, recent, window, full_mask=(0,))
+    brute = sum(oracle.attended(layer, 0, i, j) for i in range(L) for j in range(L))
+    span = window if window else sink + recent
+    assert bench.attended_pairs(L, span) == brute
