@@ -253,12 +253,47 @@ def prefill_flops(w) -> int:
     return 4 * 128 * pairs * w.batch
 
 
-def decode_bytes(batch: int, n: int, n_full: int, n_ring: int) -> int:
-    """Algorithmic bytes of one one-token decode at context n: the K and V rows
-    (2 x 128 bf16 each) every KV head attends to, read once for its 6 query
-    heads, plus q and out (48 x 128 bf16 each per sequence)."""
-    rows = batch * (n_full * n + n_ring * min(n, inputs.SINK + inputs.RECENT))
+def decode_bytes(batch: int, n: int, n_full: int, n_ring: int,
+                 span: int = inputs.SINK + inputs.RECENT) -> int:
+    """Algorithmic bytes of one one-token decode at context n (the query at
+    position n - 1, already appended): the K and V rows (2 x 128 bf16 each) every
+    KV head attends to, read once for its 6 query heads, plus q and out (48 x 128
+    bf16 each per sequence).  A ring head (sink + recent, or a sliding window)
+    attends min(n, span) rows."""
+    rows = batch * (n_full * n + n_ring * min(n, span))
     return rows * 2 * 128 * 2 + 2 * batch * 48 * 128 * 2
+
+
+def block_ring_rows(n: int, sink: int, recent: int) -> int:
+    """Cached rows of one streaming head that a verify block attends to: its
+    queries sit at positions n, n + 1, ... of a cache of n tokens, so the union
+    of their bands is the sink plus the recent - 1 cached tokens before n (the
+    first query's band reaches back the furthest)."""
+    return min(n, sink) + max(0, min(n - sink, recent - 1))
+
+
+def verify_bytes(batch: int, n: int, q_len: int, n_full: int, n_ring: int,
+                 sink: int = inputs.SINK, recent: int = inputs.RECENT) -> int:
+    """Algorithmic bytes of one verify-block decode: the cached K/V rows the
+    block's queries attend to (each read once for all of them), the block's own
+    K/V rows, and the block's q and out."""
+    rows = batch * (n_full * n + n_ring * block_ring_rows(n, sink, recent)) + \
+        batch * (n_full + n_ring) * q_len
+    return rows * 2 * 128 * 2 + 2 * batch * q_len * 48 * 128 * 2
+
+
+def stack_bytes(w) -> int:
+    """Algorithmic bytes of one decode step through the layer stack of workload
+    w: each DuoAttention layer's full and streaming heads, each sliding layer's
+    window ring."""
+    total = 0
+    for mask in inputs.stack_layer_masks(w):
+        if mask is None:
+            total += decode_bytes(w.batch, w.seq_len, 0, 8, inputs.WINDOW)
+        else:
+            n_full = sum(1 for m in mask if m)
+            total += decode_bytes(w.batch, w.seq_len, n_full, 8 - n_full)
+    return total
 
 
 class Stack40:
@@ -274,16 +309,14 @@ class Stack40:
         seed = rank_seed(w.seed, rank)
         rng = np.random.default_rng(seed)
         self.layers = []
-        self.bytes = 0
+        self.bytes = stack_bytes(w)
         max_ws = 0
         for li, mask in enumerate(masks):
             if mask is None:
                 sig = inputs.randn_f32((48,), seed * 100 + li, "cuda")
                 p = duo.DuoParams(B, 48, 8, 128, 0, 0, inputs.WINDOW, 128 ** -0.5, (0,) * 8, sig)
-                span = inputs.WINDOW
             else:
                 p = duo.DuoParams(B, 48, 8, 128, inputs.SINK, inputs.RECENT, 0, 128 ** -0.5, mask, None)
-                span = inputs.SINK + inputs.RECENT
             cache = duo.DuoCache.allocate(p, n)
             for i, t in enumerate((cache.full_k, cache.full_v, cache.strm_k, cache.strm_v)):
                 if t is not None:
@@ -296,8 +329,6 @@ class Stack40:
             out = torch.empty((B, 48, 128), dtype=torch.bfloat16, device="cuda")
             lse = torch.empty((B, 48), dtype=torch.float32, device="cuda")
             self.layers.append((p, cache, q, out, lse))
-            rows = B * (p.n_full * n + p.n_ring * min(n, span))
-            self.bytes += rows * 512 + 2 * q.numel() * 2
             max_ws = max(max_ws, duo.duo_decode_workspace_bytes(p, n))
         self.ws = torch.zeros((max_ws + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
         self.launches_per_step = 2 * len(self.layers)
@@ -438,8 +469,7 @@ class VerifyB32(DecodeB32):
         nb = duo.duo_decode_block_workspace_bytes(self.params, k, n)
         self.wsb = torch.zeros((nb + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
         n_full, n_ring = self.params.n_full, self.params.n_ring
-        rows = B * (n_full * n + n_ring * min(n, inputs.SINK + inputs.RECENT)) + B * 8 * k
-        self.bytes = rows * 2 * 128 * 2 + 2 * self.qb.numel() * 2
+        self.bytes = verify_bytes(B, n, k, n_full, n_ring)
         self.kernel = "decode_block_split + decode_block_merge (one duo_attn_decode_block call)"
 
     def step(self):

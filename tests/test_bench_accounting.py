@@ -82,3 +82,49 @@ def test_pair_count_matches_brute_force_with_small_spans(L, sink, recent, window
     brute = sum(oracle.attended(layer, 0, i, j) for i in range(L) for j in range(L))
     span = window if window else sink + recent
     assert bench.attended_pairs(L, span) == brute
+
+
+def _block_union(layer: oracle.Layer, n: int, q_len: int) -> int:
+    """Keys that any query of a block at positions n .. n + q_len - 1 attends,
+    by brute force over the oracle's per-pair rule."""
+    keys = set()
+    for t in range(q_len):
+        i = n + t
+        keys.update(j for j in range(i + 1) if oracle.attended(layer, 0, i, j))
+    return len(keys)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 5, 7, 9, 12, 20])
+@pytest.mark.parametrize("q_len", [1, 3, 8])
+@pytest.mark.parametrize("sink,recent", [(2, 3), (0, 4), (3, 1), (0, 1)])
+def test_verify_ring_rows_match_the_union_of_the_blocks_bands(n, q_len, sink, recent):
+    layer = oracle.Layer(1, 6, 1, 128, sink, recent, 0, full_mask=(0,))
+    # the union holds the cached keys plus all q_len keys of the block itself
+    assert bench.block_ring_rows(n, sink, recent) + q_len == _block_union(layer, n, q_len)
+
+
+def test_verify_bytes_of_the_verify_workload():
+    w = inputs.workload("decode_b32")
+    n, q_len = w.seq_len, 8
+    ring = _block_union(_layer("streaming"), n, q_len) - q_len
+    assert ring == inputs.SINK + inputs.RECENT - 1
+    rows = w.batch * (2 * n + 6 * ring) + w.batch * 8 * q_len
+    assert bench.verify_bytes(w.batch, n, q_len, 2, 6) == rows * 512 + 2 * w.batch * q_len * 48 * 128 * 2
+
+
+def test_stack_bytes_of_the_forty_layer_step():
+    w = inputs.workload("stack40")
+    n = w.seq_len
+
+    def last_row(kind):          # keys the query at position n - 1 attends
+        layer = _layer(kind)
+        return sum(oracle.attended(layer, 0, n - 1, j) for j in range(n))
+
+    per_full_layer = w.batch * (2 * last_row("full") + 6 * last_row("streaming")) * 512
+    per_sliding_layer = w.batch * 8 * last_row("sliding") * 512
+    q_out = 2 * w.batch * 48 * 128 * 2
+    masks = inputs.stack_layer_masks(w)
+    assert sum(m is None for m in masks) == 30 and all(sum(m) == 2 for m in masks if m is not None)
+    want = 10 * per_full_layer + 30 * per_sliding_layer + 40 * q_out
+    assert bench.stack_bytes(w) == want
+    assert want == pytest.approx(22.65e9, rel=1e-3)
