@@ -24,6 +24,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -91,18 +92,58 @@ def aggregate(units_per_rank: float, world: int, seconds_max: float) -> float:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """SM clock and clock-event reasons of this process's GPU while a timed
+    region runs.  With NVML, a thread polls back to back between begin() and
+    end(), which time_steps calls around its timed region; the GPU is found
+    by its PCI address, so a remapped device visibility cannot pick another
+    one.  Without NVML, nvidia-smi samples every 200 ms around the region."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
     def __init__(self, device_index: int):
         self.idx = device_index
         self.proc = None
         self.path = None
+        self.nv = None
+        self.handle = None
+        self.max_mhz = None
+        self.rows = []                 # (SM MHz, clock-event reason bits) per NVML sample
+        self.active = threading.Event()
+        self.done = threading.Event()
+        self.thread = None
+
+    def _nvml(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            props = torch.cuda.get_device_properties(self.idx)
+            want = (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            for i in range(nv.nvmlDeviceGetCount()):
+                h = nv.nvmlDeviceGetHandleByIndex(i)
+                pci = nv.nvmlDeviceGetPciInfo(h)
+                if (pci.domain, pci.bus, pci.device) == want:
+                    return nv, h
+        except Exception:
+            pass
+        return None, None
 
     def __enter__(self):
+        self.nv, self.handle = self._nvml()
+        if self.handle is not None:
+            try:
+                self.max_mhz = self.nv.nvmlDeviceGetMaxClockInfo(self.handle, self.nv.NVML_CLOCK_SM)
+                self.thread = threading.Thread(target=self._poll, daemon=True)
+                self.thread.start()
+                return self
+            except Exception:
+                self.handle = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -113,9 +154,33 @@ class ClockSampler:
             time.sleep(0.3)
         except OSError:
             self.proc = None
+            os.unlink(self.path)
+            self.path = None
         return self
 
+    def _poll(self):
+        nv, h = self.nv, self.handle
+        reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.done.is_set():
+            if not self.active.is_set():
+                time.sleep(0.0005)
+                continue
+            try:      # back to back while the region runs (each query releases the GIL)
+                self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), reasons(h)))
+            except Exception:
+                return
+
+    def begin(self):
+        self.active.set()
+
+    def end(self):
+        self.active.clear()
+
     def __exit__(self, *exc):
+        self.done.set()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -124,6 +189,8 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        if self.handle is not None:
+            return self._nvml_summary()
         if self.proc is None or not self.path:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         rows = []
@@ -147,7 +214,23 @@ class ClockSampler:
                     reasons.add(n)
         busy = [r[0] for r in rows] or [0.0]
         return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(r[1] for r in rows),
-                "samples": len(rows), "reasons": sorted(reasons)}
+                "samples": len(rows), "reasons": sorted(reasons),
+                "source": "nvidia-smi every 200 ms around the timed region"}
+
+    def _nvml_summary(self):
+        nv = self.nv
+        masks = [(name, getattr(nv, attr, 0)) for name, attr in self.REASONS]
+        idle = getattr(nv, "nvmlClocksEventReasonGpuIdle", 0)
+        # samples the driver flags as idle (the region's first microseconds) are
+        # left out of the median under load
+        loaded = [r for r in self.rows if not (r[1] & idle)] or self.rows
+        out = {"sm_mhz": statistics.median(r[0] for r in loaded) if loaded else None,
+               "sm_max_mhz": self.max_mhz, "samples": len(loaded),
+               "reasons": sorted({name for _, bits in self.rows for name, m in masks if bits & m}),
+               "source": "NVML, polled during the timed region"}
+        if not loaded:
+            out["reasons"] = ["no samples"]
+        return out
 
 
 # ------------------------------------------------------------------ workloads
@@ -571,7 +654,7 @@ WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40, "decode_small": Decode
 PREROLL_CYCLES = 2_000_000     # ~1 ms device spin queued ahead of the start event
 
 
-def time_steps(fn, steps, stream, world):
+def time_steps(fn, steps, stream, world, clocks=None):
     """Device time of `steps` calls of fn: CUDA events on the launching stream,
     barrier + synchronize on both sides.  A ~1 ms spin kernel is queued before
     the start event, so the host's time to issue the first step's launches is
@@ -583,10 +666,14 @@ def time_steps(fn, steps, stream, world):
     with torch.cuda.stream(stream):
         torch.cuda._sleep(PREROLL_CYCLES)
     start.record(stream)
+    if clocks is not None:
+        clocks.begin()
     for _ in range(steps):
         fn()
     stop.record(stream)
     torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.end()
     barrier(world)
     return start.elapsed_time(stop) / 1e3
 
@@ -603,7 +690,7 @@ def measure(wl, steps, warmup, world):
     if status != duo.DUO_OK:
         raise RuntimeError(f"device status {status} during warm-up")
     with ClockSampler(torch.cuda.current_device()) as clk:
-        t = time_steps(wl.step, steps, stream, world)
+        t = time_steps(wl.step, steps, stream, world, clk)
     t = max_over_ranks(t, world)
     status = duo.duo_get_device_status()
     if status != duo.DUO_OK:
@@ -757,7 +844,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(k for k in WORKLOADS if k != "decode_small"),
