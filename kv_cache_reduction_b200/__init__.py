@@ -5,7 +5,10 @@ Thin ctypes binding over ``libduoattn.so`` (the C ABI declared in
 marshal arguments: torch tensors are passed as device pointers and the
 current CUDA stream as the stream handle.  Every step of the attention runs
 in the library's CUDA kernels; there is no Python or CPU fallback, and a
-missing library raises ``DuoLibraryMissing``.
+missing library raises ``DuoLibraryMissing``.  Before a call reaches the
+library, the binding checks what plain pointers cannot carry: each tensor's
+dtype, shape, contiguity and device (the current CUDA device), raising
+``ValueError``; the library checks the rest and raises ``DuoError``.
 
 Layouts (bf16 unless noted):
   prefill  q [B][L][Hq][D], k/v [B][L][Hkv][D] -> out [B][L][Hq][D], lse fp32 [B][Hq][L]
@@ -103,7 +106,8 @@ class DuoQKPrep:
     def as_c(self) -> _Prep:
         return _Prep(self.rope_theta, self.rope_factor, self.original_max_position, self.beta_fast,
                      self.beta_slow, self.attention_factor, self.rms_eps,
-                     _ptr(self.q_norm_weight), _ptr(self.k_norm_weight))
+                     _arg(self.q_norm_weight, "q_norm_weight", torch.bfloat16, (128,), optional=True),
+                     _arg(self.k_norm_weight, "k_norm_weight", torch.bfloat16, (128,), optional=True))
 
 
 class _Params(ctypes.Structure):
@@ -194,7 +198,9 @@ class DuoParams:
         self._mask_buf = (ctypes.c_uint8 * max(1, len(self.full_mask)))(*[int(m) for m in self.full_mask])
         return _Params(self.batch, self.num_q_heads, self.num_kv_heads, self.head_dim, self.sink,
                        self.recent, self.window, float(self.softmax_scale),
-                       ctypes.addressof(self._mask_buf), _ptr(self.sink_logit))
+                       ctypes.addressof(self._mask_buf),
+                       _arg(self.sink_logit, "sink_logit", torch.float32, (self.num_q_heads,),
+                            optional=True))
 
     @property
     def n_full(self) -> int:
@@ -232,9 +238,22 @@ class DuoCache:
                         torch.zeros((B,), dtype=torch.int32, device=device),
                         torch.zeros((B,), dtype=torch.int32, device=device))
 
-    def as_c(self) -> _Cache:
-        return _Cache(_ptr(self.full_k), _ptr(self.full_v), int(self.capacity), _ptr(self.strm_k),
-                      _ptr(self.strm_v), _ptr(self.seq_len), _ptr(self.ring_head))
+    def as_c(self, params: Optional["DuoParams"] = None) -> _Cache:
+        """The duo_cache; with params, each tensor is checked against the layer's
+        geometry first (a part the layer does not use is passed as NULL)."""
+        if params is None:
+            return _Cache(_ptr(self.full_k), _ptr(self.full_v), int(self.capacity), _ptr(self.strm_k),
+                          _ptr(self.strm_v), _ptr(self.seq_len), _ptr(self.ring_head))
+        B, D, bf = params.batch, params.head_dim, torch.bfloat16
+        full = (B, params.n_full, int(self.capacity), D)
+        ring = (B, params.n_ring, params.ring_slots, D)
+        fk = _arg(self.full_k, "cache.full_k", bf, full) if params.n_full else None
+        fv = _arg(self.full_v, "cache.full_v", bf, full) if params.n_full else None
+        sk = _arg(self.strm_k, "cache.strm_k", bf, ring) if params.n_ring else None
+        sv = _arg(self.strm_v, "cache.strm_v", bf, ring) if params.n_ring else None
+        return _Cache(fk, fv, int(self.capacity), sk, sv,
+                      _arg(self.seq_len, "cache.seq_len", torch.int32, (B,)),
+                      _arg(self.ring_head, "cache.ring_head", torch.int32, (B,)))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -243,6 +262,55 @@ def _ptr(t: Optional[torch.Tensor]):
     if not t.is_contiguous():
         raise ValueError("tensors passed to the library must be contiguous")
     return t.data_ptr()
+
+
+def _on_device(t: torch.Tensor, name: str) -> None:
+    """A tensor the kernels will read or write: contiguous and on the current
+    CUDA device (a host or another GPU's pointer would fault in the kernel)."""
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    cur = torch.cuda.current_device()
+    if t.device.index is not None and t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device}, but the current CUDA device is cuda:{cur}")
+
+
+def _arg(t: Optional[torch.Tensor], name: str, dtype: torch.dtype, shape, optional: bool = False):
+    """The device pointer of t after checking its dtype, its shape (None leaves
+    a dimension free), contiguity and device; None for an optional None."""
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype})")
+    if t.dim() != len(shape) or any(s is not None and int(d) != s for d, s in zip(t.shape, shape)):
+        want = "[" + ", ".join("*" if s is None else str(s) for s in shape) + "]"
+        raise ValueError(f"{name} has shape {list(t.shape)}, expected {want}")
+    _on_device(t, name)
+    return t.data_ptr()
+
+
+def _workspace(ws: Optional[torch.Tensor]):
+    """(pointer, bytes) of a workspace tensor (any dtype), or (None, 0)."""
+    if ws is None:
+        return None, 0
+    _on_device(ws, "workspace")
+    return ws.data_ptr(), ws.numel() * ws.element_size()
+
+
+def _one_token(params: "DuoParams", t: Optional[torch.Tensor], name: str, dtype: torch.dtype,
+               tail, optional: bool = False):
+    """A one-token decode tensor: [B][tail...] or [B][1][tail...]."""
+    lead = (params.batch, 1) if t is not None and t.dim() == 2 + len(tail) else (params.batch,)
+    return _arg(t, name, dtype, lead + tuple(tail), optional)
+
+
+def _gate_arg(gate: Optional[torch.Tensor], out: torch.Tensor):
+    if gate is not None:
+        _on_device(gate, "gate")
+    return _gate(gate, out)
 
 
 def _stream(stream) -> Optional[int]:
@@ -262,9 +330,11 @@ def _check(rc: int) -> int:
 def duo_kv_append(params: DuoParams, cache: DuoCache, k: torch.Tensor, v: torch.Tensor,
                   n_new: Optional[int] = None, stream=None) -> None:
     n_new = int(k.shape[1]) if n_new is None else int(n_new)
-    p, c = params.as_c(), cache.as_c()
-    _check(load_library().duo_kv_append(ctypes.byref(p), ctypes.byref(c), _ptr(k), _ptr(v), n_new,
-                                        _stream(stream)))
+    p, c = params.as_c(), cache.as_c(params)
+    shape = (params.batch, n_new, params.num_kv_heads, params.head_dim)
+    _check(load_library().duo_kv_append(ctypes.byref(p), ctypes.byref(c),
+                                        _arg(k, "k", torch.bfloat16, shape),
+                                        _arg(v, "v", torch.bfloat16, shape), n_new, _stream(stream)))
 
 
 def duo_kv_append_prep(params: DuoParams, cache: DuoCache, prep: DuoQKPrep, q: torch.Tensor,
@@ -273,9 +343,13 @@ def duo_kv_append_prep(params: DuoParams, cache: DuoCache, prep: DuoQKPrep, q: t
     """RMSNorm + YaRN RoPE of q [B][n][Hq][D] and k [B][n][Hkv][D] in place at
     positions seq_len[b] + t, then the append of the prepared k with v."""
     n_new = int(k.shape[1]) if n_new is None else int(n_new)
-    p, c, pr = params.as_c(), cache.as_c(), prep.as_c()
+    p, c, pr = params.as_c(), cache.as_c(params), prep.as_c()
+    B, D, bf = params.batch, params.head_dim, torch.bfloat16
+    kv = (B, n_new, params.num_kv_heads, D)
     _check(load_library().duo_kv_append_prep(ctypes.byref(p), ctypes.byref(c), ctypes.byref(pr),
-                                             _ptr(q), _ptr(k), _ptr(v), n_new, _stream(stream)))
+                                             _arg(q, "q", bf, (B, n_new, params.num_q_heads, D)),
+                                             _arg(k, "k", bf, kv), _arg(v, "v", bf, kv), n_new,
+                                             _stream(stream)))
 
 
 def duo_prefill_workspace_bytes() -> int:
@@ -291,12 +365,19 @@ def duo_attn_prefill(params: DuoParams, q: torch.Tensor, k: torch.Tensor, v: tor
     duo_prefill_workspace_bytes() bytes (dynamic, balanced order).  gate: None,
     or bf16 gate pre-activations [B][L][Hq][D] (per channel) or [B][L][Hq] (per
     head); out is then multiplied by sigmoid(gate)."""
-    L = int(q.shape[1]) if seq_len is None else int(seq_len)
+    Lq = int(q.shape[1]) if q is not None and q.dim() == 4 else -1
+    L = Lq if seq_len is None else int(seq_len)
+    if L not in (0, Lq):
+        raise ValueError(f"seq_len {L} must be q's length {Lq} (or 0 for an empty prompt)")
     p = params.as_c()
-    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(load_library().duo_attn_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), L, _ptr(out),
-                                           _ptr(lse), _ptr(workspace), nbytes, _gate(gate, out),
-                                           _stream(stream)))
+    B, D, bf = params.batch, params.head_dim, torch.bfloat16
+    qs, kvs = (B, Lq, params.num_q_heads, D), (B, Lq, params.num_kv_heads, D)
+    ws, nbytes = _workspace(workspace)
+    _check(load_library().duo_attn_prefill(ctypes.byref(p), _arg(q, "q", bf, qs), _arg(k, "k", bf, kvs),
+                                           _arg(v, "v", bf, kvs), L, _arg(out, "out", bf, qs),
+                                           _arg(lse, "lse", torch.float32, (B, params.num_q_heads, Lq),
+                                                optional=True),
+                                           ws, nbytes, _gate_arg(gate, out), _stream(stream)))
 
 
 def duo_decode_workspace_bytes(params: DuoParams, max_seq_len: int) -> int:
@@ -308,11 +389,13 @@ def duo_attn_decode(params: DuoParams, cache: DuoCache, q: torch.Tensor, max_seq
                     out: torch.Tensor, lse: Optional[torch.Tensor], workspace: torch.Tensor,
                     stream=None, gate: Optional[torch.Tensor] = None) -> None:
     """gate: None, or bf16 gate pre-activations [B][Hq][D] or [B][Hq]."""
-    p, c = params.as_c(), cache.as_c()
-    nbytes = workspace.numel() * workspace.element_size()
-    _check(load_library().duo_attn_decode(ctypes.byref(p), ctypes.byref(c), _ptr(q), int(max_seq_len),
-                                          _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
-                                          _gate(gate, out), _stream(stream)))
+    p, c = params.as_c(), cache.as_c(params)
+    Hq, D, bf = params.num_q_heads, params.head_dim, torch.bfloat16
+    ws, nbytes = _workspace(workspace)
+    _check(load_library().duo_attn_decode(ctypes.byref(p), ctypes.byref(c), _one_token(params, q, "q", bf, (Hq, D)),
+                                          int(max_seq_len), _one_token(params, out, "out", bf, (Hq, D)),
+                                          _one_token(params, lse, "lse", torch.float32, (Hq,), optional=True),
+                                          ws, nbytes, _gate_arg(gate, out), _stream(stream)))
 
 
 def duo_decode_block_workspace_bytes(params: DuoParams, q_len: int, max_seq_len: int) -> int:
@@ -328,12 +411,17 @@ def duo_attn_decode_block(params: DuoParams, cache: DuoCache, q: torch.Tensor, k
     """Verify-block decode: q [B][k][Hq][D] at positions seq_len[b] + t against
     the cache plus the block's own k_new / v_new [B][k][Hkv][D]; the cache is
     not modified."""
-    p, c = params.as_c(), cache.as_c()
-    nbytes = workspace.numel() * workspace.element_size()
-    _check(load_library().duo_attn_decode_block(ctypes.byref(p), ctypes.byref(c), _ptr(q), _ptr(k_new),
-                                                _ptr(v_new), int(q.shape[1]), int(max_seq_len), _ptr(out),
-                                                _ptr(lse), _ptr(workspace), nbytes, _gate(gate, out),
-                                                _stream(stream)))
+    p, c = params.as_c(), cache.as_c(params)
+    B, D, bf = params.batch, params.head_dim, torch.bfloat16
+    k = int(q.shape[1]) if q is not None and q.dim() == 4 else -1
+    qs, kvs = (B, k, params.num_q_heads, D), (B, k, params.num_kv_heads, D)
+    ws, nbytes = _workspace(workspace)
+    _check(load_library().duo_attn_decode_block(ctypes.byref(p), ctypes.byref(c), _arg(q, "q", bf, qs),
+                                                _arg(k_new, "k_new", bf, kvs), _arg(v_new, "v_new", bf, kvs),
+                                                k, int(max_seq_len), _arg(out, "out", bf, qs),
+                                                _arg(lse, "lse", torch.float32, (B, k, params.num_q_heads),
+                                                     optional=True),
+                                                ws, nbytes, _gate_arg(gate, out), _stream(stream)))
 
 
 def duo_attn_decode_static(params: DuoParams, cache: DuoCache, q: torch.Tensor, max_seq_len: int,
@@ -342,10 +430,13 @@ def duo_attn_decode_static(params: DuoParams, cache: DuoCache, q: torch.Tensor, 
     """duo_attn_decode with the library's built-in 16 MiB scratch instead of a
     caller workspace, for callers that cannot allocate device memory when they
     decode.  Calls that may overlap on the GPU share that scratch and race."""
-    p, c = params.as_c(), cache.as_c()
-    _check(load_library().duo_attn_decode_static(ctypes.byref(p), ctypes.byref(c), _ptr(q),
-                                                 int(max_seq_len), _ptr(out), _ptr(lse),
-                                                 _gate(gate, out), _stream(stream)))
+    p, c = params.as_c(), cache.as_c(params)
+    Hq, D, bf = params.num_q_heads, params.head_dim, torch.bfloat16
+    _check(load_library().duo_attn_decode_static(
+        ctypes.byref(p), ctypes.byref(c), _one_token(params, q, "q", bf, (Hq, D)), int(max_seq_len),
+        _one_token(params, out, "out", bf, (Hq, D)),
+        _one_token(params, lse, "lse", torch.float32, (Hq,), optional=True),
+        _gate_arg(gate, out), _stream(stream)))
 
 
 def duo_cache_bytes(params: DuoParams, capacity: int, seq_len: int) -> CacheStats:
