@@ -50,9 +50,11 @@ _lib = None
 
 
 def _load():
+    """The compiled oracle: liboracle.so, or the copy DUO_ORACLE_LIB names (the
+    mutation tests point it at deliberately broken builds of duo_oracle.c)."""
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
+        lib = ctypes.CDLL(os.environ.get("DUO_ORACLE_LIB") or build())
         P, C = ctypes.POINTER(_Params), ctypes.POINTER(_Cache)
         vp, i64 = ctypes.c_void_p, ctypes.c_int64
         lib.oracle_attended.argtypes = [P, ctypes.c_int32, i64, i64]
