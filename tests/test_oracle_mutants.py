@@ -110,3 +110,76 @@ def test_every_mutant_fails_a_pin(tmp_path):
     # each mutant failed on a pin's assertion, not on a crash or a collection error
     for what, (rc, out) in results.items():
         assert rc == 1 and "failed" in out, f"{what}: pytest exited {rc}\n{out}"
+
+
+# ------------------------------------------------------------ the Python parts
+# (module, what the mistake is, the text it replaces, its replacement)
+PY_MUTANTS = [
+    ("oracle/prep.py", "rotation pairs adjacent channels",
+     "a, b = y[..., : D // 2], y[..., D // 2:]", "a, b = y[..., 0::2], y[..., 1::2]"),
+    ("oracle/prep.py", "rotation in the opposite direction",
+     "[a * c - b * s, b * c + a * s]", "[a * c + b * s, b * c - a * s]"),
+    ("oracle/prep.py", "YaRN ramp reversed",
+     "base * (1.0 - ramp) + (base / factor) * ramp", "base * ramp + (base / factor) * (1.0 - ramp)"),
+    ("oracle/prep.py", "YaRN lower bound rounded up",
+     "lo = max(math.floor(pair_index_for_turns(beta_fast)), 0)",
+     "lo = max(math.ceil(pair_index_for_turns(beta_fast)), 0)"),
+    ("oracle/prep.py", "YaRN beta_fast and beta_slow swapped",
+     "lo = max(math.floor(pair_index_for_turns(beta_fast)), 0)\n    hi = min(math.ceil(pair_index_for_turns(beta_slow)), d - 1)",
+     "lo = max(math.floor(pair_index_for_turns(beta_slow)), 0)\n    hi = min(math.ceil(pair_index_for_turns(beta_fast)), d - 1)"),
+    ("oracle/prep.py", "RMSNorm eps outside the square root",
+     "np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)",
+     "(np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps)"),
+    ("oracle/prep.py", "attention_factor dropped",
+     "b * c + a * s], axis=-1) * attention_factor", "b * c + a * s], axis=-1)"),
+    ("oracle/prep.py", "bf16 rounding ties away from zero",
+     "r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)",
+     "r = np.ldexp(np.trunc(np.ldexp(m, 8) + np.copysign(0.5, m)), e - 8)"),
+    ("oracle/prep.py", "bf16 rounding to 7 significant bits",
+     "r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)", "r = np.ldexp(np.rint(np.ldexp(m, 7)), e - 7)"),
+    ("oracle/__init__.py", "sigmoid of the negated gate",
+     "return 1.0 / (1.0 + np.exp(-x))", "return 1.0 / (1.0 + np.exp(x))"),
+    ("oracle/__init__.py", "per-head prefill gate read from the next head",
+     "gv = g[b, i, h, :] if mode == GATE_PER_ELEMENT else g[b, i, h][:, None]",
+     "gv = g[b, i, h, :] if mode == GATE_PER_ELEMENT else g[b, i, (h + 1) % Hq][:, None]"),
+    ("oracle/__init__.py", "per-channel decode gate read from the next head",
+     "gv = g[b, h, :] if mode == GATE_PER_ELEMENT else g[b, h][:, None]",
+     "gv = g[b, (h + 1) % Hq, :] if mode == GATE_PER_ELEMENT else g[b, h][:, None]"),
+]
+PY_PINS = ["tests/test_oracle_prep.py", "tests/test_oracle_gate.py"]
+
+# Runs the pins with one oracle module's source replaced in place: the module is
+# imported, the mutated text is executed over its namespace, then pytest runs.
+_BOOT = r"""
+import importlib, sys
+sys.path.insert(0, {root!r})
+mod = importlib.import_module({module!r})
+src = open(mod.__file__).read()
+assert src.count({old!r}) == 1
+exec(compile(src.replace({old!r}, {new!r}), mod.__file__, "exec"), mod.__dict__)
+import pytest
+sys.exit(pytest.main(["-x", "-q", "-p", "no:cacheprovider", "-m", "not gpu", *{pins!r}]))
+"""
+
+
+def _py_pins(module_file: str, old: str, new: str):
+    module = module_file[:-3].replace("/", ".").removesuffix(".__init__")
+    code = _BOOT.format(root=ROOT, module=module, old=old, new=new, pins=PY_PINS)
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600, env=dict(os.environ, OMP_NUM_THREADS="1"))
+    return r.returncode, r.stdout[-2000:] + r.stderr[-1000:]
+
+
+def test_every_python_mutant_fails_a_pin():
+    for module_file, what, old, new in PY_MUTANTS:
+        assert open(os.path.join(ROOT, module_file)).read().count(old) == 1, f"site not unique: {what}"
+    jobs = [("unmutated", "oracle/prep.py", "D = 128", "D = 128")] + \
+        [(what, m, old, new) for m, what, old, new in PY_MUTANTS]
+    with concurrent.futures.ThreadPoolExecutor(min(len(jobs), os.cpu_count() or 2)) as pool:
+        results = dict(zip([j[0] for j in jobs], pool.map(lambda j: _py_pins(*j[1:]), jobs)))
+    rc, out = results.pop("unmutated")
+    assert rc == 0, "the unmutated modules must pass their pins:\n" + out
+    survivors = [what for what, (rc, _) in results.items() if rc == 0]
+    assert not survivors, f"mutants no pin caught: {survivors}"
+    for what, (rc, out) in results.items():
+        assert rc == 1 and "failed" in out, f"{what}: exited {rc}\n{out}"

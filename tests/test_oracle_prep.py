@@ -3,15 +3,19 @@
 * plain RoPE: with factor 1 the frequencies are theta^(-2i/D) for every pair;
 * YaRN with the Laguna page's parameters: pairs that turn more than beta_fast
   times over the original 4096 positions keep their frequency, pairs that turn
-  fewer than beta_slow times are divided by the factor (64), and frequencies
-  fall monotonically in between (the method's definition in turns, not its
-  formula in pair indices);
+  fewer than beta_slow times are divided by the factor (64), every pair
+  strictly between is blended (strictly between the two), and frequencies fall
+  monotonically (the method's definition in turns, not its formula in pair
+  indices);
 * the rotation equals multiplication of the complex numbers y_i + i y_(i+64)
   by exp(i p f_i) (an independent formulation), is the identity at position
   0, keeps each pair's norm, and makes query-key dot products depend only on
   the position difference (the defining property of rotary embeddings);
 * RMSNorm: unit root-mean-square with unit weight and eps 0, invariance to a
-  positive scale of the input;
+  positive scale of the input, torch's own rms_norm (eps inside the root) on
+  rows small enough for eps to matter, and 1/sqrt(2) for a constant row whose
+  mean square equals eps;
+* attention_factor scales the rotated rows;
 * bf16 rounding: ties to even, and single rounding of float64 (no detour
   through float32).
 """
@@ -35,14 +39,15 @@ def test_yarn_page_parameters_by_turns():
     f = prep.yarn_inv_freq(**PAGE)
     base = PAGE["theta"] ** (-np.arange(64) / 64.0)
     turns = PAGE["original_max"] * base / (2 * math.pi)   # full turns over the original context
-    fast = turns > PAGE["beta_fast"] * 1.5                # clearly above beta_fast
-    slow = turns < PAGE["beta_slow"] / 1.5                # clearly below beta_slow
+    fast = turns > PAGE["beta_fast"]                      # above beta_fast: kept
+    slow = turns < PAGE["beta_slow"]                      # below beta_slow: interpolated
     assert fast.sum() >= 8 and slow.sum() >= 16
     assert np.array_equal(f[fast], base[fast])
     assert np.allclose(f[slow], base[slow] / PAGE["factor"], rtol=1e-15, atol=0)
     assert np.all(np.diff(f) < 0)                         # monotone: no pair overtakes another
-    mid = ~fast & ~slow
-    assert np.all(f[mid] <= base[mid]) and np.all(f[mid] >= base[mid] / PAGE["factor"])
+    mid = ~fast & ~slow                                   # every pair in between is blended
+    assert mid.sum() >= 8
+    assert np.all(f[mid] < base[mid]) and np.all(f[mid] > base[mid] / PAGE["factor"])
 
 
 def rand(shape, seed, scale=1.0):
@@ -71,6 +76,14 @@ def test_rotation_identity_at_zero_and_pair_norms_kept():
     assert np.allclose(n_in, n_out, rtol=1e-12, atol=0)
 
 
+def test_attention_factor_scales_the_rotated_rows():
+    y = rand((2, 3, 2, 128), 9)
+    f = prep.yarn_inv_freq(**PAGE)
+    pos = np.full(y.shape[:3], 777.0)
+    assert np.allclose(prep.rotate(y, pos, f, 0.75), 0.75 * prep.rotate(y, pos, f, 1.0), rtol=1e-15, atol=0)
+    assert np.allclose(prep.rotate(y, np.zeros(y.shape[:3]), f, 1.25), 1.25 * y, rtol=1e-15, atol=0)
+
+
 def test_dot_products_depend_only_on_position_difference():
     q, k = rand((1, 1, 1, 128), 4), rand((1, 1, 1, 128), 5)
     f = prep.yarn_inv_freq(**PAGE)
@@ -87,6 +100,16 @@ def test_rmsnorm_unit_rms_and_scale_invariance():
     assert np.allclose(prep.rmsnorm(3.5 * x, None, 0.0), y, rtol=1e-14, atol=0)
     w = rand(128, 7)
     assert np.allclose(prep.rmsnorm(x, w, 0.0), y * w, rtol=1e-15, atol=0)
+
+
+def test_rmsnorm_matches_torch_where_eps_matters():
+    import torch
+    x = rand((6, 128), 10, scale=2e-3)                    # mean square ~ eps
+    w = 1 + 0.1 * rand(128, 11)
+    want = torch.nn.functional.rms_norm(torch.from_numpy(x), (128,), torch.from_numpy(w), 1e-6)
+    assert np.allclose(prep.rmsnorm(x, w, 1e-6), want.numpy(), rtol=1e-13, atol=0)
+    c = np.full((1, 128), 1e-3)                           # mean square 1e-6 = eps
+    assert np.allclose(prep.rmsnorm(c, None, 1e-6), 2 ** -0.5, rtol=1e-14, atol=0)
 
 
 def test_bf16_rounding_ties_to_even_and_single_rounding():
