@@ -12,6 +12,7 @@
 #include "decode.cuh"
 #include "decode_block.cuh"
 #include "kv_append.cuh"
+#include "plan.h"
 #include "prefill.cuh"
 #include "ptx.cuh"
 #include "qk_prep.cuh"
@@ -225,29 +226,17 @@ DecodePlan plan_block(const duo_params *p, const Layout &L, int64_t max_n, int s
     const double item = 1.0 + rows / 10.0;          // per-item cost in tiles (measured ~6 at 48 rows)
     const int64_t full_units = (int64_t)p->batch * L.n_full;
     const int64_t ring_items = (int64_t)p->batch * L.n_ring * d.splits_ring;
-    const int64_t block_items = 0;                  // the block's tiles ride on the last splits
     if (full_units > 0) {
+        // (the block's own tile rides on each full head's last split: no items of its own)
         const int64_t tiles = cdiv(std::max<int64_t>(max_n, 1), duo::kTok);
-        const double c_ring = (double)cdiv(d.chunk_ring, duo::kTok) + item, c_block = 1.0 + item;
+        const double c_ring = (double)cdiv(d.chunk_ring, duo::kTok) + item;
         double best = 1e300;
         for (int64_t s = 1; s <= std::min<int64_t>(tiles, 64); ++s) {
             const int64_t chunk = cdiv(tiles, s), splits = cdiv(tiles, chunk);
-            const int64_t nf = full_units * splits, total = nf + ring_items + block_items;
+            const int64_t nf = full_units * splits, total = nf + ring_items;
             const int64_t g = std::min<int64_t>(total, sms);
-            // items of [start, start + n) that CTA b takes: b, b + g, b + 2g, ...
-            auto count = [g](int64_t b, int64_t start, int64_t n) -> int64_t {
-                if (n <= 0) return 0;
-                const int64_t k0 = start > b ? cdiv(start - b, g) : 0;
-                const int64_t last = start + n - 1;
-                if (last < b) return 0;
-                const int64_t k1 = (last - b) / g;
-                return k1 >= k0 ? k1 - k0 + 1 : 0;
-            };
-            double span = 0.0;
-            for (int64_t b = 0; b < g; ++b)
-                span = std::max(span, count(b, 0, nf) * ((double)chunk + item) +
-                                          count(b, nf, ring_items) * c_ring +
-                                          count(b, nf + ring_items, block_items) * c_block);
+            // the full heads' splits come first in the item list, the ring heads after
+            const double span = duo::round_robin_makespan(nf, (double)chunk + item, ring_items, c_ring, g);
             if (span < best - 1e-9) {
                 best = span;
                 d.chunk_full = (int)(chunk * duo::kTok);
