@@ -161,3 +161,15 @@ def test_sink_logit_and_norm_weights(host_as_device):
         p.as_c()
     with pytest.raises(ValueError, match="q_norm_weight"):
         duo.DuoQKPrep(q_norm_weight=torch.zeros((128,))).as_c()       # fp32, not bf16
+
+
+def test_prep_defaults_are_the_page_rope_parameters():
+    import json
+    import os
+    rope = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_constants.json")))[
+        "rope_full_attention"]["value"]
+    d = duo.DuoQKPrep()
+    assert (d.rope_theta, d.rope_factor, d.original_max_position, d.beta_fast, d.beta_slow,
+            d.attention_factor) == (rope["rope_theta"], rope["factor"],
+                                    rope["original_max_position_embeddings"], rope["beta_fast"],
+                                    rope["beta_slow"], rope["attention_factor"])

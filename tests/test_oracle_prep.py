@@ -19,14 +19,26 @@
 * bf16 rounding: ties to even, and single rounding of float64 (no detour
   through float32).
 """
+import json
 import math
+import os
 
 import numpy as np
 import pytest
 
 from oracle import prep
 
-PAGE = dict(theta=500000.0, factor=64.0, original_max=4096, beta_fast=64.0, beta_slow=1.0)
+# the full-attention layers' rope parameters the Laguna attention article prints
+_ROPE = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_constants.json")))[
+    "rope_full_attention"]["value"]
+PAGE = dict(theta=_ROPE["rope_theta"], factor=_ROPE["factor"],
+            original_max=_ROPE["original_max_position_embeddings"], beta_fast=_ROPE["beta_fast"],
+            beta_slow=_ROPE["beta_slow"])
+
+
+def test_page_rope_parameters():
+    assert PAGE == dict(theta=500000.0, factor=64.0, original_max=4096, beta_fast=64.0, beta_slow=1.0)
+    assert _ROPE["attention_factor"] == 1.0 and _ROPE["partial_rotary_factor"] == 1.0
 
 
 def test_factor_one_is_plain_rope():
