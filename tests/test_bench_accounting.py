@@ -128,3 +128,47 @@ def test_stack_bytes_of_the_forty_layer_step():
     want = 10 * per_full_layer + 30 * per_sliding_layer + 40 * q_out
     assert bench.stack_bytes(w) == want
     assert want == pytest.approx(22.65e9, rel=1e-3)
+
+
+def test_timed_sample_cycles_until_the_budget():
+    import time
+    ran = []
+
+    def run(u):
+        ran.append(u)
+        time.sleep(0.002)
+
+    units = ["a", "b", "c"]
+    done, t, used = bench.timed_sample(units, run, lambda u: 10, 0.025)
+    assert t >= 0.025 and used == len(ran) and done == 10 * used
+    assert used > len(units)                                   # cycled past one pass
+    assert ran[:6] == ["a", "b", "c", "a", "b", "c"]
+    # a budget below one unit still runs one unit; the pass limit caps the rest
+    assert bench.timed_sample(units, lambda u: None, lambda u: 1, 0.0)[2] == 1
+    assert bench.timed_sample(units, lambda u: None, lambda u: 1, 1e9, max_passes=2)[2] == 6
+
+
+def test_decode_cpu_baseline_leg_runs_on_host_tensors():
+    """The bench's CPU-baseline leg of the main line, driven on small host
+    tensors (the leg reads the caches back to the host, so it needs no GPU):
+    it cycles the oracle over whole (sequence, KV head) groups until its
+    budget and reports bytes per second."""
+    import types
+    import torch
+    import kv_cache_reduction_b200 as duo
+
+    wl = object.__new__(bench.DecodeB32)
+    n = 700
+    wl.w = types.SimpleNamespace(seq_len=n)
+    wl.params = duo.DuoParams(2, full_mask=(0, 0, 0, 0, 0, 1, 0, 1))
+    wl.cache = duo.DuoCache.allocate(wl.params, n, device="cpu")
+    for i, t in enumerate((wl.cache.full_k, wl.cache.full_v, wl.cache.strm_k, wl.cache.strm_v)):
+        t.copy_(inputs.randn_bf16(tuple(t.shape), 50 + i, "cpu"))
+    wl.cache.seq_len.fill_(n)
+    wl.cache.ring_head.copy_(torch.tensor([3, 200], dtype=torch.int32))
+    wl.q = inputs.randn_bf16((2, 48, 128), 60, "cpu")
+    r = wl.oracle_sample(0.3)
+    assert r["kind"] == "oracle" and r["unit"] == "GB/s" and r["value"] > 0
+    assert "passes over the 16" in r["sample"]
+    used = int(r["sample"].split()[0])
+    assert used >= 1
