@@ -235,9 +235,11 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ workloads
 class DecodeB32:
-    """One-token decode at context 32768 for 32 sequences."""
+    """One-token decode at context 32768 for 32 sequences.  With product=False
+    only the inputs are built (plain torch, no call into the library), as the
+    reference arm needs them."""
 
-    def __init__(self, rank: int):
+    def __init__(self, rank: int, product: bool = True):
         w = self.w = inputs.workload("decode_b32")
         B, n = w.batch, w.seq_len
         self.params = duo.DuoParams(B, 48, 8, 128, inputs.SINK, inputs.RECENT, 0, 128 ** -0.5,
@@ -254,11 +256,12 @@ class DecodeB32:
         self.q = inputs.randn_bf16((B, 48, 128), seed + 5, "cuda")
         self.out = torch.empty((B, 48, 128), dtype=torch.bfloat16, device="cuda")
         self.lse = torch.empty((B, 48), dtype=torch.float32, device="cuda")
-        self.ws = duo.workspace_for(self.params, n)
+        self.ws = duo.workspace_for(self.params, n) if product else None
         self.bytes = decode_bytes(B, n, self.params.n_full, self.params.n_ring)
         self.launches_per_step = 2
         self.unit = "GB/s"
         self.kernel = "decode_split + decode_merge (one duo_attn_decode call)"
+        self.traffic_key = ("decode_split", "decode_b32")
 
     def step(self):
         duo.duo_attn_decode(self.params, self.cache, self.q, self.w.seq_len, self.out, self.lse,
@@ -287,6 +290,9 @@ class DecodeB32:
 
     # -------------------------------------------------- CPU oracle on a bounded sample
     def oracle_sample(self, budget_s: float = 15.0):
+        """The oracle over whole decode steps: every (sequence, query head) row of
+        the batch in one call, so that its dynamic row schedule keeps every host
+        thread busy (the full heads' long rows outnumber the threads)."""
         import oracle
         p = self.params
         olayer = oracle.Layer(p.batch, 48, 8, 128, p.sink, p.recent, 0, p.softmax_scale,
@@ -298,22 +304,19 @@ class DecodeB32:
         hc.ring_head = self.cache.ring_head.cpu().numpy().astype(np.int32)
         qb = inputs.bits(self.q)
         n = self.w.seq_len
-        units = [(b, g) for b in range(p.batch) for g in range(8)]
+        step_bytes = decode_bytes(p.batch, n, p.n_full, p.n_ring)
+        rows = p.batch * 48
+        threads = oracle.num_threads()
 
-        def run(unit):            # one whole GQA group: its 6 query heads
-            b, g = unit
-            oracle.attn_decode(olayer, hc, qb, rows=[b * 48 + g * 6 + j for j in range(6)])
+        def run(_):
+            oracle.attn_decode(olayer, hc, qb)
 
-        def nbytes(unit):
-            tokens = n if p.full_mask[unit[1]] else min(n, p.sink + p.recent)
-            return tokens * 512 + 6 * 2 * 256
-
-        done_bytes, t_total, used = timed_sample(units, run, nbytes, budget_s)
-        return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
-                "kind": "oracle",
-                "sample": f"{used} (sequence, KV head) groups, {used / len(units):.2f} passes over "
-                          f"the {len(units)} of one decode step (6 query heads each), float64, "
-                          f"{t_total:.1f} s"}
+        done_bytes, t_total, used = timed_sample(["step"], run, lambda _: step_bytes, budget_s)
+        return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": threads,
+                "threads_busy": min(threads, p.batch * p.n_full * 6), "kind": "oracle",
+                "sample": f"{used} whole decode steps ({rows} rows per call, "
+                          f"{p.batch * p.n_full * 6} of them full-head rows of {n} keys), "
+                          f"float64, {t_total:.1f} s"}
 
 
 def timed_sample(units, run, nbytes, budget_s: float, max_passes: int = 64):
@@ -402,7 +405,7 @@ class Stack40:
     the other 30 sliding-window layers (window 512) with sink logits.  The 40
     decode calls are captured once in a CUDA graph and replayed per step."""
 
-    def __init__(self, rank: int):
+    def __init__(self, rank: int, product: bool = True):
         w = self.w = inputs.workload("stack40")
         B, n = w.batch, w.seq_len
         masks = inputs.stack_layer_masks(w)
@@ -429,11 +432,13 @@ class Stack40:
             out = torch.empty((B, 48, 128), dtype=torch.bfloat16, device="cuda")
             lse = torch.empty((B, 48), dtype=torch.float32, device="cuda")
             self.layers.append((p, cache, q, out, lse))
-            max_ws = max(max_ws, duo.duo_decode_workspace_bytes(p, n))
-        self.ws = torch.zeros((max_ws + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+            if product:
+                max_ws = max(max_ws, duo.duo_decode_workspace_bytes(p, n))
+        self.ws = torch.zeros((max_ws + 255) // 256 * 256, dtype=torch.uint8, device="cuda") if product else None
         self.launches_per_step = 2 * len(self.layers)
         self.unit = "GB/s"
         self.kernel = "40 x (decode_split + decode_merge), one CUDA graph"
+        self.traffic_key = ("decode_split", "stack40")
         self.graph = None
 
     def eager_step(self, qs=None):
@@ -481,43 +486,48 @@ class Stack40:
                 "batch_per_gpu": self.w.batch, "context": self.w.seq_len, "layers": 40,
                 "l2": "inputs larger than L2 (22.6 GB of cache per step)"}
 
-    def oracle_sample(self, budget_s: float = 15.0):
+    def _host_layer(self, li, seqs):
+        """The oracle's view of layer li restricted to the sequences seqs."""
         import oracle
-        done_bytes, t_total, used = 0, 0.0, 0
-        for li in (3, 0):                      # one DuoAttention layer, one sliding layer
-            p, cache, q, _, _ = self.layers[li]
-            ol = oracle.Layer(1, 48, 8, 128, p.sink, p.recent, p.window, p.softmax_scale,
-                              tuple(p.full_mask),
-                              None if p.sink_logit is None else p.sink_logit.cpu().numpy())
-            for b in range(2):
-                hc = oracle.Cache(ol, cache.capacity if p.n_full else 1)
-                if p.n_full:
-                    hc.full_k = inputs.bits(cache.full_k[b:b + 1])
-                    hc.full_v = inputs.bits(cache.full_v[b:b + 1])
-                hc.strm_k = inputs.bits(cache.strm_k[b:b + 1])
-                hc.strm_v = inputs.bits(cache.strm_v[b:b + 1])
-                hc.seq_len = cache.seq_len[b:b + 1].cpu().numpy().astype(np.int32)
-                hc.ring_head = cache.ring_head[b:b + 1].cpu().numpy().astype(np.int32)
-                t0 = time.perf_counter()
-                oracle.attn_decode(ol, hc, inputs.bits(q[b:b + 1]))
-                t_total += time.perf_counter() - t0
-                n = self.w.seq_len
-                span = p.window if p.window else p.sink + p.recent
-                done_bytes += (p.n_full * n + p.n_ring * min(n, span)) * 512 + 2 * 48 * 256
-                used += 1
-                if t_total >= budget_s:
-                    break
-        return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
-                "kind": "oracle",
-                "sample": f"{used} (layer, sequence) slices of one step (layers 3 and 0), "
-                          f"float64, {t_total:.1f} s"}
+        p, cache, q, _, _ = self.layers[li]
+        b0, b1 = seqs
+        ol = oracle.Layer(b1 - b0, 48, 8, 128, p.sink, p.recent, p.window, p.softmax_scale,
+                          tuple(p.full_mask), None if p.sink_logit is None else p.sink_logit.cpu().numpy())
+        hc = oracle.Cache(ol, cache.capacity if p.n_full else 1)
+        if p.n_full:
+            hc.full_k = inputs.bits(cache.full_k[b0:b1])
+            hc.full_v = inputs.bits(cache.full_v[b0:b1])
+        hc.strm_k = inputs.bits(cache.strm_k[b0:b1])
+        hc.strm_v = inputs.bits(cache.strm_v[b0:b1])
+        hc.seq_len = cache.seq_len[b0:b1].cpu().numpy().astype(np.int32)
+        hc.ring_head = cache.ring_head[b0:b1].cpu().numpy().astype(np.int32)
+        n = self.w.seq_len
+        nbytes = decode_bytes(b1 - b0, n, p.n_full, p.n_ring, p.window if p.window else p.sink + p.recent)
+        return ol, hc, inputs.bits(q[b0:b1]), nbytes
+
+    def oracle_sample(self, budget_s: float = 15.0):
+        """The oracle on two layers of the step: DuoAttention layer 3 for
+        sequences 0-3 (48 full-head rows of 131072 keys per call, enough to keep
+        the host threads busy) and sliding layer 0 for all 16 sequences."""
+        import oracle
+        units = [self._host_layer(3, (0, 4)), self._host_layer(0, (0, self.w.batch))]
+
+        def run(u):
+            oracle.attn_decode(u[0], u[1], u[2])
+
+        done_bytes, t_total, used = timed_sample(units, run, lambda u: u[3], budget_s)
+        threads = oracle.num_threads()
+        return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": threads,
+                "threads_busy": min(threads, 48), "kind": "oracle",
+                "sample": f"{used} layer calls alternating DuoAttention layer 3 (sequences 0-3) and "
+                          f"sliding layer 0 (all 16 sequences) of one step, float64, {t_total:.1f} s"}
 
 
 class Prefill:
     """Prefill of one layer: prefill_16k (B=1, L=16384, 2 of 8 heads full) or
     sliding_32k (B=2, L=32768, window 512, sink logits, RMSNorm'd Q/K)."""
 
-    def __init__(self, rank: int, name: str):
+    def __init__(self, rank: int, name: str, product: bool = True):
         w = self.w = inputs.workload(name)
         B, L = w.batch, w.seq_len
         seed = rank_seed(w.seed, rank)
@@ -532,18 +542,68 @@ class Prefill:
         self.out = torch.empty_like(self.q)
         self.lse = torch.empty((B, 48, L), dtype=torch.float32, device="cuda")
         self.flops = prefill_flops(w)
-        self.ws = torch.empty(duo.duo_prefill_workspace_bytes(), dtype=torch.uint8, device="cuda")
+        self.ws = torch.empty(duo.duo_prefill_workspace_bytes(), dtype=torch.uint8,
+                              device="cuda") if product else None
         self.launches_per_step = 1      # prefill_fwd (plus a 4-byte memset of its work counter)
         self.unit = "TFLOP/s"
         self.kernel = "prefill_fwd"
+        self.traffic_key = ("prefill_fwd", name)
 
     def step(self):
         duo.duo_attn_prefill(self.params, self.q, self.k, self.v, self.out, self.lse,
                              workspace=self.ws)
 
+    def e2e_buffers(self):
+        self.h_in = [t.cpu().pin_memory() for t in (self.q, self.k, self.v)]
+        self.d_in = [torch.empty_like(t) for t in (self.q, self.k, self.v)]
+        self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h_lse = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
+        return sum(t.numel() * 2 for t in self.h_in), self.h_out.numel() * 2 + self.h_lse.numel() * 4
+
+    def e2e_step(self):
+        for d, h in zip(self.d_in, self.h_in):
+            d.copy_(h, non_blocking=True)
+        duo.duo_attn_prefill(self.params, *self.d_in, self.out, self.lse, workspace=self.ws)
+        self.h_out.copy_(self.out, non_blocking=True)
+        self.h_lse.copy_(self.lse, non_blocking=True)
+
     def config(self):
         return {"workload": f"{self.w.name}: prefill B={self.w.batch}, L={self.w.seq_len}",
-                "window": self.w.window, "full_mask": list(self.w.full_mask)}
+                "window": self.w.window, "full_mask": list(self.w.full_mask),
+                "l2": "inputs larger than L2"}
+
+    def oracle_sample(self, budget_s: float = 15.0):
+        """The oracle on seeded sets of query positions of sequence 0 (every
+        query head of each position in one call), cycled until the budget;
+        TFLOP/s of the attended pairs those rows cover (4 * 128 flop each)."""
+        import oracle
+        w, p = self.w, self.params
+        L = w.seq_len
+        sig = None if p.sink_logit is None else p.sink_logit.cpu().numpy()
+        ol = oracle.Layer(1, 48, 8, 128, p.sink, p.recent, p.window, p.softmax_scale,
+                          tuple(p.full_mask), sig)
+        qb, kb, vb = (inputs.bits(t[:1]) for t in (self.q, self.k, self.v))
+        rng = np.random.default_rng(w.seed + 77)
+        units = []
+        for _ in range(64):
+            pos = np.sort(rng.integers(0, L, size=16))
+            rows = np.asarray([h * L + i for h in range(48) for i in pos], dtype=np.int64)
+            pairs = 0
+            for g in range(8):
+                span = p.window if p.window else (None if p.full_mask[g] else p.sink + p.recent)
+                per = [i + 1 if span is None else min(i + 1, span) for i in pos]
+                pairs += 6 * int(sum(per))
+            units.append((rows, pairs * 4 * 128))
+
+        def run(u):
+            oracle.attn_prefill(ol, qb, kb, vb, rows=u[0])
+
+        done, t_total, used = timed_sample(units, run, lambda u: u[1], budget_s)
+        return {"value": done / t_total / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                "kind": "oracle",
+                "sample": f"{used} calls of 768 rows (16 seeded query positions of sequence 0 x 48 "
+                          f"query heads), {done / 1e9:.1f} GFLOP of attended pairs, float64, "
+                          f"{t_total:.1f} s"}
 
 
 class VerifyB32(DecodeB32):
@@ -554,11 +614,10 @@ class VerifyB32(DecodeB32):
     queries), the block's K/V, q and out."""
 
     Q_LEN = 8
-    e2e_step = None          # the end-to-end and CPU legs belong to the main line
     oracle_sample = None
 
-    def __init__(self, rank: int):
-        super().__init__(rank)
+    def __init__(self, rank: int, product: bool = True):
+        super().__init__(rank, product)
         B, n, k = self.w.batch, self.w.seq_len, self.Q_LEN
         seed = rank_seed(self.w.seed, rank)
         self.qb = inputs.randn_bf16((B, k, 48, 128), seed + 6, "cuda")
@@ -566,15 +625,32 @@ class VerifyB32(DecodeB32):
         self.vb = inputs.randn_bf16((B, k, 8, 128), seed + 8, "cuda")
         self.outb = torch.empty_like(self.qb)
         self.lseb = torch.empty((B, k, 48), dtype=torch.float32, device="cuda")
-        nb = duo.duo_decode_block_workspace_bytes(self.params, k, n)
-        self.wsb = torch.zeros((nb + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+        if product:
+            nb = duo.duo_decode_block_workspace_bytes(self.params, k, n)
+            self.wsb = torch.zeros((nb + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
         n_full, n_ring = self.params.n_full, self.params.n_ring
         self.bytes = verify_bytes(B, n, k, n_full, n_ring)
         self.kernel = "decode_block_split + decode_block_merge (one duo_attn_decode_block call)"
+        self.traffic_key = ("decode_block_split", "verify_b32")
 
     def step(self):
         duo.duo_attn_decode_block(self.params, self.cache, self.qb, self.kb, self.vb, self.w.seq_len,
                                   self.outb, self.lseb, self.wsb)
+
+    def e2e_buffers(self):
+        self.h_in = [t.cpu().pin_memory() for t in (self.qb, self.kb, self.vb)]
+        self.d_in = [torch.empty_like(t) for t in (self.qb, self.kb, self.vb)]
+        self.h_out = torch.empty(self.outb.shape, dtype=self.outb.dtype).pin_memory()
+        self.h_lse = torch.empty(self.lseb.shape, dtype=self.lseb.dtype).pin_memory()
+        return sum(t.numel() * 2 for t in self.h_in), self.h_out.numel() * 2 + self.h_lse.numel() * 4
+
+    def e2e_step(self):
+        for d, h in zip(self.d_in, self.h_in):
+            d.copy_(h, non_blocking=True)
+        duo.duo_attn_decode_block(self.params, self.cache, *self.d_in, self.w.seq_len, self.outb,
+                                  self.lseb, self.wsb)
+        self.h_out.copy_(self.outb, non_blocking=True)
+        self.h_lse.copy_(self.lseb, non_blocking=True)
 
     def config(self):
         return {"workload": "verify_b32: block of 8 query tokens, B=32, context 32768, "
@@ -590,7 +666,7 @@ class Prep:
 
     APPENDS = 64                      # capacity in prompts; the cache is reset when full
 
-    def __init__(self, rank: int):
+    def __init__(self, rank: int, product: bool = True):
         w = self.w = inputs.workload("prefill_16k")
         B, L = w.batch, w.seq_len
         seed = rank_seed(w.seed, rank)
@@ -610,6 +686,7 @@ class Prep:
         self.launches_per_step = 2      # qk_prep_append + kv_append_commit
         self.unit = "GB/s"
         self.kernel = "qk_prep_append"
+        self.traffic_key = ("qk_prep_append", "prep_16k")
 
     def step(self):
         if self.appends == self.APPENDS:
@@ -624,47 +701,129 @@ class Prep:
 
 
 class DecodeSmall:
-    """B=1: a 1024-token prompt is prefilled and appended, then each step
-    appends one token and decodes it (full heads {0,3,5,6}).  Latency-bound:
-    reported in microseconds per step."""
+    """The single-layer workload end to end, B=1, full heads {0,3,5,6}: the
+    1024-token prompt is prefilled and appended, then 16 decode steps each
+    append one token and decode it.  Latency-bound, reported in microseconds:
+    the prompt's prefill, and the decode steps.  The 16 steps (each an append
+    and a decode, four kernels) are captured in one CUDA graph that first puts
+    the cache state back to the end of the prompt; one replay is 16 steps.
+    The caches (about 5 MB) would stay in L2, so L2 is flushed before every
+    timed replay and every timed prefill (and only the call is timed)."""
 
-    def __init__(self, rank: int):
+    STEPS = 16
+
+    def __init__(self, rank: int, product: bool = True):
         w = self.w = inputs.workload("decode_small")
         seed = rank_seed(w.seed, rank)
         self.params = duo.DuoParams(1, 48, 8, 128, inputs.SINK, inputs.RECENT, 0, 128 ** -0.5,
                                     w.full_mask, None)
-        self.cap = w.seq_len + 4096
+        self.n0 = w.seq_len
+        self.cap = w.seq_len + self.STEPS
         self.cache = duo.DuoCache.allocate(self.params, self.cap)
-        q = inputs.randn_bf16((1, w.seq_len, 48, 128), seed, "cuda")
-        k = inputs.randn_bf16((1, w.seq_len, 8, 128), seed + 1, "cuda")
-        v = inputs.randn_bf16((1, w.seq_len, 8, 128), seed + 2, "cuda")
-        out = torch.empty_like(q)
-        duo.duo_attn_prefill(self.params, q, k, v, out, None)
-        duo.duo_kv_append(self.params, self.cache, k, v)
-        self.n = w.seq_len
-        self.k1 = inputs.randn_bf16((1, 1, 8, 128), seed + 3, "cuda")
-        self.v1 = inputs.randn_bf16((1, 1, 8, 128), seed + 4, "cuda")
-        self.q1 = inputs.randn_bf16((1, 48, 128), seed + 5, "cuda")
-        self.out = torch.empty((1, 48, 128), dtype=torch.bfloat16, device="cuda")
-        self.lse = torch.empty((1, 48), dtype=torch.float32, device="cuda")
-        self.ws = duo.workspace_for(self.params, self.cap)
-        self.launches_per_step = 4      # append scatter + commit, decode split + merge
+        self.qp = inputs.randn_bf16((1, w.seq_len, 48, 128), seed + 2, "cuda")
+        self.kp = inputs.randn_bf16((1, w.seq_len, 8, 128), seed, "cuda")
+        self.vp = inputs.randn_bf16((1, w.seq_len, 8, 128), seed + 1, "cuda")
+        self.outp = torch.empty_like(self.qp)
+        self.lsep = torch.empty((1, 48, w.seq_len), dtype=torch.float32, device="cuda")
+        S = self.STEPS
+        self.k1 = inputs.randn_bf16((S, 1, 1, 8, 128), seed + 3, "cuda")
+        self.v1 = inputs.randn_bf16((S, 1, 1, 8, 128), seed + 4, "cuda")
+        self.q1 = inputs.randn_bf16((S, 1, 48, 128), seed + 5, "cuda")
+        self.out = torch.empty((S, 1, 48, 128), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty((S, 1, 48), dtype=torch.float32, device="cuda")
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")   # 2 x L2
         self.unit = "us/step"
         self.kernel = "kv_append_scatter + kv_append_commit + decode_split + decode_merge"
+        self.launches_per_step = 4
+        self.graph = None
+        if product:
+            self.ws_p = torch.empty(duo.duo_prefill_workspace_bytes(), dtype=torch.uint8, device="cuda")
+            self.ws = duo.workspace_for(self.params, self.cap)
+            self.prefill()
+            duo.duo_kv_append(self.params, self.cache, self.kp, self.vp)
+            self.seq0 = self.cache.seq_len.clone()
+            self.ring0 = self.cache.ring_head.clone()
 
-    def step(self):
-        duo.duo_kv_append(self.params, self.cache, self.k1, self.v1)
-        self.n += 1                       # the host knows every sequence's length
-        duo.duo_attn_decode(self.params, self.cache, self.q1, self.n, self.out, self.lse, self.ws)
+    def prefill(self):
+        duo.duo_attn_prefill(self.params, self.qp, self.kp, self.vp, self.outp, self.lsep,
+                             workspace=self.ws_p)
+
+    def steps(self):
+        """The cache back to the end of the prompt, then the 16 decode steps."""
+        self.cache.seq_len.copy_(self.seq0)
+        self.cache.ring_head.copy_(self.ring0)
+        for s in range(self.STEPS):
+            duo.duo_kv_append(self.params, self.cache, self.k1[s], self.v1[s])
+            duo.duo_attn_decode(self.params, self.cache, self.q1[s], self.n0 + s + 1, self.out[s],
+                                self.lse[s], self.ws)
+
+    def capture(self):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.steps()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.steps()
+        torch.cuda.synchronize()
+
+    def replay(self):
+        self.graph.replay()
+
+    def timed_each(self, fn, reps):
+        """Device time of reps calls of fn, L2 flushed before each: CUDA events
+        around every call on the launching stream; returns the mean seconds."""
+        stream = torch.cuda.current_stream()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        torch.cuda.synchronize()
+        for a, b in evs:
+            self.flush.fill_(1)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs) / 1e3 / reps
+
+    def measure_line(self, reps, warmup):
+        self.capture()
+        for _ in range(warmup):
+            self.replay()
+            self.prefill()
+        torch.cuda.synchronize()
+        if duo.duo_get_device_status() != duo.DUO_OK:
+            raise RuntimeError("device status set during warm-up")
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            clk.begin()
+            t_graph = self.timed_each(self.replay, reps)
+            t_eager = self.timed_each(self.steps, reps)
+            t_prefill = self.timed_each(self.prefill, reps)
+            clk.end()
+        if duo.duo_get_device_status() != duo.DUO_OK:
+            raise RuntimeError("device status set during timing")
+        S = self.STEPS
+        return {"value": round(t_graph / S * 1e6, 2), "unit": "us/step", "higher_is_better": False,
+                "steps": reps * S, "kernel": self.kernel,
+                "prefill_us": round(t_prefill * 1e6, 2),
+                "eager_us_per_step": round(t_eager / S * 1e6, 2),
+                "gpu_launches": reps * (S * self.launches_per_step + 1),
+                "note": "decode steps replayed from one CUDA graph of 16 steps (append + decode each); "
+                        "prefill_us: the 1024-token prompt's duo_attn_prefill; L2 flushed before "
+                        "every timed call",
+                "clocks": clk.summary()}
 
     def config(self):
-        return {"workload": "decode_small: B=1, 1024-token prompt, then append one token + decode per step"}
+        return {"workload": "decode_small: B=1, prefill of a 1024-token prompt, then 16 x "
+                            "(append one token + decode)"}
 
 
 WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40, "decode_small": DecodeSmall, "prep_16k": Prep,
              "verify_b32": VerifyB32,
-             "prefill_16k": lambda rank: Prefill(rank, "prefill_16k"),
-             "sliding_32k": lambda rank: Prefill(rank, "sliding_32k")}
+             "prefill_16k": lambda rank, product=True: Prefill(rank, "prefill_16k", product),
+             "sliding_32k": lambda rank, product=True: Prefill(rank, "sliding_32k", product)}
+SECONDARY = ("stack40", "verify_b32", "prefill_16k", "sliding_32k", "prep_16k", "decode_small")
 
 
 # ------------------------------------------------------------------ timing
@@ -720,7 +879,9 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
 
 
 KERNEL_SOURCES = {"decode_split": ("decode.cuh", "ptx.cuh", "kv_append.cuh"),
-                  "prefill_fwd": ("prefill.cuh", "ptx.cuh")}
+                  "prefill_fwd": ("prefill.cuh", "ptx.cuh"),
+                  "decode_block_split": ("decode_block.cuh", "decode.cuh", "ptx.cuh", "kv_append.cuh"),
+                  "qk_prep_append": ("qk_prep.cuh", "kv_append.cuh", "ptx.cuh")}
 
 
 def sources_digest(kernel: str) -> str:
@@ -766,38 +927,52 @@ def units(wl):
     return wl.bytes / 1e9 if wl.unit == "GB/s" else wl.flops / 1e12
 
 
-def run_ours(args, world, rank):
-    pk, pk_kind = peaks()
-    wl = WORKLOADS[args.workload](rank)
-    per_step, clocks = measure(wl, args.steps, args.warmup, world)
+def measure_line(wl, args, world, rank, steps, cpu_budget, pk, pk_kind):
+    """One workload's line: device-timed value and roofline, the clocks, the
+    end-to-end figure through the binding with host buffers, and (rank 0 of a
+    one-GPU run) the oracle on the host cores."""
+    per_step, clocks = measure(wl, steps, args.warmup, world)
     value = aggregate(units(wl), world, per_step)
     rf = roofline(wl, per_step, pk, pk_kind)
     rf["kernel"] = wl.kernel
-    if args.workload == "decode_b32":
-        rf["traffic"] = measured_traffic("decode_split", "decode_b32")
-        rf["traffic_unit"] = "bytes per launch (ncu dram read + write)"
-    elif wl.kernel == "prefill_fwd":
-        rf["traffic"] = measured_traffic("prefill_fwd", args.workload)
-        rf["traffic_unit"] = "bytes per launch (ncu dram read + write)"
-    res = {"metric": METRIC, "value": round(value, 2), "unit": wl.unit, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 4),
-           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-           "data": "synthetic (seeded N(0,1) bf16 inputs and caches)",
-           "config": {**wl.config(), "parallelism": f"dp{world} (independent batches, no collective)"},
-           "roofline": rf, "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks}
-    # end to end through the public API: pinned host inputs, copies in the timed region
+    key = getattr(wl, "traffic_key", None)
+    if key is not None:
+        rf["traffic"] = measured_traffic(*key)
+        rf["traffic_unit"] = "bytes per step (ncu dram read + write of the kernel's launches)"
+    res = {"value": round(value, 2), "unit": wl.unit, "ms_per_step": round(per_step * 1e3, 4),
+           "steps": steps, "roofline": rf, "gpu_launches": wl.launches_per_step * steps,
+           "clocks": clocks}
     if getattr(wl, "e2e_step", None) is not None:
         h2d, d2h = wl.e2e_buffers()
         for _ in range(args.warmup):
             wl.e2e_step()
         torch.cuda.synchronize()
-        t_e2e = max_over_ranks(time_steps(wl.e2e_step, args.steps, torch.cuda.current_stream(), world),
-                               world) / args.steps
+        t_e2e = max_over_ranks(time_steps(wl.e2e_step, steps, torch.cuda.current_stream(), world),
+                               world) / steps
         res["e2e"] = {"value": round(aggregate(units(wl), world, t_e2e), 2), "unit": wl.unit,
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                      "ms_per_step": round(t_e2e * 1e3, 4)}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and getattr(wl, "oracle_sample", None) is not None:
-        res["cpu_baseline"] = wl.oracle_sample(args.cpu_budget)
+                      "ms_per_step": round(t_e2e * 1e3, 4),
+                      "path": "pinned host inputs -> device, the library call, outputs -> pinned host"}
+    if rank == 0 and world == 1 and cpu_budget > 0 and getattr(wl, "oracle_sample", None) is not None:
+        res["cpu_baseline"] = wl.oracle_sample(cpu_budget)
+    return res
+
+
+def run_ours(args, world, rank):
+    pk, pk_kind = peaks()
+    wl = WORKLOADS[args.workload](rank)
+    budget = 0.0 if args.no_cpu_baseline else args.cpu_budget
+    line = measure_line(wl, args, world, rank, args.steps, budget, pk, pk_kind)
+    res = {"metric": METRIC, "value": line["value"], "unit": wl.unit, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": line["ms_per_step"],
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded N(0,1) bf16 inputs and caches)",
+           "config": {**wl.config(), "parallelism": f"dp{world} (independent batches, no collective)"},
+           "roofline": line["roofline"], "gpu_launches": line["gpu_launches"], "clocks": line["clocks"]}
+    for k in ("e2e", "cpu_baseline"):
+        if k in line:
+            res[k] = line[k]
+    if "cpu_baseline" in res:
         # the same oracle on one host thread, on a shorter bounded sample
         import oracle
         n_threads = oracle.num_threads()
@@ -813,20 +988,17 @@ def run_ours(args, world, rank):
         del wl
         torch.cuda.empty_cache()
         sec = {}
-        for name in ("stack40", "verify_b32", "prefill_16k", "sliding_32k", "prep_16k", "decode_small"):
+        for name in SECONDARY:
             w2 = WORKLOADS[name](rank)
             st = max(3, min(args.steps, 10))
-            ps, ck = measure(w2, st, args.warmup, world)
-            if w2.unit == "us/step":
-                sec[name] = {"value": round(ps * 1e6, 2), "unit": "us/step", "higher_is_better": False,
-                             "steps": st, "kernel": w2.kernel,
-                             "gpu_launches": w2.launches_per_step * st, "clocks": ck}
+            if hasattr(w2, "measure_line"):
+                sec[name] = w2.measure_line(st, args.warmup)
             else:
-                r2 = roofline(w2, ps, pk, pk_kind)
-                sec[name] = {"value": round(aggregate(units(w2), world, ps), 2), "unit": w2.unit,
-                             "ms_per_step": round(ps * 1e3, 4), "steps": st, "frac": r2["frac"],
-                             "bound": r2["bound"], "kernel": w2.kernel,
-                             "gpu_launches": w2.launches_per_step * st, "clocks": ck}
+                line = measure_line(w2, args, world, rank, st, budget / 2, pk, pk_kind)
+                line["frac"] = line["roofline"]["frac"]
+                line["bound"] = line["roofline"]["bound"]
+                line["kernel"] = w2.kernel
+                sec[name] = line
             del w2
             torch.cuda.empty_cache()
         res["secondary"] = sec
@@ -834,10 +1006,15 @@ def run_ours(args, world, rank):
 
 
 def run_reference(args, world, rank):
+    """The float64 CPU oracle on this host's cores, on bounded samples of the
+    workload; its inputs are built with torch alone (the library is not loaded)."""
     if rank != 0:
         return None
+    if args.workload in ("verify_b32", "prep_16k"):
+        return {"impl": "reference", "unavailable": f"no CPU oracle leg for {args.workload}; the "
+                                                    "reference arm covers the workloads of the main line"}
     import oracle
-    wl = WORKLOADS[args.workload](0)
+    wl = WORKLOADS[args.workload](0, product=False)
     vals = []
     samples = []
     per = max(1.0, args.cpu_budget / max(1, args.steps + args.warmup))
@@ -847,14 +1024,14 @@ def run_reference(args, world, rank):
             vals.append(r["value"])
             samples.append(r["sample"])
     v = statistics.median(vals)
-    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": wl.unit,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1) bf16 caches and queries)",
             "config": {**wl.config(), "parallelism": "CPU oracle, rank 0 only"},
-            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "cpu_baseline": {"value": round(v, 4), "unit": wl.unit, "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": samples[0]},
-            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": round(v, 4), "unit": wl.unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 

@@ -136,8 +136,11 @@ typedef struct {
  * sequential rule gives, and only tokens that would still be in the ring
  * after all n_new appends are written (the result equals n_new one-token
  * appends).  Afterwards seq_len[b] += n_new and ring_head advances.
- * p >= capacity on a full head sets DUO_ERR_CAPACITY on the device and skips
- * that write.  Defined by the DuoAttention card, section Summary (sink and
+ * On a layer with full heads, an append that would take seq_len[b] past
+ * capacity stops there: the positions below capacity are appended, the rest
+ * are dropped for every head, seq_len[b] becomes capacity, and
+ * DUO_ERR_CAPACITY is set on the device (duo_get_device_status).
+ * Defined by the DuoAttention card, section Summary (sink and
  * recent sizes) and section Why It Works (what each head keeps). */
 DUO_API int duo_kv_append(const duo_params *params, const duo_cache *cache, const void *k,
                   const void *v, int32_t n_new, void *stream);
@@ -273,7 +276,9 @@ DUO_API int duo_attn_decode_block(const duo_params *params, const duo_cache *cac
  * The split partials live in a 16 MiB array inside the library, reserved on
  * every GPU that loads it until the process exits; the call allocates
  * nothing.  The first call on a device looks up that array's address, so make
- * it before any stream capture begins.  A layer whose
+ * it before any stream capture begins; the address is cached per device and
+ * does not survive cudaDeviceReset (do not call this after resetting a device
+ * in the same process).  A layer whose
  * duo_decode_workspace_bytes exceeds 16 MiB returns DUO_ERR_WORKSPACE with
  * nothing launched.  All calls on a device share the array: calls whose
  * kernels may overlap on the GPU (different streams or threads) race, so

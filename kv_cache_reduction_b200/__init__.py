@@ -42,7 +42,10 @@ EXPORTED = ("duo_kv_append", "duo_kv_append_prep", "duo_prefill_workspace_bytes"
             "duo_decode_workspace_bytes", "duo_attn_decode", "duo_decode_block_workspace_bytes",
             "duo_attn_decode_block",
             "duo_attn_decode_static", "duo_cache_bytes", "duo_get_device_status",
-            "duo_status_string", "duo_last_error")
+            "duo_status_string", "duo_last_error", "duo_testing_withhold_tile")
+
+# kernels the failure-injection hook (include/duo_attn_testing.h) can select
+DUO_TESTING_DECODE, DUO_TESTING_PREFILL, DUO_TESTING_DECODE_BLOCK = 1, 2, 3
 
 
 class DuoLibraryMissing(RuntimeError):
@@ -171,6 +174,8 @@ def load_library(path: str = LIBRARY_PATH) -> ctypes.CDLL:
     lib.duo_status_string.restype = ctypes.c_char_p
     lib.duo_last_error.argtypes = []
     lib.duo_last_error.restype = ctypes.c_char_p
+    lib.duo_testing_withhold_tile.argtypes = [ctypes.c_int32, ctypes.c_int32]
+    lib.duo_testing_withhold_tile.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -458,6 +463,14 @@ def duo_status_string(code: int) -> str:
 
 def duo_last_error() -> str:
     return (load_library().duo_last_error() or b"").decode()
+
+
+def duo_testing_withhold_tile(kernel: int, tile: int) -> None:
+    """Failure injection for tests (include/duo_attn_testing.h): CTA 0's tile
+    producer of the selected kernel stops before its tile-th tile, so the
+    kernel's bounded waits expire and the call's status reads DUO_ERR_TIMEOUT.
+    tile = -1 turns it off."""
+    _check(load_library().duo_testing_withhold_tile(int(kernel), int(tile)))
 
 
 def workspace_for(params: DuoParams, max_seq_len: int, device="cuda") -> torch.Tensor:

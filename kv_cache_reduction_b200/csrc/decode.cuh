@@ -64,7 +64,7 @@ struct DecodeArgs {
     float scale_log2;               // softmax_scale * log2(e)
     const __nv_bfloat16 *gate;      // output gate pre-activations or null
     int32_t gate_mode;              // 0 none, 1 per (head, channel) [B][Hq][D], 2 per head [B][Hq]
-    int32_t withhold_tile;          // test hook: CTA 0 issues no load from this tile on (-1: off)
+    int32_t withhold_tile;          // failure-injection hook: CTA 0 issues no load from this tile on (-1: off)
     int8_t full_head[64];           // full rank -> KV head
     int8_t ring_head_of[64];        // ring rank -> KV head
     HeadTable heads;
@@ -92,7 +92,8 @@ __device__ __forceinline__ Item item_of(const DecodeArgs &a, int w) {
         it.g = a.full_head[r];
         it.ring = false;
         it.row0 = (int32_t)(((int64_t)it.b * a.n_full + r) * a.capacity);
-        const int32_t n = a.seq_len[it.b];
+        // a full head's rows end at the capacity, whatever seq_len says
+        const int32_t n = (int32_t)min((int64_t)a.seq_len[it.b], a.capacity);
         it.e_begin = it.split * a.chunk_full;
         it.e_end = min(n, it.e_begin + a.chunk_full);
         it.n_sink = 0;

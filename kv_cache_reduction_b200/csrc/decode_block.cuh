@@ -304,6 +304,9 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 for (int t = 0; t < it.n_tiles; ++t, ++jg) {
                     const int st = jg % ST;
                     if (jg >= ST && !(ok = mbar_wait(&kv_empty[st], ((jg / ST) - 1) & 1))) break;
+                    // failure-detection test: stop feeding this CTA so that its
+                    // consumers' bounded waits expire (nothing stays in flight)
+                    if (blockIdx.x == 0 && jg == d.withhold_tile) { ok = false; break; }
                     char *ks = sKV + st * kDecStageBytes;
                     mbar_expect_tx(&kv_full[st], kDecStageBytes);
                     if (t == bi.cache_tiles) {

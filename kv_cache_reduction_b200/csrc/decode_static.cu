@@ -19,6 +19,8 @@
 // separate workspaces.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "duo_attn.h"
 
 // 16 MiB of split partials: enough for B=32 at context 32768 or B=16 at
@@ -31,7 +33,11 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBy
 namespace {
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices] = {};
+// Per-device address of the array.  Host threads may make their first call
+// at the same time: both look the address up and store the same value, so
+// relaxed atomics are enough.  A cached address does not survive
+// cudaDeviceReset (the device's module, and the array with it, is reloaded).
+std::atomic<void *> g_scratch_addr[kMaxDevices] = {};
 
 // In host code the array's name is only a stand-in, not a device address.
 // The device address is looked up once per device, with that device
@@ -40,13 +46,13 @@ void *g_scratch_addr[kMaxDevices] = {};
 int scratch_for_current_device(void **addr) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DUO_ERR_CUDA;
-    if (g_scratch_addr[dev] == nullptr) {
-        void *p = nullptr;
+    void *p = g_scratch_addr[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
         const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
         if (e != cudaSuccess || p == nullptr) return DUO_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+        g_scratch_addr[dev].store(p, std::memory_order_relaxed);
     }
-    *addr = g_scratch_addr[dev];
+    *addr = p;
     return DUO_OK;
 }
 

@@ -5,10 +5,10 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
-#include <cstdlib>
 #include <cstring>
 
 #include "duo_attn.h"
+#include "duo_attn_testing.h"
 #include "decode.cuh"
 #include "decode_block.cuh"
 #include "kv_append.cuh"
@@ -45,6 +45,12 @@ int check_gate(const duo_gate *g, int *mode, const void **values) {
     *values = g->values;
     return DUO_OK;
 }
+
+// The failure-injection setting of each kernel (duo_attn_testing.h): the
+// tile from which CTA 0's producer stops, or -1.
+std::atomic<int> g_withhold[4] = {{-1}, {-1}, {-1}, {-1}};
+
+int withhold_tile(int kernel) { return g_withhold[kernel].load(std::memory_order_relaxed); }
 
 constexpr int kMaxHkv = 64;
 constexpr int kMaxWindow = 8192;
@@ -359,7 +365,7 @@ int duo_kv_append(const duo_params *params, const duo_cache *cache, const void *
     duo::kv_append_scatter<<<(unsigned)blocks, 256, 0, st>>>(a);
     if ((rc = launch_status("kv_append_scatter"))) return rc;
     duo::kv_append_commit<<<(params->batch + 127) / 128, 128, 0, st>>>(
-        cache->seq_len, cache->ring_head, params->batch, n_new, L.sink, L.ring);
+        cache->seq_len, cache->ring_head, params->batch, n_new, L.sink, L.ring, L.n_full, a.capacity);
     return launch_status("kv_append_commit");
 }
 
@@ -413,7 +419,7 @@ int duo_kv_append_prep(const duo_params *params, const duo_cache *cache, const d
     duo::qk_prep_append<<<(unsigned)blocks, duo::kPrepThreads, 0, st>>>(a);
     if ((rc = launch_status("qk_prep_append"))) return rc;
     duo::kv_append_commit<<<(params->batch + 127) / 128, 128, 0, st>>>(
-        cache->seq_len, cache->ring_head, params->batch, n_new, L.sink, L.ring);
+        cache->seq_len, cache->ring_head, params->batch, n_new, L.sink, L.ring, L.n_full, a.app.capacity);
     return launch_status("kv_append_commit");
 }
 
@@ -487,11 +493,7 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     a.scale_log2 = params->softmax_scale * duo::kLog2eF;
     a.gate = (const __nv_bfloat16 *)gate_values;
     a.gate_mode = gate_mode;
-    // Test hook for the failure-detection path: DUO_TEST_WITHHOLD_TILE=t makes
-    // the first CTA's producer stop before tile t; its consumers then time out
-    // and the call reports DUO_ERR_TIMEOUT through duo_get_device_status().
-    const char *withhold = getenv("DUO_TEST_WITHHOLD_TILE");
-    a.withhold_tile = withhold ? atoi(withhold) : -1;
+    a.withhold_tile = withhold_tile(DUO_TESTING_DECODE);
     memcpy(a.full_head, L.full_head, sizeof a.full_head);
     memcpy(a.ring_head_of, L.ring_head_of, sizeof a.ring_head_of);
     a.heads = L.heads;
@@ -540,8 +542,8 @@ int duo_attn_prefill(const duo_params *params, const void *q, const void *k, con
         return fail(DUO_ERR_INVALID_ARG, "q / k / v / out / lse must be 16-byte aligned");
     if ((rc = check_device(nullptr))) return rc;
     return duo::launch_prefill(params, L.sliding, L.heads.is_full, L.sink, L.ring, q, k, v, seq_len,
-                               out, lse, (int32_t *)workspace, gate_mode, gate_values, (cudaStream_t)stream,
-                               g_err, sizeof g_err);
+                               out, lse, (int32_t *)workspace, gate_mode, gate_values,
+                               withhold_tile(DUO_TESTING_PREFILL), (cudaStream_t)stream, g_err, sizeof g_err);
 }
 
 int duo_cache_bytes(const duo_params *params, int64_t capacity, int64_t seq_len,
@@ -645,7 +647,7 @@ int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, cons
     da.scale_log2 = params->softmax_scale * duo::kLog2eF;
     da.gate = (const __nv_bfloat16 *)gate_values;
     da.gate_mode = gate_mode;
-    da.withhold_tile = -1;
+    da.withhold_tile = withhold_tile(DUO_TESTING_DECODE_BLOCK);
     memcpy(da.full_head, L.full_head, sizeof da.full_head);
     memcpy(da.ring_head_of, L.ring_head_of, sizeof da.ring_head_of);
     da.heads = L.heads;
@@ -673,6 +675,13 @@ int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, cons
         case 7: return launch_block<7>(a, grid, st, merge_blocks);
         default: return launch_block<8>(a, grid, st, merge_blocks);
     }
+}
+
+int duo_testing_withhold_tile(int32_t kernel, int32_t tile) {
+    if (kernel < DUO_TESTING_DECODE || kernel > DUO_TESTING_DECODE_BLOCK || tile < -1)
+        return fail(DUO_ERR_INVALID_ARG, "unknown kernel %d or tile %d", (int)kernel, (int)tile);
+    g_withhold[kernel].store(tile, std::memory_order_relaxed);
+    return DUO_OK;
 }
 
 int duo_get_device_status(void *stream) {

@@ -34,6 +34,41 @@ struct AppendArgs {
 
 constexpr int kVecPerRow = 128 * 2 / 16;   // 16 x 16-byte vectors per head row
 
+// Where the append of a sequence that holds n_old tokens ends: n_old + n_new,
+// or the full cache's capacity when the layer has full heads and the append
+// would pass it.  The tokens from there on are dropped for every head (the
+// scatter records DUO_ERR_CAPACITY), so that seq_len never exceeds the
+// capacity and a later decode never reads past a full head's rows.
+__device__ __forceinline__ int64_t append_end(int64_t n_old, int32_t n_new, int32_t n_full, int64_t capacity) {
+    const int64_t n_end = n_old + n_new;
+    if (n_full == 0 || n_end <= capacity) return n_end;
+    return n_old > capacity ? n_old : capacity;
+}
+
+// Cache row that token t of sequence b writes for KV head g (*full tells
+// which cache), or -1 when it writes none: a ring position that a later token
+// of the same append overwrites, or a token past the capacity (status set).
+__device__ __forceinline__ int64_t append_row(const AppendArgs &a, int b, int g, int64_t t, bool *full) {
+    const int64_t n_old = a.seq_len[b];
+    const int64_t pos = n_old + t;
+    const int64_t n_end = append_end(n_old, a.n_new, a.n_full, a.capacity);
+    *full = a.heads.is_full[g] != 0;
+    if (pos >= n_end) {
+        record_status(-6 /* DUO_ERR_CAPACITY */);
+        return -1;
+    }
+    if (*full) return ((int64_t)b * a.n_full + a.heads.rank[g]) * a.capacity + pos;
+    int64_t slot;
+    if (pos < a.sink) {
+        slot = pos;
+    } else {
+        if (pos < n_end - a.ring) return -1;               // overwritten later in this append
+        const int64_t first = n_old > a.sink ? n_old : a.sink;   // first ring position written
+        slot = a.sink + ((int64_t)a.ring_head[b] + (pos - first)) % a.ring;
+    }
+    return ((int64_t)b * a.n_ring + a.heads.rank[g]) * a.slots + slot;
+}
+
 // One thread copies one 16-byte vector of K and of V.  Rows are
 // (b, t, g) triples in input order, so reads are fully coalesced.
 __global__ void __launch_bounds__(256) kv_append_scatter(AppendArgs a) {
@@ -45,42 +80,23 @@ __global__ void __launch_bounds__(256) kv_append_scatter(AppendArgs a) {
     const int g = (int)(row % a.hkv);
     const int64_t t = (row / a.hkv) % a.n_new;
     const int b = (int)(row / a.hkv / a.n_new);
-    const int64_t n_old = a.seq_len[b];
-    const int64_t pos = n_old + t;
-    uint4 *dk, *dv;
-    if (a.heads.is_full[g]) {
-        if (pos >= a.capacity) {
-            record_status(-6 /* DUO_ERR_CAPACITY */);
-            return;
-        }
-        const int64_t r = ((int64_t)b * a.n_full + a.heads.rank[g]) * a.capacity + pos;
-        dk = a.full_k + r * kVecPerRow;
-        dv = a.full_v + r * kVecPerRow;
-    } else {
-        int64_t slot;
-        if (pos < a.sink) {
-            slot = pos;
-        } else {
-            const int64_t n_end = n_old + a.n_new;
-            if (pos < n_end - a.ring) return;          // overwritten later in this append
-            const int64_t first = n_old > a.sink ? n_old : a.sink;   // first ring position written
-            slot = a.sink + ((int64_t)a.ring_head[b] + (pos - first)) % a.ring;
-        }
-        const int64_t r = ((int64_t)b * a.n_ring + a.heads.rank[g]) * a.slots + slot;
-        dk = a.strm_k + r * kVecPerRow;
-        dv = a.strm_v + r * kVecPerRow;
-    }
+    bool full = false;
+    const int64_t r = append_row(a, b, g, t, &full);
+    if (r < 0) return;
+    uint4 *dk = (full ? a.full_k : a.strm_k) + r * kVecPerRow;
+    uint4 *dv = (full ? a.full_v : a.strm_v) + r * kVecPerRow;
     dk[vec] = a.k[idx];
     dv[vec] = a.v[idx];
 }
 
-// Moves seq_len and ring_head forward once the scatter has read them.
-__global__ void kv_append_commit(int32_t *seq_len, int32_t *ring_head, int32_t batch,
-                                 int32_t n_new, int32_t sink, int32_t ring) {
+// Moves seq_len and ring_head forward once the scatter has read them (to the
+// append's end, which stops at the capacity as append_end says).
+__global__ void kv_append_commit(int32_t *seq_len, int32_t *ring_head, int32_t batch, int32_t n_new,
+                                 int32_t sink, int32_t ring, int32_t n_full, int64_t capacity) {
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= batch) return;
     const int64_t n_old = seq_len[b];
-    const int64_t n_end = n_old + n_new;
+    const int64_t n_end = append_end(n_old, n_new, n_full, capacity);
     const int64_t first = n_old > sink ? n_old : sink;
     const int64_t ring_writes = n_end > first ? n_end - first : 0;
     ring_head[b] = (int32_t)(((int64_t)ring_head[b] + ring_writes) % ring);

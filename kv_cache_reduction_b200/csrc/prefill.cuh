@@ -73,6 +73,7 @@ struct PrefillArgs {
     // gate layout: kGate 1 [B][L][Hq][128], kGate 2 [B][L][Hq]
     int32_t L, hq, hkv, n_qtiles, n_work, batch_pairs;
     int32_t sink, recent, window;
+    int32_t withhold_tile; // failure-injection hook: CTA 0 issues no K/V load from this tile on (-1: off)
     float scale_log2;
     int8_t kind[64];       // per KV head
 };
@@ -224,6 +225,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 for (int j = 0; j < n_kv; ++j, ++jg) {
                     const int st = jg % kPfStages;
                     if (jg >= kPfStages && !(ok = mbar_wait(&kv_empty[st], ((jg / kPfStages) - 1) & 1))) break;
+                    // failure-detection test: stop feeding this CTA so that its
+                    // consumers' bounded waits expire (nothing stays in flight)
+                    if (blockIdx.x == 0 && jg == a.withhold_tile) { ok = false; break; }
                     const int row = tl.at(j) * kPfN;
                     char *kst = sKV + st * kPfStageBytes;
                     mbar_expect_tx(&kv_full[st], kPfStageBytes);
@@ -428,12 +432,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                         const int cc = ch * 32 + e;
                         const f2 a01 = f2_fma(f2_make(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), c2, ms2);
                         const f2 a23 = f2_fma(f2_make(__uint_as_float(sr[cc + 2]), __uint_as_float(sr[cc + 3])), c2, ms2);
-                        const float p0 = ex2_approx(a01.x), p1 = ex2_approx(a01.y);
-                        const float p2 = ex2_approx(a23.x), p3 = ex2_approx(a23.y);
-                        ls01 = f2_add(ls01, f2_make(p0, p1));
-                        ls23 = f2_add(ls23, f2_make(p2, p3));
-                        pw[e / 2] = pack_bf16x2(p0, p1);
-                        pw[e / 2 + 1] = pack_bf16x2(p2, p3);
+                        const uint32_t w01 = pack_bf16x2(ex2_approx(a01.x), ex2_approx(a01.y));
+                        const uint32_t w23 = pack_bf16x2(ex2_approx(a23.x), ex2_approx(a23.y));
+                        // the row sum adds the bf16 weights the PV product uses, so
+                        // that numerator and denominator agree
+                        ls01 = f2_add(ls01, f2_make(bf16lo(w01), bf16hi(w01)));
+                        ls23 = f2_add(ls23, f2_make(bf16lo(w23), bf16hi(w23)));
+                        pw[e / 2] = w01;
+                        pw[e / 2 + 1] = w23;
                     }
                     // P of keys [64*half + 32*ch, +32) -> TMEM columns [32*half + 16*ch, +16)
                     tmem_st16(s_tmem + half * 32 + ch * 16, pw);
@@ -602,7 +608,7 @@ inline bool make_tmap(CUtensorMap *m, const void *base, int B, int L, int H, int
 inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_full, int sink,
                           int ring, const void *q, const void *k, const void *v, int32_t L, void *out,
                           float *lse, int32_t *work_counter, int gate_mode, const void *gate,
-                          cudaStream_t stream, char *err, size_t err_len) {
+                          int withhold_tile, cudaStream_t stream, char *err, size_t err_len) {
     PrefillArgs a;
     memset(&a, 0, sizeof a);
     const int B = p->batch;
@@ -624,6 +630,7 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     a.recent = sliding ? 0 : ring;
     a.window = sliding ? ring : 0;
     a.scale_log2 = p->softmax_scale * kLog2eF;
+    a.withhold_tile = withhold_tile;
     for (int g = 0; g < p->num_kv_heads; ++g)
         a.kind[g] = sliding ? kKindSliding : (is_full[g] ? kKindFull : kKindStreaming);
     void (*kernel)(PrefillArgs) = gate_mode == 1 ? prefill_fwd<1> : gate_mode == 2 ? prefill_fwd<2> : prefill_fwd<0>;

@@ -27,32 +27,6 @@ struct PrepArgs {
     int32_t hq;
 };
 
-// Cache row (in 16-byte vectors) that token t of sequence b writes for KV head
-// g, or -1 when the token is not kept (a ring position overwritten later in
-// the same append) or a full head is out of capacity (status set).
-__device__ __forceinline__ int64_t prep_cache_row(const AppendArgs &a, int b, int g, int64_t t,
-                                                  bool *full) {
-    const int64_t n_old = a.seq_len[b];
-    const int64_t pos = n_old + t;
-    *full = a.heads.is_full[g] != 0;
-    if (*full) {
-        if (pos >= a.capacity) {
-            record_status(-6 /* DUO_ERR_CAPACITY */);
-            return -1;
-        }
-        return ((int64_t)b * a.n_full + a.heads.rank[g]) * a.capacity + pos;
-    }
-    int64_t slot;
-    if (pos < a.sink) {
-        slot = pos;
-    } else {
-        if (pos < n_old + a.n_new - a.ring) return -1;
-        const int64_t first = n_old > a.sink ? n_old : a.sink;
-        slot = a.sink + ((int64_t)a.ring_head[b] + (pos - first)) % a.ring;
-    }
-    return ((int64_t)b * a.n_ring + a.heads.rank[g]) * a.slots + slot;
-}
-
 __device__ __forceinline__ void unpack8(const uint4 u, float *x) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -164,7 +138,7 @@ __global__ void __launch_bounds__(kPrepThreads) qk_prep_append(const __grid_cons
             if (!is_q) {
                 const int g = r - a.hq;
                 bool full = false;
-                const int64_t row = prep_cache_row(ap, b, g, t, &full);
+                const int64_t row = append_row(ap, b, g, t, &full);
                 if (row >= 0) {
                     const uint4 vv = ap.v[(tok_row * ap.hkv + g) * kVecPerRow + j];
                     if (full) {

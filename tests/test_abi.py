@@ -62,6 +62,20 @@ def test_status_strings(lib):
     assert duo.duo_status_string(-99) == "unknown status"
 
 
+def test_testing_hook_checks_its_arguments(lib):
+    """The failure-injection hook (include/duo_attn_testing.h) takes the three
+    pipelined kernels and a tile >= -1, and is off again after tile -1."""
+    for kernel in (0, 4, -1):
+        with pytest.raises(duo.DuoError) as e:
+            duo.duo_testing_withhold_tile(kernel, 0)
+        assert e.value.code == duo.DUO_ERR_INVALID_ARG
+    with pytest.raises(duo.DuoError):
+        duo.duo_testing_withhold_tile(duo.DUO_TESTING_PREFILL, -2)
+    for kernel in (duo.DUO_TESTING_DECODE, duo.DUO_TESTING_PREFILL, duo.DUO_TESTING_DECODE_BLOCK):
+        duo.duo_testing_withhold_tile(kernel, 3)
+        duo.duo_testing_withhold_tile(kernel, -1)
+
+
 def _params(**kw):
     base = dict(batch=2, full_mask=(1, 0, 0, 1, 0, 0, 0, 0))
     base.update(kw)

@@ -151,8 +151,8 @@ def test_timed_sample_cycles_until_the_budget():
 def test_decode_cpu_baseline_leg_runs_on_host_tensors():
     """The bench's CPU-baseline leg of the main line, driven on small host
     tensors (the leg reads the caches back to the host, so it needs no GPU):
-    it cycles the oracle over whole (sequence, KV head) groups until its
-    budget and reports bytes per second."""
+    it runs the oracle over whole decode steps (every row of the batch per
+    call) until its budget and reports bytes per second."""
     import types
     import torch
     import kv_cache_reduction_b200 as duo
@@ -169,6 +169,7 @@ def test_decode_cpu_baseline_leg_runs_on_host_tensors():
     wl.q = inputs.randn_bf16((2, 48, 128), 60, "cpu")
     r = wl.oracle_sample(0.3)
     assert r["kind"] == "oracle" and r["unit"] == "GB/s" and r["value"] > 0
-    assert "passes over the 16" in r["sample"]
+    assert "whole decode steps (96 rows per call" in r["sample"]
     used = int(r["sample"].split()[0])
     assert used >= 1
+    assert r["threads_busy"] == min(r["cores"], 2 * 2 * 6)

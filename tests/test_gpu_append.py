@@ -8,7 +8,7 @@ import oracle
 import kv_cache_reduction_b200 as duo
 from kv_cache_reduction_b200 import inputs
 
-from gpu_helpers import host_cache, layers, random_cache
+from gpu_helpers import assert_close, host_cache, layers, random_cache
 
 pytestmark = pytest.mark.gpu
 
@@ -59,18 +59,40 @@ def test_append_small_ring_and_no_sink(cuda_device):
     run_and_compare(p, o, cache, [1, 2, 7, 1, 4], seed=400)
 
 
-def test_append_capacity_overflow_sets_status(cuda_device):
-    p, o = layers(1, full_mask=(1,) + (0,) * 7)
-    cache = random_cache(p, 8, [6], [0], seed=11)
-    before = inputs.bits(cache.full_k).copy()
+def test_append_capacity_overflow_stops_at_capacity(cuda_device):
+    """An append that would take a sequence past the full cache's capacity
+    appends the positions below it, drops the rest for every head (ring heads
+    included), leaves seq_len at the capacity and sets DUO_ERR_CAPACITY, as
+    the oracle's token-by-token append does when it stops at the capacity.
+    A decode afterwards reads only the rows below the capacity."""
+    p, o = layers(1, full_mask=(1,) + (0,) * 7, sink=2, recent=3)
+    cache = random_cache(p, 8, [6], [1], seed=11)
+    ref = host_cache(o, cache)
     k = inputs.randn_bf16((1, 4, 8, 128), 500, "cuda")
-    duo.duo_kv_append(p, cache, k, k)
+    v = inputs.randn_bf16((1, 4, 8, 128), 501, "cuda")
+    duo.duo_kv_append(p, cache, k, v)
     assert duo.duo_get_device_status() == duo.DUO_ERR_CAPACITY
     assert duo.duo_get_device_status() == duo.DUO_OK       # reading clears it
-    after = inputs.bits(cache.full_k)
-    # rows 6, 7 written, nothing past the capacity
-    assert np.array_equal(after[0, 0, :6], before[0, 0, :6])
-    assert np.array_equal(after[0, 0, 6:8], inputs.bits(k)[0, :2, 0])
+    with pytest.raises(ValueError):                        # the oracle stops at the capacity too
+        oracle.kv_append(o, ref, inputs.bits(k), inputs.bits(v))
+    got = host_cache(o, cache)
+    for name in ("full_k", "full_v", "strm_k", "strm_v", "seq_len", "ring_head"):
+        assert np.array_equal(getattr(got, name), getattr(ref, name)), name
+    assert int(cache.seq_len[0]) == 8
+    # a full cache takes nothing more
+    duo.duo_kv_append(p, cache, k[:, :1].contiguous(), v[:, :1].contiguous())
+    assert duo.duo_get_device_status() == duo.DUO_ERR_CAPACITY
+    again = host_cache(o, cache)
+    for name in ("full_k", "full_v", "strm_k", "strm_v", "seq_len", "ring_head"):
+        assert np.array_equal(getattr(again, name), getattr(ref, name)), name
+    q = inputs.randn_bf16((1, 48, 128), 502, "cuda")
+    out = torch.full((1, 48, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((1, 48), float("nan"), dtype=torch.float32, device="cuda")
+    duo.duo_attn_decode(p, cache, q, 8, out, lse, duo.workspace_for(p, 8))
+    torch.cuda.synchronize()
+    assert duo.duo_get_device_status() == duo.DUO_OK
+    ro, rl = oracle.attn_decode(o, ref, inputs.bits(q))
+    assert_close(out, ro.reshape(1, 48, 128), lse, rl.reshape(1, 48), "decode at capacity")
 
 
 def test_append_prefill_16k_workload(cuda_device):

@@ -6,14 +6,11 @@ accepts (sink + recent = 8192, window = 8192).  For each: the append (caches
 byte for byte), the one-token decode after it, the prefill, and the verify
 block.  Tolerances as the other parity tests.
 
-Two prefill cases are known to miss the max-abs bar: rows that attend one or two
-keys (window 1 with a sink logit; sink 1 + recent 1) have |O| close to |v|, up
-to about 5, and two bf16 roundings stack there: P's (the kernel rounds P to
-bf16 for the PV product but sums the unrounded P into the row sum, so a
-weight is off by up to 2^-9 of |v|) and the output's own (half an ulp, 0.0156
-at that magnitude).  Measured max-abs 2.07e-2 (window 1) and 2.51e-2 (sink 1 +
-recent 1); the decode (fp32 P) and the same sizes' decode and block paths
-pass."""
+Rows that attend one or two keys (window 1 with a sink logit; sink 1 +
+recent 1) have |O| close to |v|, up to about 5, where the output's own bf16
+rounding is already half an ulp (0.0156); the prefill adds the same
+bf16-rounded probabilities to the row sum that the PV product uses, so that
+no second rounding error stacks on top.  They are held to the same bar."""
 import numpy as np
 import pytest
 import torch
@@ -75,15 +72,7 @@ def test_append_then_decode(cuda_device, sink, recent, window):
         assert_close(out, ro.reshape(B, 48, 128), lse, rl.reshape(B, 48), f"decode n={n_now}")
 
 
-_PREFILL_KNOWN = pytest.mark.xfail(
-    reason="rows of one or two keys: bf16 P rounding (unrounded P in the row sum) plus bf16 "
-           "output rounding at |O| ~ 5 exceed max-abs 2e-2 (measured 2.07e-2 and 2.51e-2)",
-    strict=False)
-PREFILL_SIZES = [pytest.param(*s, id=i, marks=_PREFILL_KNOWN) if i in ("sink1-recent1", "window1")
-                 else pytest.param(*s, id=i) for s, i in zip(SIZES, IDS)]
-
-
-@pytest.mark.parametrize("sink,recent,window", PREFILL_SIZES)
+@pytest.mark.parametrize("sink,recent,window", SIZES, ids=IDS)
 def test_prefill(cuda_device, sink, recent, window):
     B, L = 1, 600                                     # five tiles, the last one ragged
     p, o = _layer(B, sink, recent, window)

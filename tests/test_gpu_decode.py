@@ -128,14 +128,26 @@ def test_decode_reads_exactly_the_valid_slots(cuda_device):
 
 
 def test_decode_small_workload_end_to_end(cuda_device):
-    """1024-token prompt appended, then 16 steps of append-one + decode,
-    full heads {0,3,5,6}, every step against the oracle."""
+    """The single-layer workload end to end: the 1024-token prompt is
+    prefilled (every one of the 48 x 1024 rows against the oracle) and
+    appended, then 16 steps of append-one + decode, full heads {0,3,5,6},
+    every step against the oracle."""
     w = inputs.workload("decode_small")
     p, o = layers(w.batch, full_mask=w.full_mask)
     cache = duo.DuoCache.allocate(p, w.seq_len + w.decode_steps)
     ref = host_cache(o, cache)
+    qp = inputs.randn_bf16((1, w.seq_len, 48, 128), w.seed + 2, "cuda")
     k = inputs.randn_bf16((1, w.seq_len, 8, 128), w.seed, "cuda")
     v = inputs.randn_bf16((1, w.seq_len, 8, 128), w.seed + 1, "cuda")
+    out_p = torch.full((1, w.seq_len, 48, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse_p = torch.full((1, 48, w.seq_len), float("nan"), dtype=torch.float32, device="cuda")
+    ws_p = torch.empty(duo.duo_prefill_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    duo.duo_attn_prefill(p, qp, k, v, out_p, lse_p, workspace=ws_p)
+    torch.cuda.synchronize()
+    assert duo.duo_get_device_status() == duo.DUO_OK
+    ref_o, ref_l = oracle.attn_prefill(o, inputs.bits(qp), inputs.bits(k), inputs.bits(v))
+    assert_close(out_p.permute(0, 2, 1, 3).reshape(-1, 128), ref_o, lse_p.reshape(-1), ref_l,
+                 "prefill of the 1024-token prompt")
     duo.duo_kv_append(p, cache, k, v)
     oracle.kv_append(o, ref, inputs.bits(k), inputs.bits(v))
     for step in range(w.decode_steps):

@@ -1,8 +1,10 @@
 """The 40-layer decode stack (DuoAttention layers 3, 7, ..., 39 with 2 of 8
 heads full; sliding-window layers of 512 with sink logits elsewhere).
 
-* full size (B=16, context 131072) for one layer of each kind, sampled
-  sequences against the oracle;
+* full size (B=16, context 131072) for two layers of each kind, six
+  sequences of each against the oracle: sliding layers 0 and 38 (38 with every
+  ring pointer one slot before the wrap) and DuoAttention layers 3 and 39,
+  each with its own seeded head mask;
 * the whole 40-layer step captured in one CUDA graph gives the same bytes as
   the same 40 calls made eagerly (smaller context)."""
 import numpy as np
@@ -27,13 +29,17 @@ def layer_of(w, li, batch):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("li", [0, 3])
+@pytest.mark.parametrize("li", [0, 3, 38, 39])
 def test_stack40_layer_full_size_sampled(cuda_device, li):
     w = inputs.workload("stack40")
     B, n = w.batch, w.seq_len
     p, o = layer_of(w, li, B)
     rng = np.random.default_rng(w.seed + li)
-    rh = rng.integers(0, p.ring_slots - p.sink if p.window == 0 else p.window, size=B).tolist()
+    ring = p.ring_slots - p.sink if p.window == 0 else p.window
+    if li == 38:
+        rh = [ring - 1] * B             # the next ring write wraps to slot 0
+    else:
+        rh = rng.integers(0, ring, size=B).tolist()
     cache = random_cache(p, n, [n] * B, rh, seed=w.seed * 100 + li)
     q = inputs.randn_bf16((B, 48, 128), w.seed * 100 + li + 50, "cuda")
     out = torch.empty((B, 48, 128), dtype=torch.bfloat16, device="cuda")
@@ -43,7 +49,7 @@ def test_stack40_layer_full_size_sampled(cuda_device, li):
     assert duo.duo_get_device_status() == duo.DUO_OK
     o1 = oracle.Layer(1, 48, 8, 128, o.sink, o.recent, o.window, o.softmax_scale, o.full_mask,
                       o.sink_logit)
-    for b in (0, 7, 15):
+    for b in (0, 3, 6, 9, 12, 15):
         hc = oracle.Cache(o1, n if o1.n_full else 1)
         if o1.n_full:
             hc.full_k = inputs.bits(cache.full_k[b:b + 1])
