@@ -989,17 +989,20 @@ def run_ours(args, world, rank):
         torch.cuda.empty_cache()
         sec = {}
         for name in SECONDARY:
-            w2 = WORKLOADS[name](rank)
             st = max(3, min(args.steps, 10))
-            if hasattr(w2, "measure_line"):
-                sec[name] = w2.measure_line(st, args.warmup)
-            else:
-                line = measure_line(w2, args, world, rank, st, budget / 2, pk, pk_kind)
-                line["frac"] = line["roofline"]["frac"]
-                line["bound"] = line["roofline"]["bound"]
-                line["kernel"] = w2.kernel
-                sec[name] = line
-            del w2
+            try:
+                w2 = WORKLOADS[name](rank)
+                if hasattr(w2, "measure_line"):
+                    sec[name] = w2.measure_line(st, args.warmup)
+                else:
+                    line = measure_line(w2, args, world, rank, st, budget / 2, pk, pk_kind)
+                    line["frac"] = line["roofline"]["frac"]
+                    line["bound"] = line["roofline"]["bound"]
+                    line["kernel"] = w2.kernel
+                    sec[name] = line
+            except Exception as e:              # a secondary line must not lose the main one
+                sec[name] = {"error": f"{type(e).__name__}: {e}"}
+            w2 = None
             torch.cuda.empty_cache()
         res["secondary"] = sec
     return res

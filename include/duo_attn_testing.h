@@ -36,6 +36,14 @@ extern "C" {
  * tile below -1. */
 DUO_API int duo_testing_withhold_tile(int32_t kernel, int32_t tile);
 
+/* The prefill's exponential on the FMA pipe (2^x by Cody-Waite range
+ * reduction and a degree-3 polynomial, see ex2_poly2 in the sources), applied
+ * to n fp32 values: y[i] = 2^x[i].  x, y: device fp32 [n], 16-byte aligned.
+ * Inputs below -125 give about 2^-125.  For tests of its error bound against
+ * the exact 2^x; asynchronous on `stream`.  DUO_ERR_INVALID_ARG for NULL or
+ * misaligned pointers or n < 0. */
+DUO_API int duo_testing_ex2(const float *x, float *y, int64_t n, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

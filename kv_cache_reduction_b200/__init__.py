@@ -42,7 +42,7 @@ EXPORTED = ("duo_kv_append", "duo_kv_append_prep", "duo_prefill_workspace_bytes"
             "duo_decode_workspace_bytes", "duo_attn_decode", "duo_decode_block_workspace_bytes",
             "duo_attn_decode_block",
             "duo_attn_decode_static", "duo_cache_bytes", "duo_get_device_status",
-            "duo_status_string", "duo_last_error", "duo_testing_withhold_tile")
+            "duo_status_string", "duo_last_error", "duo_testing_withhold_tile", "duo_testing_ex2")
 
 # kernels the failure-injection hook (include/duo_attn_testing.h) can select
 DUO_TESTING_DECODE, DUO_TESTING_PREFILL, DUO_TESTING_DECODE_BLOCK = 1, 2, 3
@@ -176,6 +176,8 @@ def load_library(path: str = LIBRARY_PATH) -> ctypes.CDLL:
     lib.duo_last_error.restype = ctypes.c_char_p
     lib.duo_testing_withhold_tile.argtypes = [ctypes.c_int32, ctypes.c_int32]
     lib.duo_testing_withhold_tile.restype = ctypes.c_int
+    lib.duo_testing_ex2.argtypes = [vp, vp, ctypes.c_int64, vp]
+    lib.duo_testing_ex2.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -471,6 +473,17 @@ def duo_testing_withhold_tile(kernel: int, tile: int) -> None:
     kernel's bounded waits expire and the call's status reads DUO_ERR_TIMEOUT.
     tile = -1 turns it off."""
     _check(load_library().duo_testing_withhold_tile(int(kernel), int(tile)))
+
+
+def duo_testing_ex2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x by the prefill's FMA-pipe exponential (include/duo_attn_testing.h),
+    for tests of its error bound: x a contiguous fp32 CUDA tensor."""
+    if x.dtype != torch.float32:
+        raise ValueError("x must be float32")
+    _on_device(x, "x")
+    y = torch.empty_like(x)
+    _check(load_library().duo_testing_ex2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)))
+    return y
 
 
 def workspace_for(params: DuoParams, max_seq_len: int, device="cuda") -> torch.Tensor:

@@ -146,20 +146,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int c0,
         ::"r"(smem_u32(dst)), "l"(tmap), "r"(c0), "r"(c1), "r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                   "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
-                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
-                   "r"(r[6]), "r"(r[7])
-                 : "memory");
-}
-
 __device__ __forceinline__ void reg_fence8(uint32_t (&r)[8]) {
     asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
                  "+r"(r[6]), "+r"(r[7]));
@@ -217,6 +203,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    // launched as a programmatic dependent: the set-up above overlapped the
+    // previous kernel (an append, or the last call's merge, which reads the
+    // workspace this kernel writes); nothing global is touched before this
+    pdl_wait();
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer
@@ -383,7 +373,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
                 float p[kGroup];
 #pragma unroll
                 for (int h = 0; h < kGroup; ++h) {
-                    p[h] = ex2_approx(fmaf(s[h], c, -m_sub[h]));
+                    // rounded to bf16 here: the PV product and the row sum use the same weights
+                    p[h] = __bfloat162float(__float2bfloat16_rn(ex2_approx(fmaf(s[h], c, -m_sub[h]))));
                     l_part[h] = fmaf(l_part[h], alpha[h], p[h]);
                 }
                 // the previous PV must be done with P^T and with O^T
@@ -478,7 +469,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
 __global__ void __launch_bounds__(kD) decode_merge(const __grid_constant__ DecodeArgs a) {
     // launched as a programmatic dependent of decode_split: wait until that
     // grid has completed and its partials are visible
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait();
     const int bh = blockIdx.x;
     const int b = bh / (a.hkv * kGroup);
     const int h = bh % (a.hkv * kGroup);

@@ -62,9 +62,15 @@ struct BlockCfg {
     static constexpr uint32_t OpHalf = NP * 128;                 // one 64-column half of it
     // three K/V stages keep two tiles in flight behind the one being scored;
     // the operand buffers give way when the query rows grow
-    static constexpr int Stages = 3;
+#ifndef DUO_BLK_WIDE_STAGES
+#define DUO_BLK_WIDE_STAGES 3
+#endif
+#ifndef DUO_BLK_WIDE_PB
+#define DUO_BLK_WIDE_PB 1
+#endif
+    static constexpr int Stages = NP <= 32 ? 3 : DUO_BLK_WIDE_STAGES;
     static constexpr int QB = NP <= 32 ? 2 : 1;                  // Q buffers (next item's Q staged early)
-    static constexpr int PB = NP <= 16 ? 2 : 1;                  // P^T buffers
+    static constexpr int PB = NP <= 16 ? 2 : NP <= 32 ? 1 : DUO_BLK_WIDE_PB;   // P^T buffers
     static constexpr size_t Smem = 1024 + Stages * kDecStageBytes + (QB + PB) * OpBytes;
     static_assert(Smem + 4096 <= 232448, "shared memory");
     static constexpr int PartFloats = NR * (kD + 2);             // m[NR], l[NR], acc[NR][D]
@@ -531,7 +537,9 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 float p[NH];
 #pragma unroll
                 for (int q = 0; q < NH; ++q) {
-                    p[q] = ex2_approx(fmaf(s[q], c, m_run[q] == -INFINITY ? 0.f : -m_run[q]));
+                    // rounded to bf16 here: the PV product and the row sum use the same weights
+                    p[q] = __bfloat162float(__float2bfloat16_rn(
+                        ex2_approx(fmaf(s[q], c, m_run[q] == -INFINITY ? 0.f : -m_run[q]))));
                     l_part[q] += p[q];
                 }
                 // the P^T buffer was last read by the PV of tile jg - PB
@@ -628,7 +636,7 @@ template <int kQ>
 __global__ void __launch_bounds__(kD) decode_block_merge(const __grid_constant__ BlockArgs a) {
     using C = BlockCfg<kQ>;
     constexpr int NR = C::NR;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait();
     const DecodeArgs &d = a.d;
     const int hq_all = d.hkv * kGroup;
     const int idx = blockIdx.x;                      // (b * q_len + t) * Hq + h

@@ -2,6 +2,7 @@
 // planning and kernel launches.  Every check runs on the host before the
 // first launch, so a call that returns an error has launched nothing.
 #include <atomic>
+#include <utility>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -150,6 +151,27 @@ int launch_status(const char *what) {
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DUO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
     return DUO_OK;
+}
+
+// Launches kernel<<<grid, block, smem, st>>>(args...) as a programmatic
+// dependent of the kernel before it on the stream: it is scheduled while that
+// one drains, and waits for it on the device (pdl_wait) before touching
+// global memory, so that short kernels in a row overlap their launch and set-up
+// with the previous kernel's tail.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Raises a kernel's dynamic shared-memory limit once per device.  The flags
@@ -332,6 +354,15 @@ int launch_block(duo::BlockArgs &a, int grid, cudaStream_t st, int64_t merge_blo
     return launch_status("decode_block_merge");
 }
 
+// y = 2^x by the prefill's FMA-pipe exponential, two values per thread.
+__global__ void ex2_poly_kernel(const float *x, float *y, int64_t n) {
+    const int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const duo::f2 r = duo::ex2_poly2(duo::f2_make(x[i], i + 1 < n ? x[i + 1] : 0.f));
+    y[i] = r.x;
+    if (i + 1 < n) y[i + 1] = r.y;
+}
+
 }  // namespace
 
 extern "C" {
@@ -362,10 +393,11 @@ int duo_kv_append(const duo_params *params, const duo_cache *cache, const void *
     const int64_t vecs = (int64_t)params->batch * n_new * params->num_kv_heads * duo::kVecPerRow;
     const int64_t blocks = (vecs + 255) / 256;
     if (blocks > INT32_MAX) return fail(DUO_ERR_INVALID_ARG, "append too large for one launch");
-    duo::kv_append_scatter<<<(unsigned)blocks, 256, 0, st>>>(a);
-    if ((rc = launch_status("kv_append_scatter"))) return rc;
-    duo::kv_append_commit<<<(params->batch + 127) / 128, 128, 0, st>>>(
-        cache->seq_len, cache->ring_head, params->batch, n_new, L.sink, L.ring, L.n_full, a.capacity);
+    if (launch_pdl(duo::kv_append_scatter, dim3((unsigned)blocks), dim3(256), 0, st, a) != cudaSuccess)
+        return launch_status("kv_append_scatter");
+    if (launch_pdl(duo::kv_append_commit, dim3((params->batch + 127) / 128), dim3(128), 0, st, cache->seq_len,
+                   cache->ring_head, params->batch, n_new, L.sink, L.ring, L.n_full, a.capacity) != cudaSuccess)
+        return launch_status("kv_append_commit");
     return launch_status("kv_append_commit");
 }
 
@@ -416,10 +448,11 @@ int duo_kv_append_prep(const duo_params *params, const duo_cache *cache, const d
     a.rms_eps = prep->rms_eps;
     a.hq = params->num_q_heads;
     cudaStream_t st = (cudaStream_t)stream;
-    duo::qk_prep_append<<<(unsigned)blocks, duo::kPrepThreads, 0, st>>>(a);
-    if ((rc = launch_status("qk_prep_append"))) return rc;
-    duo::kv_append_commit<<<(params->batch + 127) / 128, 128, 0, st>>>(
-        cache->seq_len, cache->ring_head, params->batch, n_new, L.sink, L.ring, L.n_full, a.app.capacity);
+    if (launch_pdl(duo::qk_prep_append, dim3((unsigned)blocks), dim3(duo::kPrepThreads), 0, st, a) != cudaSuccess)
+        return launch_status("qk_prep_append");
+    if (launch_pdl(duo::kv_append_commit, dim3((params->batch + 127) / 128), dim3(128), 0, st, cache->seq_len,
+                   cache->ring_head, params->batch, n_new, L.sink, L.ring, L.n_full, a.app.capacity) != cudaSuccess)
+        return launch_status("kv_append_commit");
     return launch_status("kv_append_commit");
 }
 
@@ -501,7 +534,9 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     static std::atomic<bool> smem_set[64] = {};
     if ((rc = set_smem_once(duo::decode_split, duo::kDecSmem, "decode_split", smem_set))) return rc;
     if (d.items > 0) {
-        duo::decode_split<<<(unsigned)d.grid, duo::kDecThreads, duo::kDecSmem, st>>>(a);
+        if (launch_pdl(duo::decode_split, dim3((unsigned)d.grid), dim3(duo::kDecThreads), duo::kDecSmem, st, a) !=
+            cudaSuccess)
+            return launch_status("decode_split");
         if ((rc = launch_status("decode_split"))) return rc;
     }
     // the merge is a programmatic dependent launch: it is scheduled while
@@ -682,6 +717,18 @@ int duo_testing_withhold_tile(int32_t kernel, int32_t tile) {
         return fail(DUO_ERR_INVALID_ARG, "unknown kernel %d or tile %d", (int)kernel, (int)tile);
     g_withhold[kernel].store(tile, std::memory_order_relaxed);
     return DUO_OK;
+}
+
+int duo_testing_ex2(const float *x, float *y, int64_t n, void *stream) {
+    if (n < 0 || (n > 0 && (!x || !y || !aligned16(x) || !aligned16(y))))
+        return fail(DUO_ERR_INVALID_ARG, "x / y must be 16-byte aligned device pointers and n >= 0");
+    if (n == 0) return DUO_OK;
+    int rc;
+    if ((rc = check_device(nullptr))) return rc;
+    const int64_t blocks = ((n + 1) / 2 + 255) / 256;
+    if (blocks > INT32_MAX) return fail(DUO_ERR_INVALID_ARG, "n too large for one launch");
+    ex2_poly_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(x, y, n);
+    return launch_status("ex2_poly_kernel");
 }
 
 int duo_get_device_status(void *stream) {

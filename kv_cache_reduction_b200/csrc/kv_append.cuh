@@ -72,6 +72,7 @@ __device__ __forceinline__ int64_t append_row(const AppendArgs &a, int b, int g,
 // One thread copies one 16-byte vector of K and of V.  Rows are
 // (b, t, g) triples in input order, so reads are fully coalesced.
 __global__ void __launch_bounds__(256) kv_append_scatter(AppendArgs a) {
+    pdl_wait();        // launched as a programmatic dependent of the previous kernel
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t rows = (int64_t)a.batch * a.n_new * a.hkv;
     if (idx >= rows * kVecPerRow) return;
@@ -93,6 +94,7 @@ __global__ void __launch_bounds__(256) kv_append_scatter(AppendArgs a) {
 // append's end, which stops at the capacity as append_end says).
 __global__ void kv_append_commit(int32_t *seq_len, int32_t *ring_head, int32_t batch, int32_t n_new,
                                  int32_t sink, int32_t ring, int32_t n_full, int64_t capacity) {
+    pdl_wait();        // the scatter has read seq_len and ring_head
     const int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= batch) return;
     const int64_t n_old = seq_len[b];

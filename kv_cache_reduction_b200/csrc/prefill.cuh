@@ -12,21 +12,20 @@
 // (one per SM) and take (sequence, head pair, query tile) work tiles from a
 // list ordered heaviest first: each claims its next one from an atomic
 // counter when it is ready for it.  Keys come in 128-key tiles.
-//   warps 0-7  softmax of head 0, warps 8-15 softmax of head 1: each query
-//              row is split over two warps (64 keys each, the row max joined
-//              through shared memory); they read S from TMEM, write P (bf16)
+//   warps 0-3  softmax of head 0, warps 4-7 softmax of head 1: one thread per
+//              query row holds the row's 128 scores of a key tile, so the row
+//              max needs no exchange between threads; they write P (bf16)
 //              back over the first 64 columns of S, rescale O in TMEM only when
-//              the running max grew by more than 2^8, and write O / l (times
-//              the output gate, if any) by TMA stores and the log-sum-exp at
-//              the end of each work tile.  The two heads take
-//              turns for the exponentials, so that the MUFU units serve one head
-//              while the tensor core runs the other head's PV and next S
-//   warp 16    TMA producer: claims the work tiles (an atomic counter in the
+//              the running max grew by more than 2^8, and at the end of each
+//              work tile write O / l (times the output gate, if any) by TMA
+//              stores and the log-sum-exp.  A share of the exponentials runs
+//              on the FMA pipe (ex2_poly2) beside the MUFU units
+//   warp 8     TMA producer: claims the work tiles (an atomic counter in the
 //              caller's workspace, else a static stride over the list) and
 //              hands them on through a shared-memory ring; loads Q of both
 //              heads per work tile, K and V tiles into a two-stage ring
 //              (128-byte swizzled, no multicast)
-//   warp 17    TMEM allocator and MMA issuer (one thread), in the order
+//   warp 9     TMEM allocator and MMA issuer (one thread), in the order
 //                PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ...
 //              with S_h = Q_h K^T (both operands in shared memory) and
 //              O_h += P_h V (P_h read from tensor memory).  S_h(j+1) overwrites
@@ -48,7 +47,14 @@ namespace duo {
 
 constexpr int kPfM = 128;                  // query rows per tile
 constexpr int kPfN = 128;                  // keys per tile
-constexpr int kPfThreads = 576;            // 18 warps
+constexpr int kPfThreads = 320;            // 10 warps
+constexpr int kPfProducerWarp = 8, kPfMmaWarp = 9;
+// Pairs of each 16-pair chunk of a row whose exponentials run on the FMA pipe
+// (ex2_poly2) instead of the MUFU units.
+#ifndef DUO_PF_POLY_PAIRS
+#define DUO_PF_POLY_PAIRS 0
+#endif
+constexpr int kPfPolyPairs = DUO_PF_POLY_PAIRS;
 constexpr int kPfStages = 2;
 constexpr int kPfSlots = 4;                // work-tile ring between the producer and the consumers
 constexpr uint32_t kQTileBytes = kPfM * 128 * 2;     // 32 KB: one head's Q tile
@@ -56,8 +62,9 @@ constexpr uint32_t kQHalfBytes = kQTileBytes / 2;    // 64-column swizzled box
 constexpr uint32_t kKVTileBytes = kPfN * 128 * 2;    // 32 KB: one K or V tile
 constexpr uint32_t kKVHalfBytes = kKVTileBytes / 2;
 constexpr uint32_t kPfStageBytes = 2 * kKVTileBytes;
-constexpr uint32_t kOStageBytes = 32 * 16 * 2;    // one softmax warp's O chunk: 32 rows x 16 columns
-constexpr size_t kPfSmem = 1024 + 2 * kQTileBytes + kPfStages * kPfStageBytes + 16 * kOStageBytes;
+constexpr uint32_t kOStageBytes = 32 * 16 * 2;    // one O chunk of a softmax warp: 32 rows x 16 columns
+// each softmax warp stages its O chunks in two alternating buffers
+constexpr size_t kPfSmem = 1024 + 2 * kQTileBytes + kPfStages * kPfStageBytes + 8 * 2 * kOStageBytes;
 
 enum : int { kKindFull = 0, kKindStreaming = 1, kKindSliding = 2 };
 
@@ -143,17 +150,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     char *smem = psmem_base + ((1024u - (smem_u32(psmem_base) & 1023u)) & 1023u);
     char *sQ = smem;                                   // [2 heads][32 KB]
     char *sKV = smem + 2 * kQTileBytes;                // [stages][K 32 KB | V 32 KB]
-    char *sO = sKV + kPfStages * kPfStageBytes;        // [softmax warp][32 rows][16 columns] bf16
+    char *sO = sKV + kPfStages * kPfStageBytes;        // [softmax warp][2][32 rows][16 columns] bf16
     __shared__ uint64_t q_full, q_empty, kv_full[kPfStages], kv_empty[kPfStages];
-    __shared__ uint64_t s_full[2], p_full[2], o_done[2], turn[2];
-    // row-half exchanges between the eight softmax warps of a head (bounded
-    // mbarrier waits, so that a timed-out warp cannot strand its partners)
-    __shared__ uint64_t xmax[2][2], xsum[2];           // [tile parity][head], [head]
+    __shared__ uint64_t s_full[2], p_full[2], o_done[2];
     // work tiles claimed by the producer, read by the MMA issuer and the softmax warps
     __shared__ uint64_t work_full[kPfSlots], work_empty[kPfSlots];
     __shared__ int work_slot[kPfSlots];
-    __shared__ float red_max[2][2][2][kPfM];           // [tile parity][head][column half][row]
-    __shared__ float red_sum[2][2][kPfM];              // [head][column half][row]
     __shared__ uint32_t tmem_base;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -166,21 +168,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         }
         for (int h = 0; h < 2; ++h) {
             mbar_init(&s_full[h], 1);
-            mbar_init(&p_full[h], 8);
+            mbar_init(&p_full[h], 4);           // the head's four softmax warps
             mbar_init(&o_done[h], 1);
-            mbar_init(&turn[h], 8);
-            mbar_init(&xmax[0][h], 8);
-            mbar_init(&xmax[1][h], 8);
-            mbar_init(&xsum[h], 8);
         }
         for (int sl = 0; sl < kPfSlots; ++sl) {
             mbar_init(&work_full[sl], 1);
-            mbar_init(&work_empty[sl], 17);     // the MMA issuer and the 16 softmax warps
+            mbar_init(&work_empty[sl], 9);      // the MMA issuer and the 8 softmax warps
         }
-        for (int w8 = 0; w8 < 8; ++w8) mbar_arrive(&turn[0]);   // head 0 takes the first turn
         fence_mbar_init();
     }
-    if (warp == 17) {
+    if (warp == kPfMmaWarp) {
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
@@ -190,7 +187,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     tc_fence_after();
     const uint32_t tmem = tmem_base;
 
-    if (warp == 16) {
+    if (warp == kPfProducerWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&a.tm_q);
@@ -241,7 +238,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             }
         }
         __syncwarp();  // lanes 1..31 wait for the producer lane before the CTA barrier
-    } else if (warp == 17) {
+    } else if (warp == kPfMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(kPfM, kPfN, 0, 0);
@@ -332,9 +329,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         __syncwarp();  // lanes 1..31 wait for the MMA lane before the CTA barrier
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int h = warp >> 3;                       // head of the pair
+        const int h = warp >> 2;                       // head of the pair
         const int quarter = warp & 3;                  // TMEM lane quarter of this warp
-        const int half = (warp >> 2) & 1;              // key columns [64*half, 64*half + 64)
         const int r = quarter * 32 + lane;             // query row within the tile
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const uint32_t s_tmem = tmem + h * 128 + lane_base;
@@ -357,59 +353,60 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             const int n_kv = tl.count();
             const int i = wk.t * kPfM + r;             // query position
             const int hq = wk.h0 + h;
-            // running max (log2 units) and this half's share of the sum; a sink
-            // logit starts them at (sigma, 1), counted once (in half 0)
+            // running max (log2 units) and sum; a sink logit starts them at (sigma, 1)
             float m_run = -INFINITY, l_run = 0.f;
             if (a.sink_logit != nullptr) {
                 m_run = a.sink_logit[hq] * kLog2eF;
-                l_run = half == 0 ? 1.f : 0.f;
+                l_run = 1.f;
             }
             for (int j = 0; j < n_kv; ++j, ++jg) {
                 const bool got = mbar_wait(&s_full[h], jg & 1);
                 __syncwarp();      // tcgen05.ld below is warp-collective
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sr[64];
-                tmem_ld32(s_tmem + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(s_tmem + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_ld_wait();
-                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                const int c0 = tl.at(j) * kPfN;
-                const bool dense = tile_dense(kind, wk.t * kPfM, c0, a.sink, a.recent, a.window);
-                if (!dense) {
-                    // the row's attended keys among this half's 64 columns as a bit
-                    // mask built from their one or two ranges
-                    const int cb0 = c0 + half * 64;
-                    const int di = i - cb0;                    // the diagonal's column
-                    uint64_t m;
-                    if (kind == kKindFull)
-                        m = col_range_bits(0, di);
-                    else if (kind == kKindStreaming)
-                        m = col_range_bits(0, min(di, a.sink - 1 - cb0)) | col_range_bits(di - a.recent + 1, di);
-                    else
-                        m = col_range_bits(di - a.window + 1, di);
-                    const uint32_t mlo = (uint32_t)m, mhi = (uint32_t)(m >> 32);
+                uint32_t sr[128];
 #pragma unroll
-                    for (int cc = 0; cc < 64; ++cc)
-                        if (!((((cc < 32) ? mlo : mhi) >> (cc & 31)) & 1u)) sr[cc] = __float_as_uint(-INFINITY);
+                for (int q4 = 0; q4 < 4; ++q4)
+                    tmem_ld32(s_tmem + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q4 * 32]));
+                tmem_ld_wait();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[q4 * 32]));
+                const int c0 = tl.at(j) * kPfN;
+                if (!tile_dense(kind, wk.t * kPfM, c0, a.sink, a.recent, a.window)) {
+                    // the row's attended keys among the tile's 128 columns as two
+                    // 64-bit masks built from their one or two ranges
+                    const int di = i - c0;                     // the diagonal's column
+                    int lo0, hi0, lo1 = 1, hi1 = 0;            // attended columns [lo0, hi0] u [lo1, hi1]
+                    if (kind == kKindFull) {
+                        lo0 = 0;
+                        hi0 = di;
+                    } else if (kind == kKindStreaming) {
+                        lo0 = 0;
+                        hi0 = min(di, a.sink - 1 - c0);
+                        lo1 = di - a.recent + 1;
+                        hi1 = di;
+                    } else {
+                        lo0 = di - a.window + 1;
+                        hi0 = di;
+                    }
+                    const uint64_t m0 = col_range_bits(lo0, hi0) | col_range_bits(lo1, hi1);
+                    const uint64_t m1 = col_range_bits(lo0 - 64, hi0 - 64) | col_range_bits(lo1 - 64, hi1 - 64);
+                    const uint32_t mw[4] = {(uint32_t)m0, (uint32_t)(m0 >> 32), (uint32_t)m1, (uint32_t)(m1 >> 32)};
+#pragma unroll
+                    for (int cc = 0; cc < 128; ++cc)
+                        if (!((mw[cc >> 5] >> (cc & 31)) & 1u)) sr[cc] = __float_as_uint(-INFINITY);
                 }
+                // the row max over the tile, eight independent chains of 3-input max
                 float mx8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
 #pragma unroll
-                for (int cc = 8; cc < 64; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(sr[cc]));
-                const float mx_half = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                            fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-                // join the two halves of the row (both have read their S by now,
-                // so P may overwrite any of the first 64 columns afterwards)
-                red_max[jg & 1][h][half][r] = mx_half;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&xmax[jg & 1][h]);
-                const bool joined = mbar_wait(&xmax[jg & 1][h], (jg >> 1) & 1);
-                __syncwarp();
-                if (!__all_sync(0xffffffffu, joined)) { ok = false; break; }
-                const float m_tile = fmaxf(mx_half, red_max[jg & 1][h][half ^ 1][r]) * c;
+                for (int cc = 8; cc < 128; cc += 16)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        mx8[e] = fmax3(mx8[e], __uint_as_float(sr[cc + e]), __uint_as_float(sr[cc + 8 + e]));
+                const float m_tile = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                           fmaxf(mx8[6], mx8[7])) * c;
                 // keep the stale max unless the new one is more than 2^8 larger
                 float m_use = m_run, alpha = 1.f;
                 if (m_tile > m_run + 8.f) {
@@ -417,50 +414,47 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_tile);
                 }
                 const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-                // this head's turn on the MUFU units
-                const bool my_turn = mbar_wait(&turn[h], jg & 1);
-                __syncwarp();
-                if (!__all_sync(0xffffffffu, my_turn)) { ok = false; break; }
-                // score * c - max on the packed f32x2 pipe, two columns per instruction
+                // score * c - max on the packed f32x2 pipe, two columns per
+                // instruction; the row sum adds the bf16 weights the PV product
+                // uses, so that numerator and denominator agree
                 const f2 c2 = f2_splat(c), ms2 = f2_splat(-m_sub);
-                f2 ls01 = f2_splat(0.f), ls23 = f2_splat(0.f);
+                f2 ls0 = f2_splat(0.f), ls1 = f2_splat(0.f);
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    uint32_t pw[16];
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t pw[8];
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const int cc = ch * 32 + e;
-                        const f2 a01 = f2_fma(f2_make(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), c2, ms2);
-                        const f2 a23 = f2_fma(f2_make(__uint_as_float(sr[cc + 2]), __uint_as_float(sr[cc + 3])), c2, ms2);
-                        const uint32_t w01 = pack_bf16x2(ex2_approx(a01.x), ex2_approx(a01.y));
-                        const uint32_t w23 = pack_bf16x2(ex2_approx(a23.x), ex2_approx(a23.y));
-                        // the row sum adds the bf16 weights the PV product uses, so
-                        // that numerator and denominator agree
-                        ls01 = f2_add(ls01, f2_make(bf16lo(w01), bf16hi(w01)));
-                        ls23 = f2_add(ls23, f2_make(bf16lo(w23), bf16hi(w23)));
-                        pw[e / 2] = w01;
-                        pw[e / 2 + 1] = w23;
+                    for (int e = 0; e < 8; ++e) {
+                        const int cc = ch * 16 + 2 * e;
+                        const f2 x = f2_fma(f2_make(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), c2, ms2);
+                        f2 pe;
+                        if ((ch & 1) * 8 + e < kPfPolyPairs) {
+                            pe = ex2_poly2(x);
+                        } else {
+                            pe.x = ex2_approx(x.x);
+                            pe.y = ex2_approx(x.y);
+                        }
+                        const uint32_t wv = pack_bf16x2(pe.x, pe.y);
+                        pw[e] = wv;
+                        if (e & 1) ls1 = f2_add(ls1, f2_make(bf16lo(wv), bf16hi(wv)));
+                        else ls0 = f2_add(ls0, f2_make(bf16lo(wv), bf16hi(wv)));
                     }
-                    // P of keys [64*half + 32*ch, +32) -> TMEM columns [32*half + 16*ch, +16)
-                    tmem_st16(s_tmem + half * 32 + ch * 16, pw);
+                    // P of keys [16 ch, 16 ch + 16) -> TMEM columns [8 ch, 8 ch + 8)
+                    tmem_st8(s_tmem + ch * 8, pw);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&turn[h ^ 1]);
-                l_run = l_run * alpha + ((ls01.x + ls01.y) + (ls23.x + ls23.y));
+                l_run = l_run * alpha + ((ls0.x + ls0.y) + (ls1.x + ls1.y));
                 m_run = m_use;
                 // O holds the previous key tiles' sum (its PV is complete: this S
-                // was computed after it); rescale this half's 64 columns when the
-                // max moved
+                // was computed after it); rescale the row when the max moved
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                    for (int cb = 0; cb < 64; cb += 32) {
+                    for (int cb = 0; cb < 128; cb += 32) {
                         uint32_t orr[32];
-                        tmem_ld32(o_tmem + half * 64 + cb, orr);
+                        tmem_ld32(o_tmem + cb, orr);
                         tmem_ld_wait();
                         reg_fence32(orr);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                        tmem_st32(o_tmem + half * 64 + cb, orr);
+                        tmem_st32(o_tmem + cb, orr);
                     }
                 }
                 tmem_st_wait();
@@ -470,10 +464,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             }
             if (!ok) break;
             // ------------------------------------------------------------ work-tile epilogue
-            // the output gate of this row's 64 channels (16 at a time, one chunk
-            // ahead) or of its head; the first loads overlap the waits below
+            // the output gate of this row's channels (16 at a time, one chunk
+            // ahead) or of its head; the first loads overlap the wait below
             const uint4 *gp = reinterpret_cast<const uint4 *>(
-                a.gate + (((size_t)wk.b * a.L + i) * a.hq + hq) * 128 + half * 64);
+                a.gate + (((size_t)wk.b * a.L + i) * a.hq + hq) * 128);
             uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
             float g_head = 0.f;
             if (kGate == 1 && i < a.L) {
@@ -482,45 +476,43 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             } else if (kGate == 2 && i < a.L) {
                 g_head = __bfloat162float(a.gate[((size_t)wk.b * a.L + i) * a.hq + hq]);
             }
-            red_sum[h][half][r] = l_run;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xsum[h]);
-            const bool o_fin = mbar_wait(&o_done[h], (jg - 1) & 1) && mbar_wait(&xsum[h], wc & 1);
+            const bool o_fin = mbar_wait(&o_done[h], (jg - 1) & 1);
             __syncwarp();
             if (!__all_sync(0xffffffffu, o_fin)) { ok = false; break; }
             tc_fence_after();
-            const float l_row = red_sum[h][0][r] + red_sum[h][1][r];
-            const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
             // o * sigmoid(g): one factor per row, or one per channel below
             const float row_mul = kGate == 2 ? inv_l / (1.f + ex2_approx(-g_head * kLog2eF)) : inv_l;
-            // O / l leaves through this warp's 1 KB staging buffer as 32-row x
+            // O / l leaves through this warp's two 1 KB staging buffers as 32-row x
             // 16-column TMA stores (rows past L are clipped by the tensor map):
             // coalesced by the copy engine instead of 32 scattered rows per store
-            char *stage = sO + warp * kOStageBytes;
             const int row0 = wk.t * kPfM + quarter * 32;   // first row of this warp's boxes
 #pragma unroll
-            for (int cb = 0; cb < 64 && row0 < a.L; cb += 32) {
+            for (int cb = 0; cb < 128 && row0 < a.L; cb += 32) {
                 uint32_t orr[32];
-                tmem_ld32(o_tmem + half * 64 + cb, orr);
+                tmem_ld32(o_tmem + cb, orr);
                 tmem_ld_wait();
                 reg_fence32(orr);
 #pragma unroll
                 for (int c16 = 0; c16 < 32; c16 += 16) {
+                    const int chunk = (cb + c16) / 16;     // 0..7
                     uint4 n0 = g0, n1 = g1;                // the next chunk's gates
-                    if (kGate == 1 && cb + c16 + 16 < 64 && i < a.L) {
-                        n0 = __ldg(gp + (cb + c16 + 16) / 8);
-                        n1 = __ldg(gp + (cb + c16 + 16) / 8 + 1);
+                    if (kGate == 1 && chunk + 1 < 8 && i < a.L) {
+                        n0 = __ldg(gp + 2 * (chunk + 1));
+                        n1 = __ldg(gp + 2 * (chunk + 1) + 1);
                     }
-                    if (lane == 0) bulk_wait_read_all();   // the previous chunk has left the buffer
+                    char *stage = sO + (warp * 2 + (chunk & 1)) * kOStageBytes;
+                    // the store that last used this buffer (two chunks ago) has read it
+                    if (lane == 0) bulk_wait_read_1();
                     __syncwarp();
                     auto nb = [&](int e) {
                         float m0 = row_mul, m1 = row_mul;
                         if (kGate == 1) {
                             // channels e, e + 1 of the chunk: one bf16 pair of its gates
                             const uint4 q4 = e < 8 ? g0 : g1;
-                            const uint32_t w = (e & 7) < 2 ? q4.x : (e & 7) < 4 ? q4.y : (e & 7) < 6 ? q4.z : q4.w;
-                            m0 = inv_l / (1.f + ex2_approx(-__uint_as_float(w << 16) * kLog2eF));
-                            m1 = inv_l / (1.f + ex2_approx(-__uint_as_float(w & 0xffff0000u) * kLog2eF));
+                            const uint32_t gw = (e & 7) < 2 ? q4.x : (e & 7) < 4 ? q4.y : (e & 7) < 6 ? q4.z : q4.w;
+                            m0 = inv_l / (1.f + ex2_approx(-__uint_as_float(gw << 16) * kLog2eF));
+                            m1 = inv_l / (1.f + ex2_approx(-__uint_as_float(gw & 0xffff0000u) * kLog2eF));
                         }
                         return pack_bf16x2(__uint_as_float(orr[c16 + e]) * m0,
                                            __uint_as_float(orr[c16 + e + 1]) * m1);
@@ -533,19 +525,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     fence_proxy_async_smem();              // visible to the copy engine
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_4d(&a.tm_o, stage, half * 64 + cb + c16, hq, row0, wk.b);
+                        tma_store_4d(&a.tm_o, stage, cb + c16, hq, row0, wk.b);
                         bulk_commit_group();
                     }
                     g0 = n0;
                     g1 = n1;
                 }
             }
-            if (a.lse != nullptr && i < a.L && half == 0)
+            if (a.lse != nullptr && i < a.L)
                 a.lse[((size_t)wk.b * a.hq + hq) * a.L + i] =
-                    l_row > 0.f ? (m_run + __log2f(l_row)) * kLn2F : -INFINITY;
+                    l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2F : -INFINITY;
             // O is read before this warp's first p_full arrival of the next work
-            // tile, and red_sum before its next row-max exchange, so neither the
-            // next PV nor the next epilogue can overwrite them early
+            // tile, so the next PV (which overwrites O) cannot start early
             tc_fence_before();
         }
         if (lane == 0) bulk_wait_all();                    // this warp's O stores have landed
@@ -553,7 +544,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 17) {
+    if (warp == kPfMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -24,6 +24,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched as a programmatic dependent may start while the kernel
+// before it on the stream drains; pdl_wait() blocks until that kernel has
+// completed and its writes are visible.  Every such kernel calls it before
+// its first global-memory access that could depend on, or overwrite, what the
+// previous kernel reads or writes.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -114,6 +122,12 @@ __device__ __forceinline__ void bulk_commit_group() {
 // Waits until this thread's committed bulk stores have read their shared-memory source.
 __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Waits until at most the most recent committed bulk-store group still reads
+// its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 // Waits until this thread's committed bulk stores have completed.
@@ -219,6 +233,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+                   "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -316,6 +344,43 @@ __device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
     uint64_t d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
     return f2_from_bits(d);
+}
+
+__device__ __forceinline__ f2 f2_sub(f2 a, f2 b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return f2_from_bits(d);
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair on the FMA pipe, so that part of the softmax's exponentials
+// leave the MUFU units free.  Range reduction after Cody and Waite: x = n + f
+// with n the nearest integer (adding 1.5 * 2^23 rounds x to an integer in the
+// low mantissa bits) and |f| <= 1/2; 2^f from a degree-3 polynomial fitted
+// for this library by a Remez exchange on the relative error over [-1/2, 1/2]
+// (largest relative error 7.5e-5, below a bf16 half-ulp); 2^n enters by adding
+// n to the exponent field.  x is clamped at -125 so that the exponent stays in
+// range: inputs below it (masked scores are -inf) give about 2^-125 instead
+// of 0, which no bf16 sum of terms near 1 can see.
+__device__ __forceinline__ f2 ex2_poly2(f2 x) {
+    constexpr float kRound = 12582912.f;                   // 1.5 * 2^23
+    constexpr float kC0 = 0.99992805719375610f, kC1 = 0.69326096773147583f;
+    constexpr float kC2 = 0.24261112511157990f, kC3 = 0.05517166852951050f;
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const f2 j = f2_add(x, f2_splat(kRound));
+    const f2 f = f2_sub(x, f2_sub(j, f2_splat(kRound)));
+    f2 p = f2_fma(f2_splat(kC3), f, f2_splat(kC2));
+    p = f2_fma(p, f, f2_splat(kC1));
+    p = f2_fma(p, f, f2_splat(kC0));
+    return f2_make(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
+                   __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
 }
 
 // Packs two floats to bf16x2 (round to nearest even): lo -> bits 0..15.

@@ -7,10 +7,9 @@
 // rotary embedding).  One CTA per (sequence, token): 64 threads compute the
 // token's cos / sin table once (the angle p * inv_freq in double precision and
 // reduced modulo 2 pi in double, so that positions up to 2^30 keep their
-// phase), then 16 threads per head row
-// normalise it, rotate the pairs (i, i + 64) and write it back in place; key
-// rows also go to the cache with their values, with the append's survivor
-// rule for ring heads.
+// phase), then 8 threads per head row normalise it, rotate the pairs
+// (i, i + 64) and write it back in place; key rows also go to the cache with
+// their values, with the append's survivor rule for ring heads.
 #pragma once
 
 #include "kv_append.cuh"
@@ -36,30 +35,35 @@ __device__ __forceinline__ void unpack8(const uint4 u, float *x) {
     }
 }
 
-constexpr int kPrepThreads = 128;   // 8 head rows at a time, 16 threads each
+constexpr int kPrepThreads = 128;   // 16 head rows at a time, 8 threads each
+constexpr int kPrepBatch = 4;       // head rows an 8-thread group has in flight at once
 
-constexpr int kPrepBatch = 8;       // head rows a 16-thread group has in flight at once
-
+// One CTA per (sequence, token).  Thread j of a row's group of 8 holds the
+// channels [8j, 8j + 8) and their rotation partners [64 + 8j, 64 + 8j + 8), so
+// that the rotation needs no exchange between threads and every load and store
+// is 16 bytes wide; the sum of squares is reduced over the 8 threads.
 __global__ void __launch_bounds__(kPrepThreads) qk_prep_append(const __grid_constant__ PrepArgs a) {
+    pdl_wait();        // launched as a programmatic dependent of the previous kernel
     const AppendArgs &ap = a.app;
     const int tok = blockIdx.x;
     const int b = tok / ap.n_new;
     const int64_t t = tok % ap.n_new;
     const int64_t tok_row = (int64_t)b * ap.n_new + t;
     const int rows = a.hq + ap.hkv;
-    const int grp = (int)(threadIdx.x >> 4);        // head rows grp, grp + 8, ...
-    const int j = threadIdx.x & 15;                 // channels [8j, 8j + 8) of a row
+    const int grp = (int)(threadIdx.x >> 3);        // head rows grp, grp + 16, ...
+    const int j = threadIdx.x & 7;                  // channels [8j, 8j + 8) and [64 + 8j, 64 + 8j + 8)
+    constexpr int step = kPrepThreads / 8;
     auto row_ptr = [&](int r) -> uint4 * {
         return r < a.hq ? a.q + (tok_row * a.hq + r) * kVecPerRow
                         : a.kw + (tok_row * ap.hkv + (r - a.hq)) * kVecPerRow;
     };
-    const int step = kPrepThreads / 16;
-    // first batch of rows in flight before the cos / sin table is built
-    uint4 xin[kPrepBatch];
+    // the first batch of rows in flight before the cos / sin table is built
+    uint4 xlo[kPrepBatch], xhi[kPrepBatch];
 #pragma unroll
     for (int u = 0; u < kPrepBatch; ++u) {
         const int r = grp + u * step;
-        xin[u] = r < rows ? row_ptr(r)[j] : make_uint4(0, 0, 0, 0);
+        xlo[u] = r < rows ? row_ptr(r)[j] : make_uint4(0, 0, 0, 0);
+        xhi[u] = r < rows ? row_ptr(r)[8 + j] : make_uint4(0, 0, 0, 0);
     }
     const int64_t pos = (int64_t)ap.seq_len[b] + t;
     __shared__ float cs[64], sn[64];
@@ -80,22 +84,23 @@ __global__ void __launch_bounds__(kPrepThreads) qk_prep_append(const __grid_cons
         sn[threadIdx.x] = (float)s * a.attention_factor;
     }
     __syncthreads();
-    const int f0 = (j & 7) * 8;                     // frequency index of channel 8j (mod 64)
-    const bool lo = j < 8;                          // first half of the (i, i + 64) pairs
-    float wq[8], wk[8], c8[8], s8[8];
+    float wq[16], wk[16], c8[8], s8[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
         wq[e] = a.q_w ? __bfloat162float(a.q_w[8 * j + e]) : 1.f;
+        wq[8 + e] = a.q_w ? __bfloat162float(a.q_w[64 + 8 * j + e]) : 1.f;
         wk[e] = a.k_w ? __bfloat162float(a.k_w[8 * j + e]) : 1.f;
-        c8[e] = cs[f0 + e];
-        s8[e] = lo ? -sn[f0 + e] : sn[f0 + e];      // out = y cos -/+ partner sin
+        wk[8 + e] = a.k_w ? __bfloat162float(a.k_w[64 + 8 * j + e]) : 1.f;
+        c8[e] = cs[8 * j + e];
+        s8[e] = sn[8 * j + e];
     }
     for (int rb = 0; rb < rows; rb += kPrepBatch * step) {
         if (rb > 0) {
 #pragma unroll
             for (int u = 0; u < kPrepBatch; ++u) {
                 const int r = rb + grp + u * step;
-                xin[u] = r < rows ? row_ptr(r)[j] : make_uint4(0, 0, 0, 0);
+                xlo[u] = r < rows ? row_ptr(r)[j] : make_uint4(0, 0, 0, 0);
+                xhi[u] = r < rows ? row_ptr(r)[8 + j] : make_uint4(0, 0, 0, 0);
             }
         }
 #pragma unroll
@@ -103,51 +108,53 @@ __global__ void __launch_bounds__(kPrepThreads) qk_prep_append(const __grid_cons
             const int r = rb + grp + u * step;
             const bool active = r < rows;
             const bool is_q = r < a.hq;
-            float x[8];
-            unpack8(xin[u], x);
+            float lo[8], hi[8];
+            unpack8(xlo[u], lo);
+            unpack8(xhi[u], hi);
             // pairs of channels through the packed f32x2 pipe
-            f2 ss2 = f2_mul(f2_make(x[0], x[1]), f2_make(x[0], x[1]));
+            f2 ss2 = f2_mul(f2_make(lo[0], lo[1]), f2_make(lo[0], lo[1]));
 #pragma unroll
-            for (int e = 2; e < 8; e += 2) ss2 = f2_fma(f2_make(x[e], x[e + 1]), f2_make(x[e], x[e + 1]), ss2);
+            for (int e = 2; e < 8; e += 2) ss2 = f2_fma(f2_make(lo[e], lo[e + 1]), f2_make(lo[e], lo[e + 1]), ss2);
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) ss2 = f2_fma(f2_make(hi[e], hi[e + 1]), f2_make(hi[e], hi[e + 1]), ss2);
             float ss = f2_sum(ss2);
-            // the 16 threads of a row are 16 consecutive lanes: reduce within them
+            // the 8 threads of a row are 8 consecutive lanes: reduce within them
 #pragma unroll
-            for (int m = 1; m < 16; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+            for (int m = 1; m < 8; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
             const f2 inv2 = f2_splat(rsqrtf(ss * (1.f / 128.f) + a.rms_eps));
-            f2 y2[4];
+            uint32_t olo[4], ohi[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                y2[e] = f2_mul(f2_mul(f2_make(x[2 * e], x[2 * e + 1]), inv2),
-                               is_q ? f2_make(wq[2 * e], wq[2 * e + 1]) : f2_make(wk[2 * e], wk[2 * e + 1]));
-            f2 p2[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                p2[e].x = __shfl_xor_sync(0xffffffffu, y2[e].x, 8);   // channel +-64
-                p2[e].y = __shfl_xor_sync(0xffffffffu, y2[e].y, 8);
-            }
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const f2 r2 = f2_fma(p2[e], f2_make(s8[2 * e], s8[2 * e + 1]),
-                                     f2_mul(y2[e], f2_make(c8[2 * e], c8[2 * e + 1])));
-                o[e] = pack_bf16x2(r2.x, r2.y);
+            for (int e = 0; e < 8; e += 2) {
+                const f2 wlo = is_q ? f2_make(wq[e], wq[e + 1]) : f2_make(wk[e], wk[e + 1]);
+                const f2 whi = is_q ? f2_make(wq[8 + e], wq[9 + e]) : f2_make(wk[8 + e], wk[9 + e]);
+                const f2 ylo = f2_mul(f2_mul(f2_make(lo[e], lo[e + 1]), inv2), wlo);
+                const f2 yhi = f2_mul(f2_mul(f2_make(hi[e], hi[e + 1]), inv2), whi);
+                const f2 cc = f2_make(c8[e], c8[e + 1]), sc = f2_make(s8[e], s8[e + 1]);
+                // (y_i, y_{i+64}) rotated by the angle of pair i
+                const f2 rlo = f2_fma(yhi, f2_make(-sc.x, -sc.y), f2_mul(ylo, cc));
+                const f2 rhi = f2_fma(ylo, sc, f2_mul(yhi, cc));
+                olo[e / 2] = pack_bf16x2(rlo.x, rlo.y);
+                ohi[e / 2] = pack_bf16x2(rhi.x, rhi.y);
             }
             if (!active) continue;
-            const uint4 out = make_uint4(o[0], o[1], o[2], o[3]);
-            row_ptr(r)[j] = out;
+            const uint4 out_lo = make_uint4(olo[0], olo[1], olo[2], olo[3]);
+            const uint4 out_hi = make_uint4(ohi[0], ohi[1], ohi[2], ohi[3]);
+            uint4 *rp = row_ptr(r);
+            rp[j] = out_lo;
+            rp[8 + j] = out_hi;
             if (!is_q) {
                 const int g = r - a.hq;
                 bool full = false;
                 const int64_t row = append_row(ap, b, g, t, &full);
                 if (row >= 0) {
-                    const uint4 vv = ap.v[(tok_row * ap.hkv + g) * kVecPerRow + j];
-                    if (full) {
-                        ap.full_k[row * kVecPerRow + j] = out;
-                        ap.full_v[row * kVecPerRow + j] = vv;
-                    } else {
-                        ap.strm_k[row * kVecPerRow + j] = out;
-                        ap.strm_v[row * kVecPerRow + j] = vv;
-                    }
+                    const uint4 *vr = ap.v + (tok_row * ap.hkv + g) * kVecPerRow;
+                    const uint4 v_lo = vr[j], v_hi = vr[8 + j];
+                    uint4 *kd = (full ? ap.full_k : ap.strm_k) + row * kVecPerRow;
+                    uint4 *vd = (full ? ap.full_v : ap.strm_v) + row * kVecPerRow;
+                    kd[j] = out_lo;
+                    kd[8 + j] = out_hi;
+                    vd[j] = v_lo;
+                    vd[8 + j] = v_hi;
                 }
             }
         }
