@@ -787,7 +787,37 @@ class DecodeSmall:
         torch.cuda.synchronize()
         return sum(a.elapsed_time(b) for a, b in evs) / 1e3 / reps
 
-    def measure_line(self, reps, warmup):
+    def oracle_sample(self, budget_s: float = 15.0):
+        """The oracle on the same workload: the prompt's prefill (every row) and
+        the 16 decode steps against its own sequentially appended cache, each
+        timed on the host cores; repeated while the budget lasts."""
+        import oracle
+        p = self.params
+        ol = oracle.Layer(1, 48, 8, 128, p.sink, p.recent, 0, p.softmax_scale, tuple(p.full_mask), None)
+        qb, kb, vb = inputs.bits(self.qp), inputs.bits(self.kp), inputs.bits(self.vp)
+        k1, v1, q1 = inputs.bits(self.k1), inputs.bits(self.v1), inputs.bits(self.q1)
+        t_pre, t_dec, runs = 0.0, 0.0, 0
+        while runs == 0 or t_pre + t_dec < budget_s:
+            t0 = time.perf_counter()
+            oracle.attn_prefill(ol, qb, kb, vb)
+            t1 = time.perf_counter()
+            hc = oracle.Cache(ol, self.cap)
+            oracle.kv_append(ol, hc, kb, vb)
+            t_dec_run = 0.0
+            for s in range(self.STEPS):
+                t2 = time.perf_counter()
+                oracle.kv_append(ol, hc, k1[s], v1[s])
+                oracle.attn_decode(ol, hc, q1[s])
+                t_dec_run += time.perf_counter() - t2
+            t_pre += t1 - t0
+            t_dec += t_dec_run
+            runs += 1
+        return {"value": round(t_dec / (runs * self.STEPS) * 1e6, 2), "unit": "us/step",
+                "prefill_us": round(t_pre / runs * 1e6, 2), "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": f"{runs} runs of the whole workload (prefill of the 1024-token prompt, every row, "
+                          f"then 16 x (append + decode)), float64"}
+
+    def measure_line(self, reps, warmup, cpu_budget=0.0):
         self.capture()
         for _ in range(warmup):
             self.replay()
@@ -812,7 +842,8 @@ class DecodeSmall:
                 "note": "decode steps replayed from one CUDA graph of 16 steps (append + decode each); "
                         "prefill_us: the 1024-token prompt's duo_attn_prefill; L2 flushed before "
                         "every timed call",
-                "clocks": clk.summary()}
+                "clocks": clk.summary(),
+                **({"cpu_baseline": self.oracle_sample(cpu_budget)} if cpu_budget > 0 else {})}
 
     def config(self):
         return {"workload": "decode_small: B=1, prefill of a 1024-token prompt, then 16 x "
@@ -993,7 +1024,7 @@ def run_ours(args, world, rank):
             try:
                 w2 = WORKLOADS[name](rank)
                 if hasattr(w2, "measure_line"):
-                    sec[name] = w2.measure_line(st, args.warmup)
+                    sec[name] = w2.measure_line(st, args.warmup, budget / 2 if world == 1 and rank == 0 else 0.0)
                 else:
                     line = measure_line(w2, args, world, rank, st, budget / 2, pk, pk_kind)
                     line["frac"] = line["roofline"]["frac"]

@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
     char *sQ = smem + kDecStages * kDecStageBytes;            // [2 items][4 KB]
     char *sP = sQ + 2 * kOpBytes;                             // 4 KB
     __shared__ uint64_t kv_full[kDecStages], kv_empty[kDecStages];
-    __shared__ uint64_t s_full[2], p_full, o_done, q_ready[2];
+    __shared__ uint64_t s_full[2], p_full, o_done, q_ready[2], mma_drained;
     __shared__ uint32_t tmem_base;
     __shared__ float red_max[2][4][kGroup], red_sum[4][kGroup];
 
@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
         }
         mbar_init(&p_full, 4);
         mbar_init(&o_done, 1);
+        mbar_init(&mma_drained, 1);
         fence_mbar_init();
     }
     if (warp < 4) {
@@ -293,6 +294,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
                 mma_commit(&o_done);
                 mma_commit(&kv_empty[pend_st]);
             }
+            // every product issued has completed before the tensor memory is freed
+            // (on an early exit some may still run)
+            mma_commit(&mma_drained);
+            mbar_wait(&mma_drained, 0);
         }
         __syncwarp();
     } else {

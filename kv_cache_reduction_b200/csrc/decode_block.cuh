@@ -16,20 +16,28 @@
 // The cache is not modified; the caller appends the accepted tokens with
 // duo_kv_append afterwards.
 //
-// The structure is the one-token decode's (decode.cuh): persistent CTAs over
-// (sequence, KV head, split) items, "swap AB" products with the tokens of a
-// 128-token tile in M and the query rows in N:
-//   S^T[128 tok x NP] = K_tile . Q^T,   O^T[128 d x NP] += V_tile^T . P^T
-// with NR = 6 * q_len query rows (row t*6 + h: block token t, head h of the
-// group) padded to NP = 16, 32 or 48.  Each (sequence, KV head) has one
-// more tile for the block's keys: one 128-row tile of the block's K/V (rows
-// past q_len are zero-filled by the tensor map and masked), the last tile of
-// that head's last split item.  Every key token
-// carries the range [t_lo, t_hi] of block queries that may attend to it.
-// The softmax of a tile is split over two or three warps per TMEM lane
-// quarter (at most 16 query rows per thread), and one vote across them
-// (bar.red.or) skips the row-max reduction on tiles where no score exceeds its
-// row's running max by more than 2^8 -- the same result as reducing.
+// Work items are (sequence, KV head, split) as in the one-token decode, with
+// one more 128-row tile for the block's own keys on each head's last split
+// (rows past q_len are zero-filled by the tensor map).  Persistent CTAs claim
+// items from a counter, heaviest first.  The NR = 6 * q_len query rows of an
+// item (row t*6 + h: block token t, head h of the group) sit in the M
+// dimension of the products, spread over the four TMEM lane quarters
+// (RQ = ceil(NR / 4) rows each), so that one thread holds one query row and
+// its 128 scores of a key tile:
+//   S[128 x 128 keys] = Q . K_tile^T     (Q in tensor memory, K from shared)
+//   O[128 x 128 d]   += P . V_tile       (P over S in tensor memory)
+// with the rows past NR padding.  Two S buffers let the product of tile j + 2
+// (and j + 1) run while the softmax works on tile j.
+//   warps 0-3  softmax and epilogue: stage the next item's Q into tensor
+//              memory, read S, mask, exponentials, P back over S, the item's
+//              partial (O, running max, sum) to the workspace
+//   warp 4     key preparation: per tile, the range of block queries each key
+//              serves, as one 128-bit key mask per block token, and zeroes the
+//              V rows no query keeps (stale cache memory never reaches the PV
+//              product)
+//   warp 5     TMA producer (K and V tiles, three stages; claims the items)
+//   warp 6     TMEM owner and MMA issuer
+// TMEM: S_a | S_b | O (128 fp32 columns each) | Q_0 | Q_1 (64 columns each).
 #pragma once
 
 #include <cuda.h>
@@ -38,117 +46,22 @@
 
 namespace duo {
 
-__device__ __forceinline__ void blk_tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-        "%12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-
-__device__ __forceinline__ void blk_reg_fence16(uint32_t (&r)[16]) {
-    asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
-}
-
 template <int kQ>
 struct BlockCfg {
     static constexpr int NR = kGroup * kQ;                       // query rows per item
-    static constexpr int NP = (NR + 15) / 16 * 16;               // MMA N
-    static constexpr uint32_t OpBytes = NP * kD * 2;             // Q or P^T operand
-    static constexpr uint32_t OpHalf = NP * 128;                 // one 64-column half of it
-    // three K/V stages keep two tiles in flight behind the one being scored;
-    // the operand buffers give way when the query rows grow
-#ifndef DUO_BLK_WIDE_STAGES
-#define DUO_BLK_WIDE_STAGES 3
-#endif
-#ifndef DUO_BLK_WIDE_PB
-#define DUO_BLK_WIDE_PB 1
-#endif
-    static constexpr int Stages = NP <= 32 ? 3 : DUO_BLK_WIDE_STAGES;
-    static constexpr int QB = NP <= 32 ? 2 : 1;                  // Q buffers (next item's Q staged early)
-    static constexpr int PB = NP <= 16 ? 2 : NP <= 32 ? 1 : DUO_BLK_WIDE_PB;   // P^T buffers
-    static constexpr size_t Smem = 1024 + Stages * kDecStageBytes + (QB + PB) * OpBytes;
-    static_assert(Smem + 4096 <= 232448, "shared memory");
+    static constexpr int RQ = (NR + 3) / 4;                      // rows per TMEM lane quarter
+    static constexpr int Stages = 3;
+    static constexpr size_t Smem = 1024 + Stages * kDecStageBytes;
+    static_assert(Smem + 2048 <= 232448, "shared memory");
     static constexpr int PartFloats = NR * (kD + 2);             // m[NR], l[NR], acc[NR][D]
-    static constexpr uint32_t TmemCols = 3 * NP <= 64 ? 64 : 3 * NP <= 128 ? 128 : 256;
-    // softmax warps per TMEM lane quarter, each with NH of the query rows: more
-    // of them for wide blocks, so that no thread holds more than 16 rows
-    static constexpr int NPART = NP == 48 ? 3 : 2;
-    static constexpr int NH = NP / NPART;                        // 8 or 16 rows
-    static constexpr int RP = NH <= 4 ? 4 : NH <= 8 ? 8 : NH <= 16 ? 16 : 32;   // NH padded to 2^k
-    static constexpr int SoftmaxThreads = 128 * NPART;
-    // softmax warps 0 .. 4*NPART-1, then the producer warp and the MMA warp
-    static constexpr int Threads = SoftmaxThreads + 64;
+    static constexpr int Threads = 7 * 32;
 };
 
-__device__ __forceinline__ void blk_tmem_ld4(uint32_t taddr, uint32_t *r) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(taddr));
+// Query row r of an item <-> TMEM lane (quarter r / RQ, lane r % RQ).
+template <int kQ>
+__device__ __forceinline__ int blk_lane_of_row(int r) {
+    return (r / BlockCfg<kQ>::RQ) * 32 + r % BlockCfg<kQ>::RQ;
 }
-
-__device__ __forceinline__ void blk_tmem_st4(uint32_t taddr, const uint32_t *r) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
-                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
-                 : "memory");
-}
-
-__device__ __forceinline__ void blk_reg_fence4(uint32_t *r) {
-    asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]));
-}
-
-// Per-row reduction of v[RP] over the 32 lanes of a warp that leaves row
-// (lane >> (5 - log2 RP)) with each lane: at every step a lane keeps half of
-// its rows and hands the other half to its partner, so RP - 1 shuffles do the
-// work of RP * 5 butterflies.  op: 0 max, 1 sum.
-template <int RP, int OP>
-__device__ __forceinline__ float lane_row_reduce(float (&v)[RP], int lane) {
-    int cnt = RP;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        if (cnt >= 2) {
-            const bool up = (lane & o) != 0;
-#pragma unroll
-            for (int i = 0; i < RP / 2; ++i) {
-                if (i < cnt / 2) {
-                    const float keep = up ? v[cnt / 2 + i] : v[i];
-                    const float give = up ? v[i] : v[cnt / 2 + i];
-                    const float got = __shfl_xor_sync(0xffffffffu, give, o);
-                    v[i] = OP == 0 ? fmaxf(keep, got) : keep + got;
-                }
-            }
-            cnt >>= 1;
-        } else {
-            const float got = __shfl_xor_sync(0xffffffffu, v[0], o);
-            v[0] = OP == 0 ? fmaxf(v[0], got) : v[0] + got;
-        }
-    }
-    return v[0];
-}
-
-// OR of a predicate over the `nthreads` softmax threads (named barrier 1).
-__device__ __forceinline__ bool softmax_vote_any(bool v, int nthreads) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, 1, %2, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)v), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
-
-template <int RP>
-__host__ __device__ constexpr int rp_bits() { return RP == 4 ? 2 : RP == 8 ? 3 : RP == 16 ? 4 : 5; }
-
-template <int RP>
-__device__ __forceinline__ int lane_row(int lane) { return lane >> (5 - rp_bits<RP>()); }
 
 struct BlockArgs {
     DecodeArgs d;                   // cache maps, geometry, splits (d.q, d.out, d.lse unused)
@@ -159,15 +72,6 @@ struct BlockArgs {
     int32_t q_len, n_cache_items, part_slots;   // part_slots = the most splits of a head
     int32_t *work_counter;          // zeroed before the launch: items claimed so far
 };
-
-// Byte offset of element (row, k) in an [NP rows][128] bf16 K-major operand
-// stored as two 64-column halves with the 128-byte swizzle.
-template <int NP>
-__device__ __forceinline__ uint32_t blk_op_offset(int row, int k) {
-    const int half = k >> 6, kk = k & 63;
-    return half * (NP * 128) + (row >> 3) * 1024 + (row & 7) * 128 + ((((kk >> 3) ^ (row & 7))) << 4) +
-           (kk & 7) * 2;
-}
 
 struct BlockItem {
     Item it;                        // the cache item; n_tiles includes the block's tile
@@ -223,25 +127,20 @@ __device__ __forceinline__ void key_query_range(const BlockArgs &a, const BlockI
 template <int kQ>
 __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(const __grid_constant__ BlockArgs a) {
     using C = BlockCfg<kQ>;
-    constexpr int NR = C::NR, NP = C::NP, ST = C::Stages, NH = C::NH, RP = C::RP;
-    constexpr int NSM = C::SoftmaxThreads, NSW = NSM / 32;    // softmax threads / warps
-    constexpr int kProducer = NSW, kMma = NSW + 1;
+    constexpr int NR = C::NR, RQ = C::RQ, ST = C::Stages;
+    constexpr int kPrep = 4, kProducer = 5, kMma = 6;
     const DecodeArgs &d = a.d;
     extern __shared__ __align__(16) char bsmem_base[];
     char *smem = bsmem_base + ((1024u - (smem_u32(bsmem_base) & 1023u)) & 1023u);
     char *sKV = smem;                                         // [stages][K 32 KB | V 32 KB]
-    char *sQ = smem + ST * kDecStageBytes;                    // [2 items][OpBytes]
-    char *sP = sQ + C::QB * C::OpBytes;                       // [PB tiles][OpBytes]
-    __shared__ uint64_t kv_full[ST], kv_empty[ST];
-    // P^T is double-buffered: PV of tile j commits o_done[j & 1]
-    __shared__ uint64_t s_full[2], p_full, o_done[2], q_ready[2];
-    // items claimed by the producer, read by the MMA issuer and the softmax warps
+    __shared__ uint64_t kv_full[ST], kv_empty[ST], prep_full[ST];
+    __shared__ uint64_t s_full[2], p_full, o_done, q_ready[2], mma_drained;
+    // items claimed by the producer, read by the MMA issuer, the key preparation and the softmax warps
     constexpr int kSlots = 4;
     __shared__ uint64_t work_full[kSlots], work_empty[kSlots];
     __shared__ int work_slot[kSlots];
+    __shared__ __align__(16) uint32_t key_mask[ST][kQ][4];   // per stage and block token: keys it attends
     __shared__ uint32_t tmem_base;
-    __shared__ __align__(16) float red_max[2][4][NP];
-    __shared__ float red_sum[4][NP];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_items = a.n_cache_items;
@@ -249,28 +148,23 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         for (int i = 0; i < ST; ++i) {
             mbar_init(&kv_full[i], 1);
             mbar_init(&kv_empty[i], 1);
+            mbar_init(&prep_full[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&q_ready[i], NSW);
+            mbar_init(&q_ready[i], 4);
         }
-        mbar_init(&p_full, NSW);
-        mbar_init(&o_done[0], 1);
-        mbar_init(&o_done[1], 1);
+        mbar_init(&p_full, 4);
+        mbar_init(&o_done, 1);
+        mbar_init(&mma_drained, 1);
         for (int i = 0; i < kSlots; ++i) {
             mbar_init(&work_full[i], 1);
-            mbar_init(&work_empty[i], 1 + NSW);        // the MMA issuer and every softmax warp
+            mbar_init(&work_empty[i], 6);      // the MMA issuer, the key preparation, 4 softmax warps
         }
         fence_mbar_init();
     }
-    if (warp < NSW) {
-        // operand rows NR..NP-1 stay zero for the whole kernel
-        for (int i = threadIdx.x; i < (C::QB + C::PB) * (int)C::OpBytes / 16; i += NSM)
-            reinterpret_cast<uint4 *>(sQ)[i] = make_uint4(0, 0, 0, 0);
-        fence_proxy_async_smem();
-    }
     if (warp == kMma) {
-        tmem_alloc(&tmem_base, C::TmemCols);
+        tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
     __syncwarp();
@@ -278,6 +172,20 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    const uint32_t tm_s = tmem, tm_o = tmem + 256, tm_q = tmem + 384;
+    pdl_wait();
+
+    // Reads item slot icx (once per reading warp).
+    auto read_slot = [&](int icx, int *wout) -> bool {
+        const int sl = icx % kSlots;
+        const bool got = mbar_wait(&work_full[sl], (icx / kSlots) & 1);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got)) return false;
+        *wout = work_slot[sl];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&work_empty[sl]);
+        return true;
+    };
 
     if (warp == kProducer) {
         // ------------------------------------------------------------ producer
@@ -296,7 +204,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
             bool ok = true;
             int w = blockIdx.x;
             for (int ic = 0; ok; ++ic) {
-                // publish the item (an index >= n_items tells the consumers to stop)
+                // publish the item (an index >= n_items tells the others to stop)
                 const int sl = ic % kSlots;
                 if (ic >= kSlots && !(ok = mbar_wait(&work_empty[sl], ((ic / kSlots) - 1) & 1))) break;
                 work_slot[sl] = w;
@@ -336,287 +244,343 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
             }
         }
         __syncwarp();
+    } else if (warp == kPrep) {
+        // ------------------------------------------------------------ key preparation
+        int jg = 0, w = 0;
+        bool ok = true;
+        for (int ic = 0; ok; ++ic) {
+            if (!(ok = read_slot(ic, &w))) break;
+            if (w >= n_items) break;
+            const BlockItem bi = block_item_of(a, w);
+            for (int t = 0; t < bi.it.n_tiles; ++t, ++jg) {
+                const int st = jg % ST;
+                const bool got = mbar_wait(&kv_full[st], (jg / ST) & 1);
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                const bool block_tile = t == bi.cache_tiles;
+                char *vt = sKV + st * kDecStageBytes + kDecTileBytes;
+#pragma unroll
+                for (int grp = 0; grp < 4; ++grp) {
+                    const int k = grp * 32 + lane;         // key row of the tile
+                    const int32_t e = block_tile ? k : bi.it.e_begin + t * kTok + k;
+                    int t_lo, t_hi;
+                    key_query_range(a, bi, block_tile, e, &t_lo, &t_hi);
+                    if (t_lo > t_hi) {
+                        // a key no query keeps: its V row must not reach the PV product
+                        // (V is MN-major: row k is 128 bytes in each 64-column half)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            reinterpret_cast<uint4 *>(vt + k * 128)[i] = make_uint4(0, 0, 0, 0);
+                            reinterpret_cast<uint4 *>(vt + kDecHalfBytes + k * 128)[i] = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < kQ; ++q) {
+                        const uint32_t bits = __ballot_sync(0xffffffffu, q >= t_lo && q <= t_hi);
+                        if (lane == 0) key_mask[st][q][grp] = bits;
+                    }
+                }
+                fence_proxy_async_smem();       // the zeroed rows, for the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&prep_full[st]);
+            }
+        }
+        __syncwarp();
     } else if (warp == kMma) {
         // ------------------------------------------------------------ MMA issuer
+        // Two cursors walk the items' tiles in order: the QK cursor issues
+        // S = Q K^T up to two tiles ahead of the PV cursor, but only when its
+        // inputs are already there (a non-blocking check), so that it never holds
+        // up a PV the softmax warps wait for; the PV cursor polls for the
+        // softmax's P and the key preparation, issuing look-ahead products
+        // meanwhile.  Every poll is bounded.
         if (lane == 0) {
-            const uint32_t id_qk = idesc_bf16_f32(kTok, NP, 0, 0);
-            const uint32_t id_pv = idesc_bf16_f32(kD, NP, 1, 0);
-            const uint32_t kv_addr = smem_u32(sKV), q_addr = smem_u32(sQ), p_addr = smem_u32(sP);
-            const uint32_t o_tmem = tmem + 2 * NP;
-            auto issue_pv_blk = [&](int st, int pbuf, bool first) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(o_tmem, smem_desc_sw128(kv_addr + st * kDecStageBytes + kDecTileBytes + k * 2048,
-                                                   kDecHalfBytes, 1024),
-                           smem_desc_sw128(p_addr + (C::PB == 2 ? pbuf : 0) * C::OpBytes + (k >> 2) * C::OpHalf +
-                                               (k & 3) * 32,
-                                           16, 1024),
-                           id_pv, (first && k == 0) ? 0u : 1u);
-            };
-            int jg = 0, ic = 0;
-            bool ok = true, pend = false, pend_first = false;
-            int pend_st = 0;
-            for (; ok; ++ic) {
-                const int sl = ic % kSlots;
-                if (!(ok = mbar_wait(&work_full[sl], (ic / kSlots) & 1))) break;
+            const uint32_t id_qk = idesc_bf16_f32(128, kTok, 0, 0);
+            const uint32_t id_pv = idesc_bf16_f32(128, kD, 0, 1);
+            const uint32_t kv_addr = smem_u32(sKV);
+            constexpr int kInfo = 16;
+            int info_w[kInfo], info_n[kInfo];          // item by fetch order: work index, tiles
+            int fetched = 0;
+            int pi = 0;                                // the PV cursor's item
+            auto try_fetch = [&]() -> bool {
+                if (fetched - pi >= kInfo - 1) return false;
+                const int sl = fetched % kSlots;
+                if (!mbar_test(&work_full[sl], (fetched / kSlots) & 1)) return false;
                 const int w = work_slot[sl];
                 mbar_arrive(&work_empty[sl]);
-                if (w >= n_items) break;
-                const BlockItem bi = block_item_of(a, w);
-                const Item &it = bi.it;
-                // every item's Q is staged (an empty item's only signals), so the
-                // staging and this wait pair up item by item
-                if (!(ok = mbar_wait(&q_ready[ic & 1], (ic >> 1) & 1))) break;
-                if (it.n_tiles == 0) continue;
-                for (int t = 0; t < it.n_tiles && ok; ++t, ++jg) {
-                    const int st = jg % ST;
-                    if (!(ok = mbar_wait(&kv_full[st], (jg / ST) & 1))) break;
+                info_w[fetched % kInfo] = w;
+                info_n[fetched % kInfo] = w < n_items ? block_item_of(a, w).it.n_tiles : 0;
+                ++fetched;
+                return true;
+            };
+            int qi = 0, qt = 0, jq = 0, nq = 0;        // QK cursor: item, tile, products, non-empty items
+            bool q_end = false;
+            auto try_qk = [&]() -> bool {
+                while (!q_end) {
+                    if (qi == fetched && !try_fetch()) return false;
+                    if (info_w[qi % kInfo] >= n_items) {
+                        q_end = true;
+                        return false;
+                    }
+                    const int n = info_n[qi % kInfo];
+                    if (qt >= n) {
+                        if (n > 0) ++nq;
+                        ++qi;
+                        qt = 0;
+                        continue;
+                    }
+                    if (qt == 0 && !mbar_test(&q_ready[nq & 1], (nq >> 1) & 1)) return false;   // the item's Q
+                    const int st = jq % ST;
+                    if (!mbar_test(&kv_full[st], (jq / ST) & 1)) return false;
                     tc_fence_after();
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (k >> 2) * kDecHalfBytes + (k & 3) * 32;
-                        const uint32_t qoff = (C::QB == 2 ? (ic & 1) : 0) * C::OpBytes + (k >> 2) * C::OpHalf + (k & 3) * 32;
-                        mma_ss(tmem + (jg & 1) * NP, smem_desc_sw128(kv_addr + st * kDecStageBytes + off, 16, 1024),
-                               smem_desc_sw128(q_addr + qoff, 16, 1024), id_qk, k > 0);
-                    }
-                    mma_commit(&s_full[jg & 1]);
-                    if (pend) {
-                        if (!(ok = mbar_wait(&p_full, (jg - 1) & 1))) break;
-                        tc_fence_after();
-                        issue_pv_blk(pend_st, (jg - 1) & 1, pend_first);
-                        mma_commit(&o_done[(jg - 1) & 1]);
-                        mma_commit(&kv_empty[pend_st]);
-                    }
-                    pend = true;
-                    pend_st = st;
-                    pend_first = (t == 0);
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(tm_s + (jq & 1) * 128, tm_q + (nq & 1) * 64 + k * 8,
+                               smem_desc_sw128(kv_addr + st * kDecStageBytes + (k >> 2) * kDecHalfBytes +
+                                                   (k & 3) * 32, 16, 1024),
+                               id_qk, k > 0);
+                    mma_commit(&s_full[jq & 1]);
+                    ++jq;
+                    ++qt;
+                    return true;
                 }
-            }
-            if (ok && pend && mbar_wait(&p_full, (jg - 1) & 1)) {
+                return false;
+            };
+            int pt = 0, jp = 0;
+            bool ok = true;
+            unsigned long long t_last = clock64();
+            auto stalled = [&](bool progress) -> bool {
+                if (progress) {
+                    t_last = clock64();
+                    return false;
+                }
+                if (clock64() - t_last <= DUO_WAIT_CYCLES) return false;
+                record_status(-5 /* DUO_ERR_TIMEOUT */);
+                return true;
+            };
+            while (ok) {
+                // the PV cursor's next tile
+                bool done = false;
+                while (ok) {
+                    if (pi == fetched) {
+                        bool got = try_fetch();
+                        if (!got) got = try_qk();
+                        if (stalled(got)) ok = false;
+                        continue;
+                    }
+                    if (info_w[pi % kInfo] >= n_items) {
+                        done = true;
+                        break;
+                    }
+                    if (pt < info_n[pi % kInfo]) break;
+                    ++pi;
+                    pt = 0;
+                }
+                if (!ok || done) break;
+                const int st = jp % ST;
+                // wait for the softmax's P of tile jp and the tile's key preparation,
+                // issuing the look-ahead products as their inputs arrive
+                while (true) {
+                    bool progress = false;
+                    if (jq < jp + 3) progress = try_qk();
+                    if (jq > jp && mbar_test(&p_full, jp & 1) && mbar_test(&prep_full[st], (jp / ST) & 1)) break;
+                    if (stalled(progress)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!ok) break;
+                t_last = clock64();
                 tc_fence_after();
-                issue_pv_blk(pend_st, (jg - 1) & 1, pend_first);
-                mma_commit(&o_done[(jg - 1) & 1]);
-                mma_commit(&kv_empty[pend_st]);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tm_o, tm_s + (jp & 1) * 128 + k * 8,
+                           smem_desc_sw128(kv_addr + st * kDecStageBytes + kDecTileBytes + k * 2048,
+                                           kDecHalfBytes, 1024),
+                           id_pv, (pt == 0 && k == 0) ? 0u : 1u);
+                mma_commit(&o_done);
+                mma_commit(&kv_empty[st]);
+                ++jp;
+                ++pt;
             }
+            // every product issued has completed before the tensor memory is freed
+            // (on an early exit some may still run)
+            mma_commit(&mma_drained);
+            mbar_wait(&mma_drained, 0);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int quarter = warp & 3;                        // TMEM lane quarter: tokens / dims
-        const int part = warp >> 2;                          // query rows [part * NH, part * NH + NH)
-        const int r = quarter * 32 + lane;                   // token row / output dimension
-        const int q0 = part * NH;
+        const int quarter = warp;                            // TMEM lane quarter
+        const int r = quarter * RQ + lane;                   // query row of this thread
+        const bool has_row = lane < RQ && r < NR;
+        const int tq = has_row ? r / kGroup : 0;             // its block token
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t o_tmem = tmem + 2 * NP + q0 + lane_base;
         const float c = d.scale_log2;
-        const int tid = threadIdx.x;                         // 0 .. NSM - 1
-        auto sm_sync = [] { asm volatile("bar.sync 1, %0;" ::"r"(NSM) : "memory"); };
-        // Reads item slot icx (each softmax warp once per slot).
-        auto read_slot = [&](int icx, int *wout) -> bool {
-            const int sl = icx % kSlots;
-            const bool got = mbar_wait(&work_full[sl], (icx / kSlots) & 1);
+        // Stages the query rows of item wq into Q buffer buf (zeros in the padding rows).
+        auto stage_q = [&](int wq, int buf) {
+            uint32_t qv[64];
+            const bool real = has_row;
+            const uint4 *src = nullptr;
+            if (real) {
+                const BlockItem nx = block_item_of(a, wq);
+                src = reinterpret_cast<const uint4 *>(
+                    a.q + (((size_t)nx.it.b * kQ + tq) * d.hkv * kGroup + nx.it.g * kGroup + r % kGroup) * kD);
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint4 v = real ? src[i] : make_uint4(0, 0, 0, 0);
+                qv[4 * i] = v.x;
+                qv[4 * i + 1] = v.y;
+                qv[4 * i + 2] = v.z;
+                qv[4 * i + 3] = v.w;
+            }
+            tmem_st32(tm_q + buf * 64 + lane_base, *reinterpret_cast<uint32_t(*)[32]>(&qv[0]));
+            tmem_st32(tm_q + buf * 64 + 32 + lane_base, *reinterpret_cast<uint32_t(*)[32]>(&qv[32]));
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
-            if (!__all_sync(0xffffffffu, got)) return false;
-            *wout = work_slot[sl];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&work_empty[sl]);
-            return true;
+            if (lane == 0) mbar_arrive(&q_ready[buf]);
         };
-        // Stages the NR query rows of item w as the Q operand in buffer `buf`
-        // (nothing to copy for an empty item, but the MMA warp is still told).
-        auto stage_q = [&](int w, int buf) {
-            if (w >= n_items) return;
-            {
-                const BlockItem nx = block_item_of(a, w);
-                if (nx.it.n_tiles > 0)
-                for (int i = tid; i < NR * 16; i += NSM) {
-                    const int row = i >> 4, ch = i & 15;
-                    const int t = row / kGroup, h = row % kGroup;
-                    const uint4 v = reinterpret_cast<const uint4 *>(
-                        a.q + (((size_t)nx.it.b * kQ + t) * d.hkv * kGroup + nx.it.g * kGroup + h) * kD)[ch];
-                    *reinterpret_cast<uint4 *>(sQ + (C::QB == 2 ? buf : 0) * C::OpBytes + blk_op_offset<NP>(row, ch * 8)) = v;
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&q_ready[buf]);
+        // Q buffers alternate over the items that have tiles (an empty item needs
+        // no Q), in the order the MMA issuer counts them
+        int n_staged = 0;
+        auto stage_if_needed = [&](int wx) {
+            if (wx < n_items && block_item_of(a, wx).it.n_tiles > 0) {
+                stage_q(wx, n_staged & 1);
+                ++n_staged;
             }
         };
         int jg = 0, ic = 0, w = 0;
         bool ok = read_slot(0, &w);
-        if (ok) stage_q(w, 0);
+        if (ok) stage_if_needed(w);
         for (; ok && w < n_items; ++ic) {
             const BlockItem bi = block_item_of(a, w);
             const Item &it = bi.it;
-            float m_run[NH], l_part[NH];
-#pragma unroll
-            for (int q = 0; q < NH; ++q) {
-                m_run[q] = -INFINITY;
-                l_part[q] = 0.f;
-            }
+            // the next item's Q goes into the other buffer now (the item with
+            // tiles before this one, which used it, has had all its products read)
+            int w_next = n_items;
+            if (!(ok = read_slot(ic + 1, &w_next))) break;
+            stage_if_needed(w_next);
+            float m_run = -INFINITY, l_run = 0.f;
             for (int t = 0; t < it.n_tiles; ++t, ++jg) {
                 const bool got = mbar_wait(&s_full[jg & 1], (jg >> 1) & 1);
                 __syncwarp();
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sr[NH];
+                uint32_t sr[128];
 #pragma unroll
-                for (int cb = 0; cb < NH; cb += 4) blk_tmem_ld4(tmem + (jg & 1) * NP + q0 + cb + lane_base, &sr[cb]);
+                for (int q4 = 0; q4 < 4; ++q4)
+                    tmem_ld32(tm_s + (jg & 1) * 128 + q4 * 32 + lane_base,
+                              *reinterpret_cast<uint32_t(*)[32]>(&sr[q4 * 32]));
                 tmem_ld_wait();
 #pragma unroll
-                for (int cb = 0; cb < NH; cb += 4) blk_reg_fence4(&sr[cb]);
+                for (int q4 = 0; q4 < 4; ++q4) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[q4 * 32]));
                 const bool block_tile = t == bi.cache_tiles;
-                const int32_t e = block_tile ? r : it.e_begin + t * kTok + r;
-                int t_lo, t_hi;
-                key_query_range(a, bi, block_tile, e, &t_lo, &t_hi);
                 // a full head's tile inside the cached length: every key for every query
                 const bool dense = !block_tile && !it.ring && it.e_begin + (t + 1) * kTok <= it.e_end;
-                float s[NH];
-                bool exceed = false;
+                if (!dense) {
+                    const int st = jg % ST;
+                    const bool prepped = mbar_wait(&prep_full[st], (jg / ST) & 1);
+                    __syncwarp();
+                    if (!__all_sync(0xffffffffu, prepped)) { ok = false; break; }
+                    const uint4 mk = *reinterpret_cast<const uint4 *>(key_mask[st][tq]);
+                    const uint32_t mw[4] = {mk.x, mk.y, mk.z, mk.w};
 #pragma unroll
-                for (int q = 0; q < NH; ++q) {
-                    const int tq = (q0 + q) / kGroup;
-                    const bool keep = q0 + q < NR && (dense || (tq >= t_lo && tq <= t_hi));
-                    s[q] = keep ? __uint_as_float(sr[q]) : -INFINITY;
-                    exceed |= s[q] * c > m_run[q] + 8.f;
+                    for (int cc = 0; cc < 128; ++cc)
+                        if (!((mw[cc >> 5] >> (cc & 31)) & 1u)) sr[cc] = __float_as_uint(-INFINITY);
                 }
-                // The running max of a row moves only when some score exceeds it by
-                // more than 2^8.  One vote over the eight warps settles whether any
-                // row of this tile does; if none does, the tile's max is not needed
-                // and every row keeps its max (the same result as computing it).
-                if (softmax_vote_any(exceed, NSM)) {
-                    float mx[RP];
+                float mx8[8];
 #pragma unroll
-                    for (int q = 0; q < RP; ++q) mx[q] = q < NH ? s[q] : -INFINITY;
-                    const float mrow = lane_row_reduce<RP, 0>(mx, lane);
-                    if (lane == (lane_row<RP>(lane) << (5 - rp_bits<RP>())) && lane_row<RP>(lane) < NH)
-                        red_max[jg & 1][quarter][q0 + lane_row<RP>(lane)] = mrow;
-                    sm_sync();
-                    float alpha[NH];
-                    bool rescale = false;
+                for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
 #pragma unroll
-                    for (int q = 0; q < NH; q += 4) {
-                        float4 v4[4];
+                for (int cc = 8; cc < 128; cc += 16)
 #pragma unroll
-                        for (int w4 = 0; w4 < 4; ++w4)
-                            v4[w4] = *reinterpret_cast<const float4 *>(&red_max[jg & 1][w4][q0 + q]);
-                        const float mj[4] = {fmaxf(fmaxf(v4[0].x, v4[1].x), fmaxf(v4[2].x, v4[3].x)),
-                                             fmaxf(fmaxf(v4[0].y, v4[1].y), fmaxf(v4[2].y, v4[3].y)),
-                                             fmaxf(fmaxf(v4[0].z, v4[1].z), fmaxf(v4[2].z, v4[3].z)),
-                                             fmaxf(fmaxf(v4[0].w, v4[1].w), fmaxf(v4[2].w, v4[3].w))};
+                    for (int e = 0; e < 8; ++e)
+                        mx8[e] = fmax3(mx8[e], __uint_as_float(sr[cc + e]), __uint_as_float(sr[cc + 8 + e]));
+                const float m_tile = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                           fmaxf(mx8[6], mx8[7])) * c;
+                // keep the stale max unless the new one is more than 2^8 larger
+                float m_use = m_run, alpha = 1.f;
+                if (m_tile > m_run + 8.f) {
+                    m_use = m_tile;
+                    alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_tile);
+                }
+                const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+                const f2 c2 = f2_splat(c), ms2 = f2_splat(-m_sub);
+                f2 ls0 = f2_splat(0.f), ls1 = f2_splat(0.f);
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const float m_tile = mj[u] * c;
-                            alpha[q + u] = 1.f;
-                            if (m_tile > m_run[q + u] + 8.f) {
-                                alpha[q + u] = (m_run[q + u] == -INFINITY) ? 0.f : ex2_approx(m_run[q + u] - m_tile);
-                                m_run[q + u] = m_tile;
-                                l_part[q + u] *= alpha[q + u];
-                                rescale = true;
-                            }
-                        }
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t pw[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int cc = ch * 16 + 2 * e;
+                        const f2 x = f2_fma(f2_make(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), c2, ms2);
+                        // rounded to bf16: the PV product and the row sum use the same weights
+                        const uint32_t wv = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
+                        pw[e] = wv;
+                        if (e & 1) ls1 = f2_add(ls1, f2_make(bf16lo(wv), bf16hi(wv)));
+                        else ls0 = f2_add(ls0, f2_make(bf16lo(wv), bf16hi(wv)));
                     }
-                    if (t > 0 && __any_sync(0xffffffffu, rescale)) {
-                        // O^T must hold every earlier tile's product before it is scaled
-                        const bool prev = mbar_wait(&o_done[(jg - 1) & 1], ((jg - 1) >> 1) & 1);
-                        __syncwarp();
-                        if (!__all_sync(0xffffffffu, prev)) { ok = false; break; }
-                        tc_fence_after();
-#pragma unroll
-                        for (int cb = 0; cb < NH; cb += 4) {
-                            uint32_t orr[4];
-                            blk_tmem_ld4(o_tmem + cb, orr);
-                            tmem_ld_wait();
-                            blk_reg_fence4(orr);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * alpha[cb + q]);
-                            blk_tmem_st4(o_tmem + cb, orr);
-                        }
-                        tmem_st_wait();
-                    }
+                    // P of keys [16 ch, 16 ch + 16) -> TMEM columns [8 ch, 8 ch + 8) of this S buffer
+                    tmem_st8(tm_s + (jg & 1) * 128 + ch * 8 + lane_base, pw);
                 }
-                float p[NH];
-#pragma unroll
-                for (int q = 0; q < NH; ++q) {
-                    // rounded to bf16 here: the PV product and the row sum use the same weights
-                    p[q] = __bfloat162float(__float2bfloat16_rn(
-                        ex2_approx(fmaf(s[q], c, m_run[q] == -INFINITY ? 0.f : -m_run[q]))));
-                    l_part[q] += p[q];
-                }
-                // the P^T buffer was last read by the PV of tile jg - PB
-                if (jg >= C::PB) {
-                    const int pj = jg - C::PB;
-                    const bool prev = mbar_wait(&o_done[pj & 1], (pj >> 1) & 1);
+                l_run = l_run * alpha + ((ls0.x + ls0.y) + (ls1.x + ls1.y));
+                m_run = m_use;
+                if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    // O must hold every earlier tile's product before it is scaled
+                    const bool prev = mbar_wait(&o_done, (jg - 1) & 1);
                     __syncwarp();
                     if (!__all_sync(0xffffffffu, prev)) { ok = false; break; }
                     tc_fence_after();
-                }
-                if (t_lo > t_hi && part == 0) {
-                    // a key no query keeps: its V row must not reach the PV product
-                    char *vrow = sKV + (jg % ST) * kDecStageBytes + kDecTileBytes + r * 128;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        reinterpret_cast<uint4 *>(vrow)[i] = make_uint4(0, 0, 0, 0);
-                        reinterpret_cast<uint4 *>(vrow + kDecHalfBytes)[i] = make_uint4(0, 0, 0, 0);
+                    for (int cb = 0; cb < 128; cb += 32) {
+                        uint32_t orr[32];
+                        tmem_ld32(tm_o + cb + lane_base, orr);
+                        tmem_ld_wait();
+                        reg_fence32(orr);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                        tmem_st32(tm_o + cb + lane_base, orr);
                     }
                 }
-#pragma unroll
-                for (int q = 0; q < NH; ++q)
-                    if (q0 + q < NR)
-                        *reinterpret_cast<__nv_bfloat16 *>(sP + (C::PB == 2 ? (jg & 1) : 0) * C::OpBytes +
-                                                           blk_op_offset<NP>(q0 + q, r)) =
-                            __float2bfloat16_rn(p[q]);
-                fence_proxy_async_smem();
+                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full);
             }
             if (!ok) break;
-            // the next item: its Q may be staged now (this item's S products are all read)
-            int w_next = n_items;
-            if (!(ok = read_slot(ic + 1, &w_next))) break;
-            stage_q(w_next, (ic + 1) & 1);
             // ------------------------------------------------------------ item epilogue
-            float acc[NH];
-#pragma unroll
-            for (int q = 0; q < NH; ++q) acc[q] = 0.f;
+            float *part = d.part + (((size_t)it.b * d.hkv + it.g) * a.part_slots + it.split) * C::PartFloats;
             if (it.n_tiles > 0) {
-                const bool done = mbar_wait(&o_done[(jg - 1) & 1], ((jg - 1) >> 1) & 1);
+                const bool done = mbar_wait(&o_done, (jg - 1) & 1);
                 __syncwarp();
                 if (!__all_sync(0xffffffffu, done)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
-                for (int cb = 0; cb < NH; cb += 4) {
-                    uint32_t orr[4];
-                    blk_tmem_ld4(o_tmem + cb, orr);
+                for (int cb = 0; cb < 128; cb += 32) {
+                    uint32_t orr[32];
+                    tmem_ld32(tm_o + cb + lane_base, orr);
                     tmem_ld_wait();
-                    blk_reg_fence4(orr);
+                    reg_fence32(orr);
+                    if (has_row) {
+                        float4 *dst = reinterpret_cast<float4 *>(part + 2 * NR + r * kD + cb);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[cb + q] = __uint_as_float(orr[q]);
+                        for (int e = 0; e < 32; e += 4)
+                            dst[e / 4] = make_float4(__uint_as_float(orr[e]), __uint_as_float(orr[e + 1]),
+                                                     __uint_as_float(orr[e + 2]), __uint_as_float(orr[e + 3]));
+                    }
                 }
+            } else if (has_row) {
+                float4 *dst = reinterpret_cast<float4 *>(part + 2 * NR + r * kD);
+                for (int e = 0; e < kD / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            // l: this warp's 32 tokens per row, then the four quarters in a fixed order
-            float lsum[RP];
-#pragma unroll
-            for (int q = 0; q < RP; ++q) lsum[q] = q < NH ? l_part[q] : 0.f;
-            const float lrow = lane_row_reduce<RP, 1>(lsum, lane);
-            const int my_row = lane_row<RP>(lane);
-            const bool row_writer = lane == (my_row << (5 - rp_bits<RP>()));
-            if (row_writer && my_row < NH) red_sum[quarter][q0 + my_row] = lrow;
-            sm_sync();
-            float *part = d.part + (((size_t)it.b * d.hkv + it.g) * a.part_slots + it.split) * C::PartFloats;
-#pragma unroll
-            for (int q = 0; q < NH; ++q)
-                if (q0 + q < NR) part[2 * NR + (q0 + q) * kD + r] = acc[q];
-            if (quarter == 0 && row_writer && my_row < NH && q0 + my_row < NR) {
-                const int q = q0 + my_row;
-                float mq = -INFINITY;
-#pragma unroll
-                for (int i = 0; i < NH; ++i)
-                    if (i == my_row) mq = m_run[i];
-                part[q] = mq;
-                part[NR + q] = (red_sum[0][q] + red_sum[1][q]) + (red_sum[2][q] + red_sum[3][q]);
+            if (has_row) {
+                part[r] = m_run;
+                part[NR + r] = l_run;
             }
-            sm_sync();
+            // O is read before this warp's first p_full arrival of the next item
+            tc_fence_before();
             w = w_next;
         }
         __syncwarp();
@@ -626,7 +590,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (warp == kMma) {
         tc_fence_after();
-        tmem_dealloc(tmem, C::TmemCols);
+        tmem_dealloc(tmem, 512);
     }
 }
 

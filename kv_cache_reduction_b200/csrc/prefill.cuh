@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     char *sKV = smem + 2 * kQTileBytes;                // [stages][K 32 KB | V 32 KB]
     char *sO = sKV + kPfStages * kPfStageBytes;        // [softmax warp][2][32 rows][16 columns] bf16
     __shared__ uint64_t q_full, q_empty, kv_full[kPfStages], kv_empty[kPfStages];
-    __shared__ uint64_t s_full[2], p_full[2], o_done[2];
+    __shared__ uint64_t s_full[2], p_full[2], o_done[2], mma_drained;
     // work tiles claimed by the producer, read by the MMA issuer and the softmax warps
     __shared__ uint64_t work_full[kPfSlots], work_empty[kPfSlots];
     __shared__ int work_slot[kPfSlots];
@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             mbar_init(&work_full[sl], 1);
             mbar_init(&work_empty[sl], 9);      // the MMA issuer and the 8 softmax warps
         }
+        mbar_init(&mma_drained, 1);
         fence_mbar_init();
     }
     if (warp == kPfMmaWarp) {
@@ -325,6 +326,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 n_kv = n_kv_next;
                 ++wc;
             }
+            // every product issued has completed before the tensor memory is freed
+            // (on an early exit some may still run)
+            mma_commit(&mma_drained);
+            mbar_wait(&mma_drained, 0);
         }
         __syncwarp();  // lanes 1..31 wait for the MMA lane before the CTA barrier
     } else {

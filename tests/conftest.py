@@ -19,3 +19,12 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_sessionstart(session):
+    # DUO_TEST_LIBRARY runs the GPU tests against another build of the library
+    # (a variant under study); by default the in-tree libduoattn.so is used
+    path = os.environ.get("DUO_TEST_LIBRARY")
+    if path:
+        import kv_cache_reduction_b200 as duo
+        duo.load_library(path)

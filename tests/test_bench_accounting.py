@@ -173,3 +173,25 @@ def test_decode_cpu_baseline_leg_runs_on_host_tensors():
     used = int(r["sample"].split()[0])
     assert used >= 1
     assert r["threads_busy"] == min(r["cores"], 2 * 2 * 6)
+
+
+def test_decode_small_cpu_baseline_leg_runs_on_host_tensors():
+    """The config-1 line's CPU leg on small host tensors: the oracle's prefill
+    of the prompt, then append + decode steps, timed per step."""
+    import torch
+    import kv_cache_reduction_b200 as duo
+
+    wl = object.__new__(bench.DecodeSmall)
+    wl.STEPS = 3
+    L = 40
+    wl.params = duo.DuoParams(1, full_mask=(1, 0, 0, 1, 0, 1, 1, 0))
+    wl.cap = L + wl.STEPS
+    wl.qp = inputs.randn_bf16((1, L, 48, 128), 70, "cpu")
+    wl.kp = inputs.randn_bf16((1, L, 8, 128), 71, "cpu")
+    wl.vp = inputs.randn_bf16((1, L, 8, 128), 72, "cpu")
+    wl.k1 = inputs.randn_bf16((wl.STEPS, 1, 1, 8, 128), 73, "cpu")
+    wl.v1 = inputs.randn_bf16((wl.STEPS, 1, 1, 8, 128), 74, "cpu")
+    wl.q1 = inputs.randn_bf16((wl.STEPS, 1, 48, 128), 75, "cpu")
+    r = wl.oracle_sample(0.05)
+    assert r["kind"] == "oracle" and r["unit"] == "us/step" and r["value"] > 0 and r["prefill_us"] > 0
+    assert r["sample"].split()[0].isdigit()
