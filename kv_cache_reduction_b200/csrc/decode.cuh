@@ -378,8 +378,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
                 float p[kGroup];
 #pragma unroll
                 for (int h = 0; h < kGroup; ++h) {
-                    // rounded to bf16 here: the PV product and the row sum use the same weights
-                    p[h] = __bfloat162float(__float2bfloat16_rn(ex2_approx(fmaf(s[h], c, -m_sub[h]))));
+                    p[h] = ex2_approx(fmaf(s[h], c, -m_sub[h]));
                     l_part[h] = fmaf(l_part[h], alpha[h], p[h]);
                 }
                 // the previous PV must be done with P^T and with O^T

@@ -26,8 +26,8 @@
 // its 128 scores of a key tile:
 //   S[128 x 128 keys] = Q . K_tile^T     (Q in tensor memory, K from shared)
 //   O[128 x 128 d]   += P . V_tile       (P over S in tensor memory)
-// with the rows past NR padding.  Two S buffers let the product of tile j + 2
-// (and j + 1) run while the softmax works on tile j.
+// with the rows past NR padding.  Two S buffers let the product of tile j + 1
+// run while the softmax works on tile j.
 //   warps 0-3  softmax and epilogue: stage the next item's Q into tensor
 //              memory, read S, mask, exponentials, P back over S, the item's
 //              partial (O, running max, sum) to the workspace
@@ -134,7 +134,10 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
     char *smem = bsmem_base + ((1024u - (smem_u32(bsmem_base) & 1023u)) & 1023u);
     char *sKV = smem;                                         // [stages][K 32 KB | V 32 KB]
     __shared__ uint64_t kv_full[ST], kv_empty[ST], prep_full[ST];
-    __shared__ uint64_t s_full[2], p_full, o_done, q_ready[2], mma_drained;
+    // s_full and p_full alternate with the tile parity, like the S buffers, so
+    // that the softmax finishing two tiles before the issuer looks cannot
+    // complete two phases of one barrier
+    __shared__ uint64_t s_full[2], p_full[2], o_done, q_ready[2], mma_drained;
     // items claimed by the producer, read by the MMA issuer, the key preparation and the softmax warps
     constexpr int kSlots = 4;
     __shared__ uint64_t work_full[kSlots], work_empty[kSlots];
@@ -153,8 +156,8 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&q_ready[i], 4);
+            mbar_init(&p_full[i], 4);
         }
-        mbar_init(&p_full, 4);
         mbar_init(&o_done, 1);
         mbar_init(&mma_drained, 1);
         for (int i = 0; i < kSlots; ++i) {
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
     } else if (warp == kMma) {
         // ------------------------------------------------------------ MMA issuer
         // Two cursors walk the items' tiles in order: the QK cursor issues
-        // S = Q K^T up to two tiles ahead of the PV cursor, but only when its
+        // S = Q K^T up to one tile ahead of the PV cursor, but only when its
         // inputs are already there (a non-blocking check), so that it never holds
         // up a PV the softmax warps wait for; the PV cursor polls for the
         // softmax's P and the key preparation, issuing look-ahead products
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 while (ok) {
                     if (pi == fetched) {
                         bool got = try_fetch();
-                        if (!got) got = try_qk();
+                        if (!got && jq < jp + 2) got = try_qk();
                         if (stalled(got)) ok = false;
                         continue;
                     }
@@ -380,10 +383,13 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 const int st = jp % ST;
                 // wait for the softmax's P of tile jp and the tile's key preparation,
                 // issuing the look-ahead products as their inputs arrive
+                // (S of tile jp + 2 would overwrite P of tile jp: at most one tile ahead)
                 while (true) {
                     bool progress = false;
-                    if (jq < jp + 3) progress = try_qk();
-                    if (jq > jp && mbar_test(&p_full, jp & 1) && mbar_test(&prep_full[st], (jp / ST) & 1)) break;
+                    if (jq < jp + 2) progress = try_qk();
+                    if (jq > jp && mbar_test(&p_full[jp & 1], (jp >> 1) & 1) &&
+                        mbar_test(&prep_full[st], (jp / ST) & 1))
+                        break;
                     if (stalled(progress)) {
                         ok = false;
                         break;
@@ -516,11 +522,10 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                     for (int e = 0; e < 8; ++e) {
                         const int cc = ch * 16 + 2 * e;
                         const f2 x = f2_fma(f2_make(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), c2, ms2);
-                        // rounded to bf16: the PV product and the row sum use the same weights
-                        const uint32_t wv = pack_bf16x2(ex2_approx(x.x), ex2_approx(x.y));
-                        pw[e] = wv;
-                        if (e & 1) ls1 = f2_add(ls1, f2_make(bf16lo(wv), bf16hi(wv)));
-                        else ls0 = f2_add(ls0, f2_make(bf16lo(wv), bf16hi(wv)));
+                        const f2 pe = f2_make(ex2_approx(x.x), ex2_approx(x.y));
+                        pw[e] = pack_bf16x2(pe.x, pe.y);     // bf16 for the PV product
+                        if (e & 1) ls1 = f2_add(ls1, pe);
+                        else ls0 = f2_add(ls0, pe);
                     }
                     // P of keys [16 ch, 16 ch + 16) -> TMEM columns [8 ch, 8 ch + 8) of this S buffer
                     tmem_st8(tm_s + (jg & 1) * 128 + ch * 8 + lane_base, pw);
@@ -547,7 +552,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full);
+                if (lane == 0) mbar_arrive(&p_full[jg & 1]);
             }
             if (!ok) break;
             // ------------------------------------------------------------ item epilogue

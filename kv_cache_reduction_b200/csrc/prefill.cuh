@@ -47,8 +47,16 @@ namespace duo {
 
 constexpr int kPfM = 128;                  // query rows per tile
 constexpr int kPfN = 128;                  // keys per tile
-constexpr int kPfThreads = 320;            // 10 warps
-constexpr int kPfProducerWarp = 8, kPfMmaWarp = 9;
+constexpr int kPfThreads = 512;            // 16 warps
+constexpr int kPfEpiWarp0 = 8, kPfProducerWarp = 12, kPfMmaWarp = 13;   // warps 14, 15 only balance the split
+// Register split (setmaxnreg): the block launches with 128 registers per thread;
+// the 8 softmax warps take 192, the 4 epilogue warps keep 80, the producer, the
+// MMA issuer and the two spare warps 48: 8*32*192 + 4*32*80 + 4*32*48 = 512*128,
+// and each SM sub-partition (warps k, k+4, k+8, k+12) holds 192+192+80+48 = 512
+// registers per lane, its whole register file.
+constexpr int kPfLaunchRegs = 128, kPfSoftmaxRegs = 192, kPfEpiRegs = 80, kPfOtherRegs = 48;
+static_assert(8 * 32 * kPfSoftmaxRegs + 4 * 32 * kPfEpiRegs + 4 * 32 * kPfOtherRegs == kPfThreads * kPfLaunchRegs,
+              "register split");
 // Pairs of each 16-pair chunk of a row whose exponentials run on the FMA pipe
 // (ex2_poly2) instead of the MUFU units.
 #ifndef DUO_PF_POLY_PAIRS
@@ -64,7 +72,7 @@ constexpr uint32_t kKVHalfBytes = kKVTileBytes / 2;
 constexpr uint32_t kPfStageBytes = 2 * kKVTileBytes;
 constexpr uint32_t kOStageBytes = 32 * 16 * 2;    // one O chunk of a softmax warp: 32 rows x 16 columns
 // each softmax warp stages its O chunks in two alternating buffers
-constexpr size_t kPfSmem = 1024 + 2 * kQTileBytes + kPfStages * kPfStageBytes + 8 * 2 * kOStageBytes;
+constexpr size_t kPfSmem = 1024 + 2 * kQTileBytes + kPfStages * kPfStageBytes + 4 * 2 * kOStageBytes;
 
 enum : int { kKindFull = 0, kKindStreaming = 1, kKindSliding = 2 };
 
@@ -150,9 +158,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     char *smem = psmem_base + ((1024u - (smem_u32(psmem_base) & 1023u)) & 1023u);
     char *sQ = smem;                                   // [2 heads][32 KB]
     char *sKV = smem + 2 * kQTileBytes;                // [stages][K 32 KB | V 32 KB]
-    char *sO = sKV + kPfStages * kPfStageBytes;        // [softmax warp][2][32 rows][16 columns] bf16
+    char *sO = sKV + kPfStages * kPfStageBytes;        // [epilogue warp][2][32 rows][16 columns] bf16
     __shared__ uint64_t q_full, q_empty, kv_full[kPfStages], kv_empty[kPfStages];
     __shared__ uint64_t s_full[2], p_full[2], o_done[2], mma_drained;
+    // a work tile's rows handed from the softmax to the epilogue warps: (running
+    // max, sum) per row, double-buffered by work tile; O of a head is free again
+    // once the epilogue has read it
+    __shared__ uint64_t ml_full[2], o_free[2];
+    __shared__ float4 row_ml[2][2][kPfM];             // [work tile parity][head][row]: m, l, l exact
     // work tiles claimed by the producer, read by the MMA issuer and the softmax warps
     __shared__ uint64_t work_full[kPfSlots], work_empty[kPfSlots];
     __shared__ int work_slot[kPfSlots];
@@ -170,10 +183,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             mbar_init(&s_full[h], 1);
             mbar_init(&p_full[h], 4);           // the head's four softmax warps
             mbar_init(&o_done[h], 1);
+            mbar_init(&ml_full[h], 4);
+            mbar_init(&o_free[h], 4);           // the four epilogue warps
         }
         for (int sl = 0; sl < kPfSlots; ++sl) {
             mbar_init(&work_full[sl], 1);
-            mbar_init(&work_empty[sl], 9);      // the MMA issuer and the 8 softmax warps
+            mbar_init(&work_empty[sl], 13);     // the MMA issuer, 8 softmax and 4 epilogue warps
         }
         mbar_init(&mma_drained, 1);
         fence_mbar_init();
@@ -187,8 +202,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
-
+    // each role sets its register budget first thing in its own branch, so that
+    // the compiler allocates that branch's code within it
     if (warp == kPfProducerWarp) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfOtherRegs));
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&a.tm_q);
@@ -240,6 +257,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         }
         __syncwarp();  // lanes 1..31 wait for the producer lane before the CTA barrier
     } else if (warp == kPfMmaWarp) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfOtherRegs));
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(kPfM, kPfN, 0, 0);
@@ -305,6 +323,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     const bool more = !last || w_next < a.n_work;
                     for (int h = 0; h < 2 && ok; ++h) {
                         if (!(ok = mbar_wait(&p_full[h], jg & 1))) break;
+                        // the first PV of a work tile overwrites O: the epilogue of the
+                        // previous one must have read it
+                        if (j == 0 && wc > 0 && !(ok = mbar_wait(&o_free[h], (wc - 1) & 1))) break;
                         tc_fence_after();
                         issue_pv(h, st, j == 0);
                         if (more) {
@@ -332,8 +353,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             mbar_wait(&mma_drained, 0);
         }
         __syncwarp();  // lanes 1..31 wait for the MMA lane before the CTA barrier
-    } else {
-        // ------------------------------------------------------------ softmax + epilogue
+    } else if (warp < 8) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPfSoftmaxRegs));
+        // ------------------------------------------------------------ softmax
         const int h = warp >> 2;                       // head of the pair
         const int quarter = warp & 3;                  // TMEM lane quarter of this warp
         const int r = quarter * 32 + lane;             // query row within the tile
@@ -358,11 +380,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             const int n_kv = tl.count();
             const int i = wk.t * kPfM + r;             // query position
             const int hq = wk.h0 + h;
-            // running max (log2 units) and sum; a sink logit starts them at (sigma, 1)
-            float m_run = -INFINITY, l_run = 0.f;
+            // running max (log2 units) and two sums: of the bf16 weights the PV
+            // product uses (it normalises O) and of the unrounded ones (the
+            // log-sum-exp); a sink logit starts them at (sigma, 1, 1)
+            float m_run = -INFINITY, l_run = 0.f, l_exact = 0.f;
             if (a.sink_logit != nullptr) {
                 m_run = a.sink_logit[hq] * kLog2eF;
                 l_run = 1.f;
+                l_exact = 1.f;
             }
             for (int j = 0; j < n_kv; ++j, ++jg) {
                 const bool got = mbar_wait(&s_full[h], jg & 1);
@@ -423,7 +448,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 // instruction; the row sum adds the bf16 weights the PV product
                 // uses, so that numerator and denominator agree
                 const f2 c2 = f2_splat(c), ms2 = f2_splat(-m_sub);
-                f2 ls0 = f2_splat(0.f), ls1 = f2_splat(0.f);
+                f2 ls0 = f2_splat(0.f), ls1 = f2_splat(0.f), lx0 = f2_splat(0.f), lx1 = f2_splat(0.f);
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
                     uint32_t pw[8];
@@ -440,13 +465,19 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                         }
                         const uint32_t wv = pack_bf16x2(pe.x, pe.y);
                         pw[e] = wv;
-                        if (e & 1) ls1 = f2_add(ls1, f2_make(bf16lo(wv), bf16hi(wv)));
-                        else ls0 = f2_add(ls0, f2_make(bf16lo(wv), bf16hi(wv)));
+                        if (e & 1) {
+                            ls1 = f2_add(ls1, f2_make(bf16lo(wv), bf16hi(wv)));
+                            lx1 = f2_add(lx1, pe);
+                        } else {
+                            ls0 = f2_add(ls0, f2_make(bf16lo(wv), bf16hi(wv)));
+                            lx0 = f2_add(lx0, pe);
+                        }
                     }
                     // P of keys [16 ch, 16 ch + 16) -> TMEM columns [8 ch, 8 ch + 8)
                     tmem_st8(s_tmem + ch * 8, pw);
                 }
                 l_run = l_run * alpha + ((ls0.x + ls0.y) + (ls1.x + ls1.y));
+                l_exact = l_exact * alpha + ((lx0.x + lx0.y) + (lx1.x + lx1.y));
                 m_run = m_use;
                 // O holds the previous key tiles' sum (its PV is complete: this S
                 // was computed after it); rescale the row when the max moved
@@ -468,59 +499,83 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 if (lane == 0) mbar_arrive(&p_full[h]);
             }
             if (!ok) break;
-            // ------------------------------------------------------------ work-tile epilogue
-            // the output gate of this row's channels (16 at a time, one chunk
-            // ahead) or of its head; the first loads overlap the wait below
-            const uint4 *gp = reinterpret_cast<const uint4 *>(
-                a.gate + (((size_t)wk.b * a.L + i) * a.hq + hq) * 128);
-            uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
-            float g_head = 0.f;
-            if (kGate == 1 && i < a.L) {
-                g0 = __ldg(gp);
-                g1 = __ldg(gp + 1);
-            } else if (kGate == 2 && i < a.L) {
-                g_head = __bfloat162float(a.gate[((size_t)wk.b * a.L + i) * a.hq + hq]);
-            }
-            const bool o_fin = mbar_wait(&o_done[h], (jg - 1) & 1);
+            // hand the row's (max, sum) to the epilogue warps and go on with the
+            // next work tile; they read O once its last PV is done
+            row_ml[wc & 1][h][r] = make_float4(m_run, l_run, l_exact, 0.f);
             __syncwarp();
-            if (!__all_sync(0xffffffffu, o_fin)) { ok = false; break; }
-            tc_fence_after();
-            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-            // o * sigmoid(g): one factor per row, or one per channel below
-            const float row_mul = kGate == 2 ? inv_l / (1.f + ex2_approx(-g_head * kLog2eF)) : inv_l;
-            // O / l leaves through this warp's two 1 KB staging buffers as 32-row x
-            // 16-column TMA stores (rows past L are clipped by the tensor map):
-            // coalesced by the copy engine instead of 32 scattered rows per store
+            if (lane == 0) mbar_arrive(&ml_full[h]);
+        }
+        __syncwarp();
+    } else if (warp >= kPfEpiWarp0 && warp < kPfEpiWarp0 + 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfEpiRegs));
+        // ------------------------------------------------------------ work-tile epilogue
+        const int quarter = warp & 3;                  // TMEM lane quarter of this warp
+        const int r = quarter * 32 + lane;             // query row within the tile
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        int jg = 0;
+        bool ok = true;
+        for (int wc = 0; ok; ++wc) {
+            const int sl = wc % kPfSlots;
+            const bool have = mbar_wait(&work_full[sl], (wc / kPfSlots) & 1);
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, have)) { ok = false; break; }
+            const int w = work_slot[sl];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&work_empty[sl]);
+            if (w >= a.n_work) break;
+            const PfWork wk = work_of(a, w);
+            jg += tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window).count();
+            const int i = wk.t * kPfM + r;             // query position
             const int row0 = wk.t * kPfM + quarter * 32;   // first row of this warp's boxes
-#pragma unroll
-            for (int cb = 0; cb < 128 && row0 < a.L; cb += 32) {
-                uint32_t orr[32];
-                tmem_ld32(o_tmem + cb, orr);
-                tmem_ld_wait();
-                reg_fence32(orr);
-#pragma unroll
-                for (int c16 = 0; c16 < 32; c16 += 16) {
-                    const int chunk = (cb + c16) / 16;     // 0..7
+            for (int h = 0; h < 2 && ok; ++h) {
+                const int hq = wk.h0 + h;
+                const uint32_t o_tmem = tmem + 256 + h * 128 + lane_base;
+                // the output gate of this row's channels (16 at a time, one chunk
+                // ahead) or of its head; the first loads overlap the waits below
+                const uint4 *gp = reinterpret_cast<const uint4 *>(
+                    a.gate + (((size_t)wk.b * a.L + i) * a.hq + hq) * 128);
+                uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0;
+                float g_head = 0.f;
+                if (kGate == 1 && i < a.L) {
+                    g0 = __ldg(gp);
+                    g1 = __ldg(gp + 1);
+                } else if (kGate == 2 && i < a.L) {
+                    g_head = __bfloat162float(a.gate[((size_t)wk.b * a.L + i) * a.hq + hq]);
+                }
+                const bool ready = mbar_wait(&ml_full[h], wc & 1) && mbar_wait(&o_done[h], (jg - 1) & 1);
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
+                tc_fence_after();
+                const float4 ml = row_ml[wc & 1][h][r];
+                const float m_run = ml.x, l_run = ml.y, l_exact = ml.z;
+                const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+                // o * sigmoid(g): one factor per row, or one per channel below
+                const float row_mul = kGate == 2 ? inv_l / (1.f + ex2_approx(-g_head * kLog2eF)) : inv_l;
+                // O / l leaves through this warp's two 1 KB staging buffers as 32-row x
+                // 16-column TMA stores (rows past L are clipped by the tensor map)
+                for (int chunk = 0; chunk < 8 && row0 < a.L; ++chunk) {
+                    uint32_t orr[16];
+                    tmem_ld16(o_tmem + chunk * 16, orr);
+                    tmem_ld_wait();
+                    reg_fence16(orr);
                     uint4 n0 = g0, n1 = g1;                // the next chunk's gates
                     if (kGate == 1 && chunk + 1 < 8 && i < a.L) {
                         n0 = __ldg(gp + 2 * (chunk + 1));
                         n1 = __ldg(gp + 2 * (chunk + 1) + 1);
                     }
-                    char *stage = sO + (warp * 2 + (chunk & 1)) * kOStageBytes;
+                    char *stage = sO + ((warp - kPfEpiWarp0) * 2 + (chunk & 1)) * kOStageBytes;
                     // the store that last used this buffer (two chunks ago) has read it
                     if (lane == 0) bulk_wait_read_1();
                     __syncwarp();
                     auto nb = [&](int e) {
                         float m0 = row_mul, m1 = row_mul;
                         if (kGate == 1) {
-                            // channels e, e + 1 of the chunk: one bf16 pair of its gates
                             const uint4 q4 = e < 8 ? g0 : g1;
                             const uint32_t gw = (e & 7) < 2 ? q4.x : (e & 7) < 4 ? q4.y : (e & 7) < 6 ? q4.z : q4.w;
                             m0 = inv_l / (1.f + ex2_approx(-__uint_as_float(gw << 16) * kLog2eF));
                             m1 = inv_l / (1.f + ex2_approx(-__uint_as_float(gw & 0xffff0000u) * kLog2eF));
                         }
-                        return pack_bf16x2(__uint_as_float(orr[c16 + e]) * m0,
-                                           __uint_as_float(orr[c16 + e + 1]) * m1);
+                        return pack_bf16x2(__uint_as_float(orr[e]) * m0, __uint_as_float(orr[e + 1]) * m1);
                     };
                     const uint4 v0 = make_uint4(nb(0), nb(2), nb(4), nb(6));
                     const uint4 v1 = make_uint4(nb(8), nb(10), nb(12), nb(14));
@@ -530,22 +585,26 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     fence_proxy_async_smem();              // visible to the copy engine
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_4d(&a.tm_o, stage, cb + c16, hq, row0, wk.b);
+                        tma_store_4d(&a.tm_o, stage, chunk * 16, hq, row0, wk.b);
                         bulk_commit_group();
                     }
                     g0 = n0;
                     g1 = n1;
                 }
+                if (a.lse != nullptr && i < a.L)
+                    a.lse[((size_t)wk.b * a.hq + hq) * a.L + i] =
+                        l_exact > 0.f ? (m_run + __log2f(l_exact)) * kLn2F : -INFINITY;
+                // O of this head has been read: the next work tile's first PV may overwrite it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&o_free[h]);
             }
-            if (a.lse != nullptr && i < a.L)
-                a.lse[((size_t)wk.b * a.hq + hq) * a.L + i] =
-                    l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2F : -INFINITY;
-            // O is read before this warp's first p_full arrival of the next work
-            // tile, so the next PV (which overwrites O) cannot start early
-            tc_fence_before();
         }
         if (lane == 0) bulk_wait_all();                    // this warp's O stores have landed
         __syncwarp();
+    } else {
+        // warps 14 and 15 hold no role: they only give up their registers
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfOtherRegs));
     }
     tc_fence_before();
     __syncthreads();
@@ -638,6 +697,14 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
         if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmem) !=
             cudaSuccess) {
             snprintf(err, err_len, "cudaFuncSetAttribute(prefill_fwd) failed");
+            return DUO_ERR_CUDA;
+        }
+        // the warps' register split adds up to exactly the launch allocation: a
+        // build with another register count would leave a setmaxnreg.inc waiting
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.numRegs != kPfLaunchRegs) {
+            snprintf(err, err_len, "prefill_fwd was built with %d registers per thread, not %d",
+                     fa.numRegs, kPfLaunchRegs);
             return DUO_ERR_CUDA;
         }
         if (dev >= 0 && dev < 64) smem_set[gate_mode][dev].store(true, std::memory_order_release);
