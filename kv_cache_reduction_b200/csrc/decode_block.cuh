@@ -463,11 +463,6 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         for (; ok && w < n_items; ++ic) {
             const BlockItem bi = block_item_of(a, w);
             const Item &it = bi.it;
-            // the next item's Q goes into the other buffer now (the item with
-            // tiles before this one, which used it, has had all its products read)
-            int w_next = n_items;
-            if (!(ok = read_slot(ic + 1, &w_next))) break;
-            stage_if_needed(w_next);
             float m_run = -INFINITY, l_run = 0.f;
             for (int t = 0; t < it.n_tiles; ++t, ++jg) {
                 const bool got = mbar_wait(&s_full[jg & 1], (jg >> 1) & 1);
@@ -555,6 +550,15 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 if (lane == 0) mbar_arrive(&p_full[jg & 1]);
             }
             if (!ok) break;
+            // The next item's Q goes into the other buffer now, before this item's
+            // epilogue, so that its first products can run meanwhile (the item
+            // with tiles before this one, which used that buffer, has had all its
+            // products read).  Its slot is read only now: the producer publishes
+            // it after loading all of this item's tiles, which needs this
+            // item's tiles to have gone through the softmax.
+            int w_next = n_items;
+            if (!(ok = read_slot(ic + 1, &w_next))) break;
+            stage_if_needed(w_next);
             // ------------------------------------------------------------ item epilogue
             float *part = d.part + (((size_t)it.b * d.hkv + it.g) * a.part_slots + it.split) * C::PartFloats;
             if (it.n_tiles > 0) {

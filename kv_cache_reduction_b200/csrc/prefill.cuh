@@ -63,6 +63,12 @@ static_assert(8 * 32 * kPfSoftmaxRegs + 4 * 32 * kPfEpiRegs + 4 * 32 * kPfOtherR
 #define DUO_PF_POLY_PAIRS 0
 #endif
 constexpr int kPfPolyPairs = DUO_PF_POLY_PAIRS;
+// The two heads take turns for their exponentials (1: on), so that the MUFU
+// units serve one head while the tensor core runs the other head's products.
+#ifndef DUO_PF_TURNS
+#define DUO_PF_TURNS 0
+#endif
+constexpr bool kPfTurns = DUO_PF_TURNS != 0;
 constexpr int kPfStages = 2;
 constexpr int kPfSlots = 4;                // work-tile ring between the producer and the consumers
 constexpr uint32_t kQTileBytes = kPfM * 128 * 2;     // 32 KB: one head's Q tile
@@ -164,7 +170,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     // a work tile's rows handed from the softmax to the epilogue warps: (running
     // max, sum) per row, double-buffered by work tile; O of a head is free again
     // once the epilogue has read it
-    __shared__ uint64_t ml_full[2], o_free[2];
+    // ml_full alternates with the work tile's parity like row_ml: the softmax
+    // may finish a one-tile work tile before the epilogue has waited for the
+    // one before it, and must not complete two phases of one barrier
+    __shared__ uint64_t ml_full[2][2], o_free[2];     // [work tile parity][head], [head]
+    __shared__ uint64_t turn[2];                      // the heads' turns on the MUFU units
     __shared__ float4 row_ml[2][2][kPfM];             // [work tile parity][head][row]: m, l, l exact
     // work tiles claimed by the producer, read by the MMA issuer and the softmax warps
     __shared__ uint64_t work_full[kPfSlots], work_empty[kPfSlots];
@@ -183,9 +193,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             mbar_init(&s_full[h], 1);
             mbar_init(&p_full[h], 4);           // the head's four softmax warps
             mbar_init(&o_done[h], 1);
-            mbar_init(&ml_full[h], 4);
+            mbar_init(&ml_full[0][h], 4);
+            mbar_init(&ml_full[1][h], 4);
             mbar_init(&o_free[h], 4);           // the four epilogue warps
+            mbar_init(&turn[h], 4);
         }
+        for (int w4 = 0; w4 < 4; ++w4) mbar_arrive(&turn[0]);   // head 0 takes the first turn
         for (int sl = 0; sl < kPfSlots; ++sl) {
             mbar_init(&work_full[sl], 1);
             mbar_init(&work_empty[sl], 13);     // the MMA issuer, 8 softmax and 4 epilogue warps
@@ -447,6 +460,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 // score * c - max on the packed f32x2 pipe, two columns per
                 // instruction; the row sum adds the bf16 weights the PV product
                 // uses, so that numerator and denominator agree
+                if (kPfTurns) {
+                    const bool my_turn = mbar_wait(&turn[h], jg & 1);
+                    __syncwarp();
+                    if (!__all_sync(0xffffffffu, my_turn)) { ok = false; break; }
+                }
                 const f2 c2 = f2_splat(c), ms2 = f2_splat(-m_sub);
                 f2 ls0 = f2_splat(0.f), ls1 = f2_splat(0.f), lx0 = f2_splat(0.f), lx1 = f2_splat(0.f);
 #pragma unroll
@@ -476,6 +494,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     // P of keys [16 ch, 16 ch + 16) -> TMEM columns [8 ch, 8 ch + 8)
                     tmem_st8(s_tmem + ch * 8, pw);
                 }
+                if (kPfTurns) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&turn[h ^ 1]);
+                }
                 l_run = l_run * alpha + ((ls0.x + ls0.y) + (ls1.x + ls1.y));
                 l_exact = l_exact * alpha + ((lx0.x + lx0.y) + (lx1.x + lx1.y));
                 m_run = m_use;
@@ -503,7 +525,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             // next work tile; they read O once its last PV is done
             row_ml[wc & 1][h][r] = make_float4(m_run, l_run, l_exact, 0.f);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ml_full[h]);
+            if (lane == 0) mbar_arrive(&ml_full[wc & 1][h]);
         }
         __syncwarp();
     } else if (warp >= kPfEpiWarp0 && warp < kPfEpiWarp0 + 4) {
@@ -542,7 +564,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 } else if (kGate == 2 && i < a.L) {
                     g_head = __bfloat162float(a.gate[((size_t)wk.b * a.L + i) * a.hq + hq]);
                 }
-                const bool ready = mbar_wait(&ml_full[h], wc & 1) && mbar_wait(&o_done[h], (jg - 1) & 1);
+                const bool ready = mbar_wait(&ml_full[wc & 1][h], (wc >> 1) & 1) &&
+                                   mbar_wait(&o_done[h], (jg - 1) & 1);
                 __syncwarp();
                 if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
                 tc_fence_after();
