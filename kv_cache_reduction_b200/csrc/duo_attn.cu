@@ -249,9 +249,15 @@ DecodePlan plan_decode(const duo_params *p, const Layout &L, int64_t max_n, int 
 // pipeline, writing their partials), so the full heads' split count is chosen
 // on the makespan of the persistent CTAs' round-robin share of all the items,
 // in tiles plus that cost.
+#ifndef DUO_BLK_ITEM_COST
+#define DUO_BLK_ITEM_COST 3.0
+#endif
 DecodePlan plan_block(const duo_params *p, const Layout &L, int64_t max_n, int sms, int rows) {
     DecodePlan d = plan_decode(p, L, max_n, sms);
-    const double item = 1.0 + rows / 10.0;          // per-item cost in tiles (measured ~6 at 48 rows)
+    (void)rows;
+    // per-item cost in tiles: staging the item's Q into tensor memory and
+    // writing its partials; the pipeline runs on across items
+    const double item = DUO_BLK_ITEM_COST;
     const int64_t full_units = (int64_t)p->batch * L.n_full;
     const int64_t ring_items = (int64_t)p->batch * L.n_ring * d.splits_ring;
     if (full_units > 0) {
