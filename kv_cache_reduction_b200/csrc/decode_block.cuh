@@ -134,10 +134,11 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
     char *smem = bsmem_base + ((1024u - (smem_u32(bsmem_base) & 1023u)) & 1023u);
     char *sKV = smem;                                         // [stages][K 32 KB | V 32 KB]
     __shared__ uint64_t kv_full[ST], kv_empty[ST], prep_full[ST];
-    // s_full and p_full alternate with the tile parity, like the S buffers, so
-    // that the softmax finishing two tiles before the issuer looks cannot
-    // complete two phases of one barrier
-    __shared__ uint64_t s_full[2], p_full[2], o_done, q_ready[2], mma_drained;
+    // s_full, p_full and o_done alternate with the tile parity, like the S
+    // buffers: with the look-ahead QK^T, the softmax can finish a tile while
+    // the PVs of the two tiles before it are still outstanding, and a wait by
+    // parity on one barrier would then see an older phase as this one
+    __shared__ uint64_t s_full[2], p_full[2], o_done[2], q_ready[2], mma_drained;
     // items claimed by the producer, read by the MMA issuer, the key preparation and the softmax warps
     constexpr int kSlots = 4;
     __shared__ uint64_t work_full[kSlots], work_empty[kSlots];
@@ -158,7 +159,8 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
             mbar_init(&q_ready[i], 4);
             mbar_init(&p_full[i], 4);
         }
-        mbar_init(&o_done, 1);
+        mbar_init(&o_done[0], 1);
+        mbar_init(&o_done[1], 1);
         mbar_init(&mma_drained, 1);
         for (int i = 0; i < kSlots; ++i) {
             mbar_init(&work_full[i], 1);
@@ -404,7 +406,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                            smem_desc_sw128(kv_addr + st * kDecStageBytes + kDecTileBytes + k * 2048,
                                            kDecHalfBytes, 1024),
                            id_pv, (pt == 0 && k == 0) ? 0u : 1u);
-                mma_commit(&o_done);
+                mma_commit(&o_done[jp & 1]);
                 mma_commit(&kv_empty[st]);
                 ++jp;
                 ++pt;
@@ -529,7 +531,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 m_run = m_use;
                 if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                     // O must hold every earlier tile's product before it is scaled
-                    const bool prev = mbar_wait(&o_done, (jg - 1) & 1);
+                    const bool prev = mbar_wait(&o_done[(jg - 1) & 1], ((jg - 1) >> 1) & 1);
                     __syncwarp();
                     if (!__all_sync(0xffffffffu, prev)) { ok = false; break; }
                     tc_fence_after();
@@ -562,7 +564,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
             // ------------------------------------------------------------ item epilogue
             float *part = d.part + (((size_t)it.b * d.hkv + it.g) * a.part_slots + it.split) * C::PartFloats;
             if (it.n_tiles > 0) {
-                const bool done = mbar_wait(&o_done, (jg - 1) & 1);
+                const bool done = mbar_wait(&o_done[(jg - 1) & 1], ((jg - 1) >> 1) & 1);
                 __syncwarp();
                 if (!__all_sync(0xffffffffu, done)) { ok = false; break; }
                 tc_fence_after();
