@@ -468,42 +468,164 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
     }
 }
 
+// The split fold of one output element: M = max(M, m_s) over the splits, then
+// den = sum_s 2^(m_s - M) l_s and num = sum_s 2^(m_s - M) acc_s in split order
+// (splits with m_s = -inf skipped).  m_s, l_s, acc_s sit at floats m_off,
+// l_off, a_off of split s's record of `stride` floats.  The partials were
+// written by the previous grid and sit in L2: the loads go out kFoldBatch
+// splits at a time (only real records are read), so a fold costs about two L2
+// round trips per batch instead of two per split.
+template <int kFoldBatch>
+__device__ __forceinline__ void fold_splits(const float *part, int stride, int splits, int m_off, int l_off,
+                                            int a_off, float *M_io, float *den_io, float *num_io) {
+    float M = *M_io;
+    for (int s0 = 0; s0 < splits; s0 += kFoldBatch) {
+        float mv[kFoldBatch];
+#pragma unroll
+        for (int i = 0; i < kFoldBatch; ++i) {
+            mv[i] = -INFINITY;
+            if (s0 + i < splits) mv[i] = part[(s0 + i) * stride + m_off];
+        }
+#pragma unroll
+        for (int i = 0; i < kFoldBatch; ++i) M = fmaxf(M, mv[i]);
+    }
+    float den = 0.f, num = 0.f;
+    if (M != -INFINITY) {
+        for (int s0 = 0; s0 < splits; s0 += kFoldBatch) {
+            float mv[kFoldBatch], lv[kFoldBatch], av[kFoldBatch];
+#pragma unroll
+            for (int i = 0; i < kFoldBatch; ++i) {
+                mv[i] = -INFINITY;
+                lv[i] = av[i] = 0.f;
+                if (s0 + i < splits) {
+                    const float *ps = part + (s0 + i) * stride;
+                    mv[i] = ps[m_off];
+                    lv[i] = ps[l_off];
+                    av[i] = ps[a_off];
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kFoldBatch; ++i) {
+                if (mv[i] == -INFINITY) continue;
+                const float f = ex2_approx(mv[i] - M);
+                den += f * lv[i];
+                num += f * av[i];
+            }
+        }
+    }
+    *M_io = M;
+    *den_io = den;
+    *num_io = num;
+}
+
+// The split fold of four consecutive output elements: M = max(M, m_s) over
+// the splits, then den = sum_s 2^(m_s - M) l_s and num = sum_s 2^(m_s - M)
+// acc_s in split order (splits with m_s = -inf skipped).  m_s, l_s sit at
+// floats m_off, l_off of split s's record of `stride` floats, the four acc_s at
+// a_off (16-byte aligned).  The partials were written by the previous grid and
+// sit in L2: the loads go out kFoldBatch splits at a time (only real records
+// are read), so a fold costs about two L2 round trips per batch.
+template <int kFoldBatch>
+__device__ __forceinline__ void fold_splits4(const float *part, int stride, int splits, int m_off, int l_off,
+                                             int a_off, float *M_io, float *den_io, float4 *num_io) {
+    float M = *M_io;
+    for (int s0 = 0; s0 < splits; s0 += kFoldBatch) {
+        float mv[kFoldBatch];
+#pragma unroll
+        for (int i = 0; i < kFoldBatch; ++i) {
+            mv[i] = -INFINITY;
+            if (s0 + i < splits) mv[i] = part[(s0 + i) * stride + m_off];
+        }
+#pragma unroll
+        for (int i = 0; i < kFoldBatch; ++i) M = fmaxf(M, mv[i]);
+    }
+    float den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+        for (int s0 = 0; s0 < splits; s0 += kFoldBatch) {
+            float mv[kFoldBatch], lv[kFoldBatch];
+            float4 av[kFoldBatch];
+#pragma unroll
+            for (int i = 0; i < kFoldBatch; ++i) {
+                mv[i] = -INFINITY;
+                lv[i] = 0.f;
+                av[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s0 + i < splits) {
+                    const float *ps = part + (s0 + i) * stride;
+                    mv[i] = ps[m_off];
+                    lv[i] = ps[l_off];
+                    av[i] = *reinterpret_cast<const float4 *>(ps + a_off);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kFoldBatch; ++i) {
+                if (mv[i] == -INFINITY) continue;
+                const float f = ex2_approx(mv[i] - M);
+                den += f * lv[i];
+                num.x += f * av[i].x;
+                num.y += f * av[i].y;
+                num.z += f * av[i].z;
+                num.w += f * av[i].w;
+            }
+        }
+    }
+    *M_io = M;
+    *den_io = den;
+    *num_io = num;
+}
+
+// O = num / den for four output elements, times sigmoid of the output gate
+// (per channel: the four gates at gate4; per head: g_head), as four bf16.
+__device__ __forceinline__ uint2 fold_out4(float4 num, float den, int gate_mode, const __nv_bfloat16 *gate4,
+                                           float g_head) {
+    float o[4] = {num.x, num.y, num.z, num.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = den > 0.f ? o[e] / den : 0.f;
+    if (gate_mode == 1) {
+        const uint2 gw = *reinterpret_cast<const uint2 *>(gate4);
+        const uint32_t gv[2] = {gw.x, gw.y};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float gx = __uint_as_float(e & 1 ? (gv[e >> 1] & 0xffff0000u) : (gv[e >> 1] << 16));
+            o[e] = o[e] / (1.f + ex2_approx(-gx * kLog2eF));
+        }
+    } else if (gate_mode == 2) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] = o[e] / (1.f + ex2_approx(-g_head * kLog2eF));
+    }
+    return make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+}
+
+constexpr int kMergeThreads = kGroup * 32;      // decode_block_merge: a warp per query head
+
 // Folds the splits of every (sequence, query head) and the sink logit:
 // O = sum_s 2^(m_s - M) acc_s / (sum_s 2^(m_s - M) l_s + 2^(sigma*log2e - M)).
-__global__ void __launch_bounds__(kD) decode_merge(const __grid_constant__ DecodeArgs a) {
+// One CTA per (sequence, KV head), thread (hh, r) giving dimension r of head
+// hh: six times fewer CTAs than one per head (the launch of many small CTAs
+// bounds a merge this short).
+__global__ void __launch_bounds__(kD * kGroup) decode_merge(const __grid_constant__ DecodeArgs a) {
     // launched as a programmatic dependent of decode_split: wait until that
     // grid has completed and its partials are visible
     pdl_wait();
-    const int bh = blockIdx.x;
-    const int b = bh / (a.hkv * kGroup);
-    const int h = bh % (a.hkv * kGroup);
-    const int g = h / kGroup, hh = h % kGroup;
+    const int b = blockIdx.x / a.hkv, g = blockIdx.x % a.hkv;
+    const int hh = threadIdx.x / kD, r = threadIdx.x % kD;
+    const int h = g * kGroup + hh;
+    const size_t bh = (size_t)b * a.hkv * kGroup + h;
     const int splits = a.heads.is_full[g] ? a.splits_full : a.splits_ring;
     const float *part = a.part + ((size_t)b * a.hkv + g) * a.max_splits * kPartFloats;
     const bool has_sink = a.sink_logit != nullptr;
     const float sig = has_sink ? a.sink_logit[h] * kLog2eF : -INFINITY;
-    float M = sig;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, part[s * kPartFloats + hh]);
-    float den = 0.f, num = 0.f;
-    if (M != -INFINITY) {
-        for (int s = 0; s < splits; ++s) {
-            const float ms = part[s * kPartFloats + hh];
-            if (ms == -INFINITY) continue;
-            const float f = ex2_approx(ms - M);
-            den += f * part[s * kPartFloats + kGroup + hh];
-            num += f * part[s * kPartFloats + 2 * kGroup + hh * kD + threadIdx.x];
-        }
-        if (has_sink) den += ex2_approx(sig - M);
-    }
+    float M = sig, den = 0.f, num = 0.f;
+    fold_splits<4>(part, kPartFloats, splits, hh, kGroup + hh, 2 * kGroup + hh * kD + r, &M, &den, &num);
+    if (M != -INFINITY && has_sink) den += ex2_approx(sig - M);
     float o = den > 0.f ? num / den : 0.f;
     if (a.gate_mode != 0) {
         // output gate: o * sigmoid(g), g per channel or per head
-        const float g = __bfloat162float(a.gate[a.gate_mode == 1 ? (size_t)bh * kD + threadIdx.x : (size_t)bh]);
-        o = o / (1.f + ex2_approx(-g * kLog2eF));
+        const float gv = __bfloat162float(a.gate[a.gate_mode == 1 ? bh * kD + r : bh]);
+        o = o / (1.f + ex2_approx(-gv * kLog2eF));
     }
-    a.out[(size_t)bh * kD + threadIdx.x] = __float2bfloat16_rn(o);
-    if (a.lse != nullptr && threadIdx.x == 0)
-        a.lse[bh] = den > 0.f ? (M + log2f(den)) * kLn2F : -INFINITY;
+    a.out[bh * kD + r] = __float2bfloat16_rn(o);
+    if (a.lse != nullptr && r == 0) a.lse[bh] = den > 0.f ? (M + log2f(den)) * kLn2F : -INFINITY;
 }
 
 }  // namespace duo

@@ -606,44 +606,35 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
 }
 
 // Folds the splits (the last one holds the block's keys too) and the sink
-// logit of every (sequence, block token, query head).
+// logit of the six query heads of one (sequence, block token, KV head): one
+// warp per head, four output dimensions per thread (few threads: how fast they
+// launch is what bounds a merge this short).  Each fold runs in split order.
 template <int kQ>
-__global__ void __launch_bounds__(kD) decode_block_merge(const __grid_constant__ BlockArgs a) {
+__global__ void __launch_bounds__(kMergeThreads) decode_block_merge(const __grid_constant__ BlockArgs a) {
     using C = BlockCfg<kQ>;
     constexpr int NR = C::NR;
     pdl_wait();
     const DecodeArgs &d = a.d;
-    const int hq_all = d.hkv * kGroup;
-    const int idx = blockIdx.x;                      // (b * q_len + t) * Hq + h
-    const int h = idx % hq_all;
-    const int t = (idx / hq_all) % kQ;
-    const int b = idx / hq_all / kQ;
-    const int g = h / kGroup, row = t * kGroup + h % kGroup;
+    const int grp = blockIdx.x;                      // (b * q_len + t) * Hkv + g
+    const int g = grp % d.hkv;
+    const int t = (grp / d.hkv) % kQ;
+    const int b = grp / d.hkv / kQ;
+    const int hh = threadIdx.x >> 5, c4 = (threadIdx.x & 31) * 4;
+    const int h = g * kGroup + hh;
+    const size_t idx = ((size_t)b * kQ + t) * d.hkv * kGroup + h;   // (b, t, query head)
+    const int row = t * kGroup + hh;
     const int splits = d.heads.is_full[g] ? d.splits_full : d.splits_ring;
     const float *part = d.part + ((size_t)b * d.hkv + g) * a.part_slots * C::PartFloats;
     const bool has_sink = d.sink_logit != nullptr;
     const float sig = has_sink ? d.sink_logit[h] * kLog2eF : -INFINITY;
-    float M = sig;
-    for (int i = 0; i < splits; ++i) M = fmaxf(M, part[i * C::PartFloats + row]);
-    float den = 0.f, num = 0.f;
-    if (M != -INFINITY) {
-        for (int i = 0; i < splits; ++i) {
-            const float *ps = part + i * C::PartFloats;
-            const float ms = ps[row];
-            if (ms == -INFINITY) continue;
-            const float f = ex2_approx(ms - M);
-            den += f * ps[NR + row];
-            num += f * ps[2 * NR + row * kD + threadIdx.x];
-        }
-        if (has_sink) den += ex2_approx(sig - M);
-    }
-    float o = den > 0.f ? num / den : 0.f;
-    if (d.gate_mode != 0) {
-        const float gv = __bfloat162float(d.gate[d.gate_mode == 1 ? (size_t)idx * kD + threadIdx.x : (size_t)idx]);
-        o = o / (1.f + ex2_approx(-gv * kLog2eF));
-    }
-    a.out[(size_t)idx * kD + threadIdx.x] = __float2bfloat16_rn(o);
-    if (a.lse != nullptr && threadIdx.x == 0)
+    float M = sig, den = 0.f;
+    float4 num;
+    fold_splits4<2>(part, C::PartFloats, splits, row, NR + row, 2 * NR + row * kD + c4, &M, &den, &num);
+    if (M != -INFINITY && has_sink) den += ex2_approx(sig - M);
+    const float g_head = d.gate_mode == 2 ? __bfloat162float(d.gate[idx]) : 0.f;
+    *reinterpret_cast<uint2 *>(a.out + idx * kD + c4) =
+        fold_out4(num, den, d.gate_mode, d.gate_mode == 1 ? d.gate + idx * kD + c4 : nullptr, g_head);
+    if (a.lse != nullptr && c4 == 0)
         a.lse[idx] = den > 0.f ? (M + __log2f(den)) * kLn2F : -INFINITY;
 }
 

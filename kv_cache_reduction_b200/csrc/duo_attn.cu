@@ -348,7 +348,7 @@ int launch_block(duo::BlockArgs &a, int grid, cudaStream_t st, int64_t merge_blo
     if ((rc = launch_status("decode_block_split"))) return rc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)merge_blocks);
-    cfg.blockDim = dim3(duo::kD);
+    cfg.blockDim = dim3(duo::kMergeThreads);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -548,8 +548,8 @@ int duo_attn_decode(const duo_params *params, const duo_cache *cache, const void
     // the merge is a programmatic dependent launch: it is scheduled while
     // decode_split drains and waits on the device for its results
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((int64_t)params->batch * params->num_q_heads));
-    cfg.blockDim = dim3(duo::kD);
+    cfg.gridDim = dim3((unsigned)((int64_t)params->batch * params->num_kv_heads));   // one per (b, KV head)
+    cfg.blockDim = dim3(duo::kD * duo::kGroup);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -704,7 +704,7 @@ int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, cons
         return fail(DUO_ERR_CUDA, "zeroing the block decode's work counter failed");
     const int64_t items = d.items;
     const int grid = (int)std::min<int64_t>(items, sms);
-    const int64_t merge_blocks = (int64_t)params->batch * q_len * params->num_q_heads;
+    const int64_t merge_blocks = (int64_t)params->batch * q_len * params->num_kv_heads;   // one per (b, t, KV head)
     cudaStream_t st = (cudaStream_t)stream;
     switch (q_len) {
         case 1: return launch_block<1>(a, grid, st, merge_blocks);
