@@ -293,36 +293,42 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         __syncwarp();
     } else if (warp == kMma) {
         // ------------------------------------------------------------ MMA issuer
-        // Two cursors walk the items' tiles in order: the QK cursor issues
-        // S = Q K^T up to one tile ahead of the PV cursor, but only when its
-        // inputs are already there (a non-blocking check), so that it never holds
-        // up a PV the softmax warps wait for; the PV cursor polls for the
-        // softmax's P and the key preparation, issuing look-ahead products
-        // meanwhile.  Every poll is bounded.
+        // Two cursors walk the items' tiles in order.  Before PV(j) the issuer
+        // issues S(j+1) = Q K(j+1)^T (the look-ahead, so that the softmax finds
+        // the next S ready), then PV(j) once the softmax's P(j) and the key
+        // preparation of tile j are there.  Both waits suspend the thread until
+        // the barrier's phase completes (bounded), so the issuer reacts as soon
+        // as its inputs land and takes no issue slots from the softmax warp on
+        // its sub-partition meanwhile.
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16_f32(128, kTok, 0, 0);
             const uint32_t id_pv = idesc_bf16_f32(128, kD, 0, 1);
             const uint32_t kv_addr = smem_u32(sKV);
-            constexpr int kInfo = 16;
-            int info_w[kInfo], info_n[kInfo];          // item by fetch order: work index, tiles
+            constexpr int kInfo = 8;
+            __shared__ int info_w[kInfo], info_n[kInfo];   // items by fetch order: work index, tiles
             int fetched = 0;
-            int pi = 0;                                // the PV cursor's item
-            auto try_fetch = [&]() -> bool {
-                if (fetched - pi >= kInfo - 1) return false;
+            bool ok = true;
+            auto fetch = [&]() {
                 const int sl = fetched % kSlots;
-                if (!mbar_test(&work_full[sl], (fetched / kSlots) & 1)) return false;
+                if (!(ok = mbar_wait(&work_full[sl], (fetched / kSlots) & 1))) return;
                 const int w = work_slot[sl];
                 mbar_arrive(&work_empty[sl]);
                 info_w[fetched % kInfo] = w;
                 info_n[fetched % kInfo] = w < n_items ? block_item_of(a, w).it.n_tiles : 0;
                 ++fetched;
-                return true;
             };
+            int pi = 0, pt = 0, jp = 0;                // PV cursor: item, tile, products
             int qi = 0, qt = 0, jq = 0, nq = 0;        // QK cursor: item, tile, products, non-empty items
             bool q_end = false;
-            auto try_qk = [&]() -> bool {
-                while (!q_end) {
-                    if (qi == fetched && !try_fetch()) return false;
+            // issues the next S product; false at the end of the list, on a failed
+            // wait, or while the item ring holds kInfo - 1 items ahead of the PV cursor
+            auto next_qk = [&]() -> bool {
+                while (!q_end && ok) {
+                    if (qi == fetched) {
+                        if (fetched - pi >= kInfo - 1) return false;
+                        fetch();
+                        if (!ok) return false;
+                    }
                     if (info_w[qi % kInfo] >= n_items) {
                         q_end = true;
                         return false;
@@ -334,9 +340,10 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                         qt = 0;
                         continue;
                     }
-                    if (qt == 0 && !mbar_test(&q_ready[nq & 1], (nq >> 1) & 1)) return false;   // the item's Q
+                    // the item's Q (staged by the softmax warps), then the key tile
+                    if (qt == 0 && !(ok = mbar_wait(&q_ready[nq & 1], (nq >> 1) & 1))) return false;
                     const int st = jq % ST;
-                    if (!mbar_test(&kv_full[st], (jq / ST) & 1)) return false;
+                    if (!(ok = mbar_wait(&kv_full[st], (jq / ST) & 1))) return false;
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
@@ -351,54 +358,24 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 }
                 return false;
             };
-            int pt = 0, jp = 0;
-            bool ok = true;
-            unsigned long long t_last = clock64();
-            auto stalled = [&](bool progress) -> bool {
-                if (progress) {
-                    t_last = clock64();
-                    return false;
-                }
-                if (clock64() - t_last <= DUO_WAIT_CYCLES) return false;
-                record_status(-5 /* DUO_ERR_TIMEOUT */);
-                return true;
-            };
+            next_qk();                                 // S(0)
             while (ok) {
-                // the PV cursor's next tile
-                bool done = false;
-                while (ok) {
-                    if (pi == fetched) {
-                        bool got = try_fetch();
-                        if (!got && jq < jp + 2) got = try_qk();
-                        if (stalled(got)) ok = false;
-                        continue;
-                    }
-                    if (info_w[pi % kInfo] >= n_items) {
-                        done = true;
-                        break;
-                    }
-                    if (pt < info_n[pi % kInfo]) break;
+                // the PV cursor's next tile: past finished and empty items
+                while (true) {
+                    if (pi == fetched) fetch();
+                    if (!ok || info_w[pi % kInfo] >= n_items || pt < info_n[pi % kInfo]) break;
                     ++pi;
                     pt = 0;
                 }
-                if (!ok || done) break;
-                const int st = jp % ST;
-                // wait for the softmax's P of tile jp and the tile's key preparation,
-                // issuing the look-ahead products as their inputs arrive
-                // (S of tile jp + 2 would overwrite P of tile jp: at most one tile ahead)
-                while (true) {
-                    bool progress = false;
-                    if (jq < jp + 2) progress = try_qk();
-                    if (jq > jp && mbar_test(&p_full[jp & 1], (jp >> 1) & 1) &&
-                        mbar_test(&prep_full[st], (jp / ST) & 1))
-                        break;
-                    if (stalled(progress)) {
-                        ok = false;
-                        break;
-                    }
+                if (!ok || info_w[pi % kInfo] >= n_items) break;
+                // S(jp) and the look-ahead S(jp + 1) before PV(jp) (S(jp + 2) would
+                // overwrite P(jp))
+                while (ok && jq < jp + 2 && next_qk()) {
                 }
-                if (!ok) break;
-                t_last = clock64();
+                if (!ok || jq <= jp) break;
+                const int st = jp % ST;
+                if (!(ok = mbar_wait(&p_full[jp & 1], (jp >> 1) & 1) && mbar_wait(&prep_full[st], (jp / ST) & 1)))
+                    break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
