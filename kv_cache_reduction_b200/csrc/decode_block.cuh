@@ -401,6 +401,14 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         const bool has_row = lane < RQ && r < NR;
         const int tq = has_row ? r / kGroup : 0;             // its block token
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        // The softmax reads S and writes P with the 16-lane shapes: the quad of
+        // threads 4L..4L+3 shares rows A (lane L of the quarter) and B (lane L + 8),
+        // thread qd of the quad holding columns 8k + 2 qd and 8k + 2 qd + 1 of each,
+        // so that all 32 threads work on the quarter's (at most 16) query rows.
+        const int qd = lane & 3, rl = lane >> 2;
+        const int rowA = quarter * RQ + rl, rowB = rowA + 8;
+        const bool hasA = rl < RQ && rowA < NR, hasB = rl + 8 < RQ && rowB < NR;
+        const int tqA = hasA ? rowA / kGroup : 0, tqB = hasB ? rowB / kGroup : 0;
         const float c = d.scale_log2;
         // Stages the query rows of item wq into Q buffer buf (zeros in the padding rows).
         auto stage_q = [&](int wq, int buf) {
@@ -442,20 +450,22 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         for (; ok && w < n_items; ++ic) {
             const BlockItem bi = block_item_of(a, w);
             const Item &it = bi.it;
-            float m_run = -INFINITY, l_run = 0.f;
+            // rows A, B of this thread: running max and its share of the row sum
+            float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
             for (int t = 0; t < it.n_tiles; ++t, ++jg) {
                 const bool got = mbar_wait(&s_full[jg & 1], (jg >> 1) & 1);
                 __syncwarp();
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sr[128];
+                const uint32_t s_tm = tm_s + (jg & 1) * 128 + lane_base;
+                // sr[4k..4k+3]: (A, c), (A, c + 1), (B, c), (B, c + 1) with c = 8k + 2 qd
+                uint32_t sr[64];
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4)
-                    tmem_ld32(tm_s + (jg & 1) * 128 + q4 * 32 + lane_base,
-                              *reinterpret_cast<uint32_t(*)[32]>(&sr[q4 * 32]));
+                    tmem_ld_q16(s_tm + q4 * 32, *reinterpret_cast<uint32_t(*)[16]>(&sr[q4 * 16]));
                 tmem_ld_wait();
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[q4 * 32]));
+                for (int q4 = 0; q4 < 4; ++q4) reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&sr[q4 * 16]));
                 const bool block_tile = t == bi.cache_tiles;
                 // a full head's tile inside the cached length: every key for every query
                 const bool dense = !block_tile && !it.ring && it.e_begin + (t + 1) * kTok <= it.e_end;
@@ -464,49 +474,73 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                     const bool prepped = mbar_wait(&prep_full[st], (jg / ST) & 1);
                     __syncwarp();
                     if (!__all_sync(0xffffffffu, prepped)) { ok = false; break; }
-                    const uint4 mk = *reinterpret_cast<const uint4 *>(key_mask[st][tq]);
-                    const uint32_t mw[4] = {mk.x, mk.y, mk.z, mk.w};
+                    const uint4 ka = *reinterpret_cast<const uint4 *>(key_mask[st][tqA]);
+                    const uint4 kb = *reinterpret_cast<const uint4 *>(key_mask[st][tqB]);
+                    const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-                    for (int cc = 0; cc < 128; ++cc)
-                        if (!((mw[cc >> 5] >> (cc & 31)) & 1u)) sr[cc] = __float_as_uint(-INFINITY);
-                }
-                float mx8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
-#pragma unroll
-                for (int cc = 8; cc < 128; cc += 16)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        mx8[e] = fmax3(mx8[e], __uint_as_float(sr[cc + e]), __uint_as_float(sr[cc + 8 + e]));
-                const float m_tile = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                                           fmaxf(mx8[6], mx8[7])) * c;
-                // keep the stale max unless the new one is more than 2^8 larger
-                float m_use = m_run, alpha = 1.f;
-                if (m_tile > m_run + 8.f) {
-                    m_use = m_tile;
-                    alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_tile);
-                }
-                const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-                const f2 c2 = f2_splat(c), ms2 = f2_splat(-m_sub);
-                f2 ls0 = f2_splat(0.f), ls1 = f2_splat(0.f);
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t pw[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int cc = ch * 16 + 2 * e;
-                        const f2 x = f2_fma(f2_make(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), c2, ms2);
-                        const f2 pe = f2_make(ex2_approx(x.x), ex2_approx(x.y));
-                        pw[e] = pack_bf16x2(pe.x, pe.y);     // bf16 for the PV product
-                        if (e & 1) ls1 = f2_add(ls1, pe);
-                        else ls0 = f2_add(ls0, pe);
+                    for (int k = 0; k < 16; ++k) {
+                        const int sh = 8 * (k & 3) + 2 * qd;   // bit of column 8k + 2 qd in its word
+                        const uint32_t ba = wa[k >> 2] >> sh, bb = wb[k >> 2] >> sh;
+                        if (!(ba & 1u)) sr[4 * k] = __float_as_uint(-INFINITY);
+                        if (!(ba & 2u)) sr[4 * k + 1] = __float_as_uint(-INFINITY);
+                        if (!(bb & 1u)) sr[4 * k + 2] = __float_as_uint(-INFINITY);
+                        if (!(bb & 2u)) sr[4 * k + 3] = __float_as_uint(-INFINITY);
                     }
-                    // P of keys [16 ch, 16 ch + 16) -> TMEM columns [8 ch, 8 ch + 8) of this S buffer
-                    tmem_st8(tm_s + (jg & 1) * 128 + ch * 8 + lane_base, pw);
                 }
-                l_run = l_run * alpha + ((ls0.x + ls0.y) + (ls1.x + ls1.y));
-                m_run = m_use;
-                if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                // the rows' maxima: this thread's 32 columns of each, then its quad
+                float xa[4], xb[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    xa[e] = fmaxf(__uint_as_float(sr[4 * e]), __uint_as_float(sr[4 * e + 1]));
+                    xb[e] = fmaxf(__uint_as_float(sr[4 * e + 2]), __uint_as_float(sr[4 * e + 3]));
+                }
+#pragma unroll
+                for (int k = 4; k < 16; k += 4)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        xa[e] = fmax3(xa[e], __uint_as_float(sr[4 * (k + e)]), __uint_as_float(sr[4 * (k + e) + 1]));
+                        xb[e] = fmax3(xb[e], __uint_as_float(sr[4 * (k + e) + 2]), __uint_as_float(sr[4 * (k + e) + 3]));
+                    }
+                float ta = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
+                float tb = fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3]));
+                ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, 1));
+                tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, 1));
+                ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, 2)) * c;
+                tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, 2)) * c;
+                // keep the stale max unless the new one is more than 2^8 larger
+                float alA = 1.f, alB = 1.f;
+                if (ta > mA + 8.f) {
+                    alA = (mA == -INFINITY) ? 0.f : ex2_approx(mA - ta);
+                    mA = ta;
+                }
+                if (tb > mB + 8.f) {
+                    alB = (mB == -INFINITY) ? 0.f : ex2_approx(mB - tb);
+                    mB = tb;
+                }
+                const f2 c2 = f2_splat(c);
+                const f2 msA = f2_splat(mA == -INFINITY ? 0.f : -mA), msB = f2_splat(mB == -INFINITY ? 0.f : -mB);
+                f2 sa = f2_splat(0.f), sb = f2_splat(0.f);
+                // P: keys (c, c + 1) of each row packed into column 4k + qd of this S buffer
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pw[16];
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int k = half * 8 + kk;
+                        const f2 x0 = f2_fma(f2_make(__uint_as_float(sr[4 * k]), __uint_as_float(sr[4 * k + 1])), c2, msA);
+                        const f2 x1 = f2_fma(f2_make(__uint_as_float(sr[4 * k + 2]), __uint_as_float(sr[4 * k + 3])), c2, msB);
+                        const f2 pa = f2_make(ex2_approx(x0.x), ex2_approx(x0.y));
+                        const f2 pb = f2_make(ex2_approx(x1.x), ex2_approx(x1.y));
+                        pw[2 * kk] = pack_bf16x2(pa.x, pa.y);     // bf16 for the PV product
+                        pw[2 * kk + 1] = pack_bf16x2(pb.x, pb.y);
+                        sa = f2_add(sa, pa);
+                        sb = f2_add(sb, pb);
+                    }
+                    tmem_st_p16(s_tm + half * 32, pw);
+                }
+                lA = lA * alA + (sa.x + sa.y);
+                lB = lB * alB + (sb.x + sb.y);
+                if (t > 0 && __any_sync(0xffffffffu, alA != 1.f || alB != 1.f)) {
                     // O must hold every earlier tile's product before it is scaled
                     const bool prev = mbar_wait(&o_done[(jg - 1) & 1], ((jg - 1) >> 1) & 1);
                     __syncwarp();
@@ -514,13 +548,14 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                     tc_fence_after();
 #pragma unroll
                     for (int cb = 0; cb < 128; cb += 32) {
-                        uint32_t orr[32];
-                        tmem_ld32(tm_o + cb + lane_base, orr);
+                        uint32_t orr[16];
+                        tmem_ld_q16(tm_o + cb + lane_base, orr);
                         tmem_ld_wait();
-                        reg_fence32(orr);
+                        reg_fence16(orr);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                        tmem_st32(tm_o + cb + lane_base, orr);
+                        for (int e = 0; e < 16; ++e)
+                            orr[e] = __float_as_uint(__uint_as_float(orr[e]) * ((e & 2) ? alB : alA));
+                        tmem_st_q16(tm_o + cb + lane_base, orr);
                     }
                 }
                 tmem_st_wait();
@@ -547,25 +582,41 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
                 tc_fence_after();
 #pragma unroll
                 for (int cb = 0; cb < 128; cb += 32) {
-                    uint32_t orr[32];
-                    tmem_ld32(tm_o + cb + lane_base, orr);
+                    uint32_t orr[16];
+                    tmem_ld_q16(tm_o + cb + lane_base, orr);
                     tmem_ld_wait();
-                    reg_fence32(orr);
-                    if (has_row) {
-                        float4 *dst = reinterpret_cast<float4 *>(part + 2 * NR + r * kD + cb);
+                    reg_fence16(orr);
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            dst[e / 4] = make_float4(__uint_as_float(orr[e]), __uint_as_float(orr[e + 1]),
-                                                     __uint_as_float(orr[e + 2]), __uint_as_float(orr[e + 3]));
+                    for (int k = 0; k < 4; ++k) {
+                        const int col = cb + 8 * k + 2 * qd;
+                        if (hasA)
+                            *reinterpret_cast<float2 *>(part + 2 * NR + rowA * kD + col) =
+                                make_float2(__uint_as_float(orr[4 * k]), __uint_as_float(orr[4 * k + 1]));
+                        if (hasB)
+                            *reinterpret_cast<float2 *>(part + 2 * NR + rowB * kD + col) =
+                                make_float2(__uint_as_float(orr[4 * k + 2]), __uint_as_float(orr[4 * k + 3]));
                     }
                 }
-            } else if (has_row) {
-                float4 *dst = reinterpret_cast<float4 *>(part + 2 * NR + r * kD);
-                for (int e = 0; e < kD / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+#pragma unroll 1
+                for (int k = 0; k < 16; ++k) {
+                    const int col = 8 * k + 2 * qd;
+                    if (hasA) *reinterpret_cast<float2 *>(part + 2 * NR + rowA * kD + col) = make_float2(0.f, 0.f);
+                    if (hasB) *reinterpret_cast<float2 *>(part + 2 * NR + rowB * kD + col) = make_float2(0.f, 0.f);
+                }
             }
-            if (has_row) {
-                part[r] = m_run;
-                part[NR + r] = l_run;
+            // each row's sum over its quad, in a fixed order
+            lA += __shfl_xor_sync(0xffffffffu, lA, 1);
+            lB += __shfl_xor_sync(0xffffffffu, lB, 1);
+            lA += __shfl_xor_sync(0xffffffffu, lA, 2);
+            lB += __shfl_xor_sync(0xffffffffu, lB, 2);
+            if (qd == 0 && hasA) {
+                part[rowA] = mA;
+                part[NR + rowA] = lA;
+            }
+            if (qd == 0 && hasB) {
+                part[rowB] = mB;
+                part[NR + rowB] = lB;
             }
             // O is read before this warp's first p_full arrival of the next item
             tc_fence_before();
