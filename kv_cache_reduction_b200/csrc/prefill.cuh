@@ -466,7 +466,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     if (!__all_sync(0xffffffffu, my_turn)) { ok = false; break; }
                 }
                 const f2 c2 = f2_splat(c), ms2 = f2_splat(-m_sub);
-                f2 ls0 = f2_splat(0.f), ls1 = f2_splat(0.f), lx0 = f2_splat(0.f), lx1 = f2_splat(0.f);
+                f2 lx0 = f2_splat(0.f), lx1 = f2_splat(0.f);
+                float lsa = 0.f, lsb = 0.f, lsc = 0.f, lsd = 0.f;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
                     uint32_t pw[8];
@@ -484,10 +485,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                         const uint32_t wv = pack_bf16x2(pe.x, pe.y);
                         pw[e] = wv;
                         if (e & 1) {
-                            ls1 = f2_add(ls1, f2_make(bf16lo(wv), bf16hi(wv)));
+                            add_bf16x2_f32(lsc, lsd, wv);
                             lx1 = f2_add(lx1, pe);
                         } else {
-                            ls0 = f2_add(ls0, f2_make(bf16lo(wv), bf16hi(wv)));
+                            add_bf16x2_f32(lsa, lsb, wv);
                             lx0 = f2_add(lx0, pe);
                         }
                     }
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&turn[h ^ 1]);
                 }
-                l_run = l_run * alpha + ((ls0.x + ls0.y) + (ls1.x + ls1.y));
+                l_run = l_run * alpha + ((lsa + lsb) + (lsc + lsd));
                 l_exact = l_exact * alpha + ((lx0.x + lx0.y) + (lx1.x + lx1.y));
                 m_run = m_use;
                 // O holds the previous key tiles' sum (its PV is complete: this S

@@ -424,6 +424,15 @@ __device__ __forceinline__ f2 ex2_poly2(f2 x) {
                    __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
 }
 
+// s_lo += the bf16 in bits 0..15 of w, s_hi += the one in bits 16..31: the
+// sm_100 mixed-precision add widens the bf16 exactly and adds in f32, one
+// instruction per value with no separate unpack.
+__device__ __forceinline__ void add_bf16x2_f32(float &s_lo, float &s_hi, uint32_t w) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(s_lo), "+f"(s_hi) : "r"(w));
+}
+
 // Packs two floats to bf16x2 (round to nearest even): lo -> bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
