@@ -657,6 +657,101 @@ class VerifyB32(DecodeB32):
                             "2 of 8 KV heads full"}
 
 
+class ChunkPrefill:
+    """Chunked prefill: a 4096-token prompt chunk that continues 28672 cached
+    tokens (32768 in all), B=1, prefill_16k's head mask, through
+    duo_attn_decode_block's long-block path (the cache untouched).  TFLOP/s of
+    the attended (query, key) pairs, 4 * 128 flop each."""
+
+    CACHED, CHUNK = 28672, 4096
+
+    def __init__(self, rank: int, product: bool = True):
+        w = self.w = inputs.workload("prefill_16k")
+        B, n, C = 1, self.CACHED, self.CHUNK
+        seed = rank_seed(w.seed + 31, rank)
+        self.params = duo.DuoParams(B, 48, 8, 128, inputs.SINK, inputs.RECENT, 0, 128 ** -0.5,
+                                    w.full_mask, None)
+        self.cache = duo.DuoCache.allocate(self.params, n)
+        for i, t in enumerate((self.cache.full_k, self.cache.full_v, self.cache.strm_k,
+                               self.cache.strm_v)):
+            inputs.randn_bf16_into(t, seed * 10 + i)
+        self.cache.seq_len.fill_(n)
+        self.cache.ring_head.fill_(int(np.random.default_rng(seed).integers(0, inputs.RECENT)))
+        self.q = inputs.randn_bf16((B, C, 48, 128), seed + 5, "cuda")
+        self.kb = inputs.randn_bf16((B, C, 8, 128), seed + 6, "cuda")
+        self.vb = inputs.randn_bf16((B, C, 8, 128), seed + 7, "cuda")
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty((B, C, 48), dtype=torch.float32, device="cuda")
+        if product:
+            nb = duo.duo_decode_block_workspace_bytes(self.params, C, n)
+            self.ws = torch.empty((nb + 255) // 256 * 256, dtype=torch.uint8, device="cuda")
+        n_full = sum(1 for g in range(8) if w.full_mask[g])
+        span = inputs.SINK + inputs.RECENT
+        pairs = 6 * n_full * (C * n + C * (C + 1) // 2) + 6 * (8 - n_full) * C * span
+        self.flops = 4 * 128 * pairs * B
+        self.launches_per_step = 3      # prefill_fwd twice (cached keys, own keys) + block_combine
+        self.unit = "TFLOP/s"
+        self.kernel = "prefill_fwd (cache mode) + prefill_fwd + block_combine (one duo_attn_decode_block call)"
+        self.traffic_key = ("prefill_fwd", "chunk_32k")
+
+    def step(self):
+        duo.duo_attn_decode_block(self.params, self.cache, self.q, self.kb, self.vb, self.CACHED,
+                                  self.out, self.lse, self.ws)
+
+    def e2e_buffers(self):
+        self.h_in = [t.cpu().pin_memory() for t in (self.q, self.kb, self.vb)]
+        self.d_in = [torch.empty_like(t) for t in (self.q, self.kb, self.vb)]
+        self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h_lse = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
+        return sum(t.numel() * 2 for t in self.h_in), self.h_out.numel() * 2 + self.h_lse.numel() * 4
+
+    def e2e_step(self):
+        for d, h in zip(self.d_in, self.h_in):
+            d.copy_(h, non_blocking=True)
+        duo.duo_attn_decode_block(self.params, self.cache, *self.d_in, self.CACHED, self.out, self.lse,
+                                  self.ws)
+        self.h_out.copy_(self.out, non_blocking=True)
+        self.h_lse.copy_(self.lse, non_blocking=True)
+
+    def config(self):
+        return {"workload": f"chunk_32k: chunked prefill, B=1, a {self.CHUNK}-token chunk after "
+                            f"{self.CACHED} cached tokens, 2 of 8 KV heads full",
+                "full_mask": list(self.w.full_mask), "l2": "inputs larger than L2"}
+
+    def oracle_sample(self, budget_s: float = 15.0):
+        """The oracle's block decode on seeded sets of 16 chunk positions (every
+        query head of each, in one call), cycled until the budget; TFLOP/s of the
+        attended pairs those rows cover."""
+        import oracle
+        p, n, C = self.params, self.CACHED, self.CHUNK
+        ol = oracle.Layer(1, 48, 8, 128, p.sink, p.recent, 0, p.softmax_scale, tuple(p.full_mask), None)
+        hc = oracle.Cache(ol, n)
+        hc.full_k[...] = inputs.bits(self.cache.full_k)
+        hc.full_v[...] = inputs.bits(self.cache.full_v)
+        hc.strm_k[...] = inputs.bits(self.cache.strm_k)
+        hc.strm_v[...] = inputs.bits(self.cache.strm_v)
+        hc.seq_len[...] = self.cache.seq_len.cpu().numpy()
+        hc.ring_head[...] = self.cache.ring_head.cpu().numpy()
+        qb, kb, vb = (inputs.bits(t) for t in (self.q, self.kb, self.vb))
+        rng = np.random.default_rng(self.w.seed + 78)
+        n_full = sum(1 for g in range(8) if p.full_mask[g])
+        units = []
+        for _ in range(64):
+            pos = np.sort(rng.integers(0, C, size=16))
+            rows = np.asarray([t * 48 + h for t in pos for h in range(48)], dtype=np.int64)
+            pairs = sum(6 * n_full * (n + int(t) + 1) + 6 * (8 - n_full) * (p.sink + p.recent) for t in pos)
+            units.append((rows, pairs * 4 * 128))
+
+        def run(u):
+            oracle.attn_decode_block(ol, hc, qb, kb, vb, rows=u[0])
+
+        done, t_total, used = timed_sample(units, run, lambda u: u[1], budget_s)
+        return {"value": done / t_total / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                "kind": "oracle",
+                "sample": f"{used} calls of 768 rows (16 seeded chunk positions x 48 query heads), "
+                          f"{done / 1e9:.1f} GFLOP of attended pairs, float64, {t_total:.1f} s"}
+
+
 class Prep:
     """The fused query/key preparation + append of a 16384-token prompt on the
     prefill_16k layer (2 of 8 KV heads full): RMSNorm + YaRN RoPE of q and k in
@@ -853,8 +948,9 @@ class DecodeSmall:
 WORKLOADS = {"decode_b32": DecodeB32, "stack40": Stack40, "decode_small": DecodeSmall, "prep_16k": Prep,
              "verify_b32": VerifyB32,
              "prefill_16k": lambda rank, product=True: Prefill(rank, "prefill_16k", product),
-             "sliding_32k": lambda rank, product=True: Prefill(rank, "sliding_32k", product)}
-SECONDARY = ("stack40", "verify_b32", "prefill_16k", "sliding_32k", "prep_16k", "decode_small")
+             "sliding_32k": lambda rank, product=True: Prefill(rank, "sliding_32k", product),
+             "chunk_32k": ChunkPrefill}
+SECONDARY = ("stack40", "verify_b32", "prefill_16k", "sliding_32k", "prep_16k", "decode_small", "chunk_32k")
 
 
 # ------------------------------------------------------------------ timing
@@ -1044,7 +1140,7 @@ def run_reference(args, world, rank):
     workload; its inputs are built with torch alone (the library is not loaded)."""
     if rank != 0:
         return None
-    if args.workload in ("verify_b32", "prep_16k"):
+    if args.workload in ("verify_b32", "prep_16k", "chunk_32k"):
         return {"impl": "reference", "unavailable": f"no CPU oracle leg for {args.workload}; the "
                                                     "reference arm covers the workloads of the main line"}
     import oracle

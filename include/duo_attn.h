@@ -238,30 +238,37 @@ DUO_API int duo_attn_decode(const duo_params *params, const duo_cache *cache, co
                     size_t workspace_bytes, const duo_gate *gate, void *stream);
 
 /* Bytes of device workspace duo_attn_decode_block needs (0 on invalid
- * arguments or q_len outside [1, 8]). */
+ * arguments or q_len outside [1, 2^30]). */
 DUO_API size_t duo_decode_block_workspace_bytes(const duo_params *params, int32_t q_len,
                                                 int32_t max_seq_len);
 
-/* Block decode: q_len (1..8) query tokens per sequence against the cache as
- * it stands BEFORE they are appended -- the verify pass of block speculative
+/* Block decode: q_len query tokens per sequence against the cache as it
+ * stands BEFORE they are appended -- the verify pass of block speculative
  * decoding (Laguna-XS-2.1 cookbook, section 3.1 DFlash: the target checks a
- * drafted block in one forward pass and keeps the tokens it accepts).
+ * drafted block in one forward pass and keeps the tokens it accepts), and, for
+ * long blocks, chunked prefill: a prompt chunk that continues cached tokens.
  * Query t of sequence b sits at position i = seq_len[b] + t and attends to
  * the keys its head's rule allows at i: cached ones (a full head every cached
  * row; a ring head its sink slots and the ring slots holding a position
  * j > i - recent, resp. window) and the block's own keys u <= t under the same
  * rule, read from k_new / v_new.  The cache is not modified: append the
  * accepted tokens with duo_kv_append afterwards (rejected draft tokens never
- * reach the ring, which could not take them back).
+ * reach the ring, which could not take them back; a prompt chunk is appended
+ * whole, after this call, before the next chunk).
+ * Blocks of up to 8 tokens run as one split kernel over the cache (the
+ * block's keys ride on each head's last split) and a merge.  Longer blocks run
+ * the prefill kernel twice, over the cached keys and over the block's own
+ * keys, and fold the two by their log-sum-exps.
  * q: device bf16 [B][q_len][Hq][D]; k_new, v_new: [B][q_len][Hkv][D];
  * out: [B][q_len][Hq][D]; lse: fp32 [B][q_len][Hq] or NULL.  max_seq_len
  * bounds every seq_len[b] (the cached length, without the block).
  * workspace: >= duo_decode_block_workspace_bytes(params, q_len, max_seq_len)
  * bytes, 256-byte aligned, contents need not be initialised (it holds the
- * split partials and a work-item counter that the call zeroes on the stream;
- * calls that may run at the same time need separate workspaces).  gate: NULL or an
- * output gate (values [B][q_len][Hq][D] or [B][q_len][Hq]).  q_len outside
- * [1, 8] is DUO_ERR_UNSUPPORTED; other errors as duo_attn_decode. */
+ * split partials, or for long blocks the two halves' outputs, and work-item
+ * counters that the call zeroes on the stream; calls that may run at the same
+ * time need separate workspaces).  gate: NULL or an output gate (values
+ * [B][q_len][Hq][D] or [B][q_len][Hq]).  q_len outside [1, 2^30] is
+ * DUO_ERR_UNSUPPORTED; other errors as duo_attn_decode. */
 DUO_API int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, const void *q,
                                   const void *k_new, const void *v_new, int32_t q_len,
                                   int32_t max_seq_len, void *out, float *lse, void *workspace,

@@ -415,9 +415,10 @@ def duo_attn_decode_block(params: DuoParams, cache: DuoCache, q: torch.Tensor, k
                           v_new: torch.Tensor, max_seq_len: int, out: torch.Tensor,
                           lse: Optional[torch.Tensor], workspace: torch.Tensor, stream=None,
                           gate: Optional[torch.Tensor] = None) -> None:
-    """Verify-block decode: q [B][k][Hq][D] at positions seq_len[b] + t against
-    the cache plus the block's own k_new / v_new [B][k][Hkv][D]; the cache is
-    not modified."""
+    """Block decode: q [B][k][Hq][D] at positions seq_len[b] + t against the
+    cache plus the block's own k_new / v_new [B][k][Hkv][D]; the cache is not
+    modified.  k <= 8 is a verify block; longer blocks (chunked prefill: a
+    prompt chunk continuing cached tokens) take the two-pass prefill path."""
     p, c = params.as_c(), cache.as_c(params)
     B, D, bf = params.batch, params.head_dim, torch.bfloat16
     k = int(q.shape[1]) if q is not None and q.dim() == 4 else -1

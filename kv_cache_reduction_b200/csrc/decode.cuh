@@ -574,6 +574,14 @@ __device__ __forceinline__ void fold_splits4(const float *part, int stride, int 
     *num_io = num;
 }
 
+// Four bf16 (two packed words) to floats.
+__device__ __forceinline__ void unpack_bf16x4(uint2 w, float (&f)[4]) {
+    f[0] = __uint_as_float(w.x << 16);
+    f[1] = __uint_as_float(w.x & 0xffff0000u);
+    f[2] = __uint_as_float(w.y << 16);
+    f[3] = __uint_as_float(w.y & 0xffff0000u);
+}
+
 // O = num / den for four output elements, times sigmoid of the output gate
 // (per channel: the four gates at gate4; per head: g_head), as four bf16.
 __device__ __forceinline__ uint2 fold_out4(float4 num, float den, int gate_mode, const __nv_bfloat16 *gate4,

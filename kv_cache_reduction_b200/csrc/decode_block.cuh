@@ -666,4 +666,62 @@ __global__ void __launch_bounds__(kMergeThreads) decode_block_merge(const __grid
         a.lse[idx] = den > 0.f ? (M + __log2f(den)) * kLn2F : -INFINITY;
 }
 
+// A block longer than the verify kernel takes is computed in two passes: its
+// queries against the cached keys (prefill_fwd's cache mode; a full head's keys
+// in kv_splits runs, each written as its own slice) and against its own keys
+// (prefill_fwd's prompt mode, which also adds the sink logit).  Each part is
+// normalised by its own sum and rounded to bf16; they are folded here by their
+// sums: O = sum_p e^Lp Op / sum_p e^Lp, LSE = ln sum_p e^Lp.
+struct CombineArgs {
+    const __nv_bfloat16 *oa, *ob;   // [S][B][C][Hq][D], [B][C][Hq][D]
+    const float *lse_a, *lse_b;     // [S][B][Hq][C], [B][Hq][C]
+    __nv_bfloat16 *out;             // [B][C][Hq][D]
+    float *lse;                     // [B][C][Hq] or null
+    const __nv_bfloat16 *gate;      // output gate pre-activations or null
+    int32_t gate_mode, C, hq, batch, kv_splits, split_tiles, capacity;
+    const int32_t *seq_len;         // cached tokens per sequence
+    int8_t is_full[64];             // per KV head: its cached keys come in split slices (else one)
+};
+
+// One warp per (sequence, block token, query head), four output dimensions per thread.
+__global__ void __launch_bounds__(kMergeThreads) block_combine(const __grid_constant__ CombineArgs a) {
+    const int hh = threadIdx.x >> 5, c4 = (threadIdx.x & 31) * 4;
+    const int64_t row = (int64_t)blockIdx.x * kGroup + hh;          // (b * C + t) * Hq + h
+    const int h = (int)(row % a.hq);
+    const int64_t bt = row / a.hq;
+    const int64_t t = bt % a.C, b = bt / a.C;
+    // a full head's slices: as many as its cached rows fill (prefill_fwd passes
+    // over the rest unwritten); split 0 always, maybe with no key
+    int parts = 1;
+    if (a.is_full[h / kGroup]) {
+        const int tiles = (min(max(a.seq_len[b], 0), a.capacity) + 127) / 128;
+        parts = min(a.kv_splits, max(1, (tiles + a.split_tiles - 1) / a.split_tiles));
+    }
+    const size_t slice_o = (size_t)a.batch * a.C * a.hq * kD, slice_l = (size_t)a.batch * a.hq * a.C;
+    const size_t li = ((size_t)b * a.hq + h) * a.C + t;
+    float M = a.lse_b[li] * kLog2eF;
+    for (int s = 0; s < parts; ++s) M = fmaxf(M, a.lse_a[s * slice_l + li] * kLog2eF);
+    float den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+        for (int s = 0; s <= parts; ++s) {          // the cached slices, then the block's own part
+            const bool own = s == parts;
+            const float l = (own ? a.lse_b[li] : a.lse_a[s * slice_l + li]) * kLog2eF;
+            if (l == -INFINITY) continue;
+            const float wgt = ex2_approx(l - M);
+            float f[4];
+            unpack_bf16x4(*reinterpret_cast<const uint2 *>((own ? a.ob : a.oa + s * slice_o) + row * kD + c4), f);
+            den += wgt;
+            num.x += wgt * f[0];
+            num.y += wgt * f[1];
+            num.z += wgt * f[2];
+            num.w += wgt * f[3];
+        }
+    }
+    const float g_head = a.gate_mode == 2 ? __bfloat162float(a.gate[row]) : 0.f;
+    *reinterpret_cast<uint2 *>(a.out + row * kD + c4) =
+        fold_out4(num, den, a.gate_mode, a.gate_mode == 1 ? a.gate + row * kD + c4 : nullptr, g_head);
+    if (a.lse != nullptr && c4 == 0) a.lse[row] = den > 0.f ? (M + __log2f(den)) * kLn2F : -INFINITY;
+}
+
 }  // namespace duo

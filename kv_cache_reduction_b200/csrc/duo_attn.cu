@@ -608,18 +608,100 @@ int duo_cache_bytes(const duo_params *params, int64_t capacity, int64_t seq_len,
 }
 
 // ------------------------------------------------------------------ block decode
+// A block longer than kMaxBlock tokens.  The full heads' cached keys are cut
+// into kv_splits runs so that the pass over the cache has enough work tiles for
+// the SMs: the count minimises the estimated makespan of the persistent CTAs
+// (a work tile costs its key tiles plus two for its fill and epilogue).
+struct LongBlockPlan {
+    int kv_splits, split_tiles;
+    size_t o_bytes, l_bytes, total;     // one bf16 [B][q_len][Hq][D] slice, one fp32 [B][Hq][q_len] slice
+};
+
+LongBlockPlan long_block_plan(const duo_params *p, const Layout &L, int64_t q_len, int64_t max_seq_len, int sms) {
+    LongBlockPlan w;
+    const int64_t qtiles = (q_len + duo::kPfM - 1) / duo::kPfM;
+    const int64_t tiles = std::max<int64_t>(1, (max_seq_len + duo::kPfN - 1) / duo::kPfN);
+    const int64_t units = (int64_t)p->batch * L.n_full * (duo::kGroup / 2) * qtiles;    // full head pairs x query tiles
+    const int64_t ring_units = (int64_t)p->batch * L.n_ring * (duo::kGroup / 2) * qtiles;
+    w.kv_splits = 1;
+    w.split_tiles = (int)tiles;
+    if (units > 0) {
+        double best = 1e300;
+        for (int64_t s = 1; s <= std::min<int64_t>(tiles, 64); ++s) {
+            const int64_t chunk = (tiles + s - 1) / s;
+            const double span = (double)((units * s + ring_units + sms - 1) / sms) * (double)(chunk + 2);
+            if (span < best - 1e-9) {
+                best = span;
+                w.kv_splits = (int)s;
+                w.split_tiles = (int)chunk;
+            }
+        }
+    }
+    w.o_bytes = ((size_t)p->batch * q_len * p->num_q_heads * duo::kD * 2 + 255) / 256 * 256;
+    w.l_bytes = ((size_t)p->batch * p->num_q_heads * q_len * sizeof(float) + 255) / 256 * 256;
+    // the cache pass's slices, the block pass's output and LSE, two work-tile counters
+    w.total = (size_t)(w.kv_splits + 1) * (w.o_bytes + w.l_bytes) + 2 * 256;
+    return w;
+}
+
 size_t duo_decode_block_workspace_bytes(const duo_params *params, int32_t q_len, int32_t max_seq_len) {
     Layout L;
-    if (check_params(params, &L) || q_len < 1 || q_len > kMaxBlock || max_seq_len < 0 ||
-        max_seq_len > kMaxPos)
+    if (check_params(params, &L) || q_len < 1 || q_len > kMaxPos || max_seq_len < 0 || max_seq_len > kMaxPos)
         return 0;
     int sms = 148;
     if (check_device(&sms)) sms = 148;
+    if (q_len > kMaxBlock) return long_block_plan(params, L, q_len, max_seq_len, sms).total;
     const DecodePlan d = plan_block(params, L, max_seq_len, sms, duo::kGroup * q_len);
     const size_t slots = (size_t)std::max(d.splits_full, d.splits_ring);
     const size_t partials = (size_t)params->batch * params->num_kv_heads * slots *
                             (size_t)(duo::kGroup * q_len) * (duo::kD + 2) * sizeof(float);
     return (partials + 255) / 256 * 256 + 256;       // + the work-item counter
+}
+
+// The block q [B][q_len][Hq][D] (q_len > kMaxBlock) against the cache before it is
+// appended, plus its own keys: prefill_fwd in cache mode over the cached keys,
+// prefill_fwd in prompt mode over the block's keys (its sink shifted by each
+// sequence's cached length; the sink logit joins here), then block_combine.
+int long_block(const duo_params *params, const Layout &L, const duo_cache *cache, const void *q,
+               const void *k_new, const void *v_new, int32_t q_len, int32_t max_seq_len, void *out, float *lse,
+               void *workspace, int gate_mode, const void *gate_values, int sms, cudaStream_t st) {
+    const LongBlockPlan pl = long_block_plan(params, L, q_len, max_seq_len, sms);
+    char *w = (char *)workspace;
+    void *oa = w;                                                  // [S][B][q_len][Hq][D]
+    void *ob = w + (size_t)pl.kv_splits * pl.o_bytes;              // [B][q_len][Hq][D]
+    float *la = (float *)(w + (size_t)(pl.kv_splits + 1) * pl.o_bytes);   // [S][B][Hq][q_len]
+    float *lb = (float *)((char *)la + (size_t)pl.kv_splits * pl.l_bytes);
+    int32_t *ca = (int32_t *)((char *)lb + pl.l_bytes), *cb = ca + 64;
+    char err[256];
+    int rc = duo::launch_prefill_cache(params, L.sliding, L.heads.is_full, L.heads.rank, L.n_full, L.n_ring,
+                                       L.sink, L.ring, L.n_full > 0 ? cache->capacity : 0, cache->full_k,
+                                       cache->full_v, cache->strm_k, cache->strm_v, cache->seq_len, cache->ring_head,
+                                       q, q_len, pl.kv_splits, pl.split_tiles, oa, la, ca, -1, st, err, sizeof err);
+    if (rc) return fail(rc, "%s", err);
+    rc = duo::launch_prefill(params, L.sliding, L.heads.is_full, L.sink, L.ring, q, k_new, v_new, q_len, ob, lb,
+                             cb, 0, nullptr, -1, st, err, sizeof err, cache->seq_len);
+    if (rc) return fail(rc, "%s", err);
+    duo::CombineArgs c;
+    memset(&c, 0, sizeof c);
+    c.oa = (const __nv_bfloat16 *)oa;
+    c.ob = (const __nv_bfloat16 *)ob;
+    c.lse_a = la;
+    c.lse_b = lb;
+    c.out = (__nv_bfloat16 *)out;
+    c.lse = lse;
+    c.gate = (const __nv_bfloat16 *)gate_values;
+    c.gate_mode = gate_mode;
+    c.C = q_len;
+    c.hq = params->num_q_heads;
+    c.batch = params->batch;
+    c.kv_splits = pl.kv_splits;
+    c.split_tiles = pl.split_tiles;
+    c.capacity = L.n_full > 0 ? (int32_t)std::min<int64_t>(cache->capacity, INT32_MAX) : 0;
+    c.seq_len = cache->seq_len;
+    for (int g = 0; g < params->num_kv_heads; ++g) c.is_full[g] = L.heads.is_full[g];
+    duo::block_combine<<<(unsigned)((int64_t)params->batch * q_len * params->num_kv_heads), duo::kMergeThreads, 0,
+                         st>>>(c);
+    return launch_status("block_combine");
 }
 
 int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, const void *q,
@@ -630,8 +712,8 @@ int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, cons
     int rc = check_params(params, &L);
     if (rc) return rc;
     if ((rc = check_cache(cache, L))) return rc;
-    if (q_len < 1 || q_len > kMaxBlock)
-        return fail(DUO_ERR_UNSUPPORTED, "q_len must be in [1, %d] (got %d)", kMaxBlock, q_len);
+    if (q_len < 1 || q_len > kMaxPos)
+        return fail(DUO_ERR_UNSUPPORTED, "q_len must be in [1, 2^30] (got %d)", q_len);
     int gate_mode = 0;
     const void *gate_values = nullptr;
     if ((rc = check_gate(gate, &gate_mode, &gate_values))) return rc;
@@ -648,11 +730,17 @@ int duo_attn_decode_block(const duo_params *params, const duo_cache *cache, cons
         return fail(DUO_ERR_UNSUPPORTED, "cache rows exceed 2^31 (tensor-map coordinates are 32-bit)");
     int sms = 148;
     if ((rc = check_device(&sms))) return rc;
-    const DecodePlan d = plan_block(params, L, max_seq_len, sms, duo::kGroup * q_len);
     const size_t need = duo_decode_block_workspace_bytes(params, q_len, max_seq_len);
     if (!workspace || workspace_size < need || ((uintptr_t)workspace & 255u))
         return fail(DUO_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
                     workspace_size);
+    if (q_len > kMaxBlock) {
+        if ((int64_t)params->batch * params->num_q_heads / 2 * ((q_len + duo::kPfM - 1) / duo::kPfM) > INT32_MAX - 4096)
+            return fail(DUO_ERR_UNSUPPORTED, "too many query tiles for one block");
+        return long_block(params, L, cache, q, k_new, v_new, q_len, max_seq_len, out, lse, workspace, gate_mode,
+                          gate_values, sms, (cudaStream_t)stream);
+    }
+    const DecodePlan d = plan_block(params, L, max_seq_len, sms, duo::kGroup * q_len);
     duo::BlockArgs a;
     memset(&a, 0, sizeof a);
     duo::DecodeArgs &da = a.d;

@@ -97,6 +97,21 @@ struct PrefillArgs {
     int32_t withhold_tile; // failure-injection hook: CTA 0 issues no K/V load from this tile on (-1: off)
     float scale_log2;
     int8_t kind[64];       // per KV head
+    // The block's keys: in prompt mode, seq_len (or null) gives the position each
+    // sequence's block starts at, which shifts the sink.  In cache mode (the block's
+    // queries against the cache as it stands before the block), tm_k / tm_v map the
+    // full caches [B][n_full][capacity][128] as (128, capacity, n_full, B) and
+    // tm_k2 / tm_v2 the sink + ring caches [B][n_ring][slots][128] as
+    // (128, slots, n_ring, B); seq_len holds each sequence's cached tokens.
+    CUtensorMap tm_k2, tm_v2;
+    const int32_t *seq_len, *ring_head;
+    int32_t capacity;
+    // cache mode: a full head's cached key tiles are cut into kv_splits chunks of
+    // split_tiles tiles, each its own work tile writing O and the LSE to slice s
+    // of out ([S][B][L][Hq][128]) and lse ([S][B][Hq][L]); ring heads use slice 0
+    // only.  Prompt mode: 1.
+    int32_t kv_splits, split_tiles, batch;
+    int8_t rank[64];       // cache mode: per KV head, its rank among heads of its kind
 };
 
 // Key tiles of query tile t for one head kind: an optional run of sink
@@ -140,25 +155,128 @@ __device__ __forceinline__ bool tile_dense(int kind, int r0, int c0, int sink, i
     return c0 > r1 - window;
 }
 
+// The key tiles of a work tile.  Prompt mode: the TileList of its query tile
+// (with this sequence's sink).  Cache mode: tiles [0, count) of the head's
+// cache (a full head's rows, a ring head's slots), never empty: a work tile with
+// no cached key gets one tile in which every key is masked.
+struct PfKeys {
+    TileList tl;
+    int sink;              // prompt mode: the sink keys among the block's keys
+    int n, ns, cnt, rh;    // cache mode: cached tokens, sink slots and ring slots holding
+                           // one, ring cursor
+    __device__ int count() const { return tl.count(); }
+    __device__ int at(int j) const { return tl.at(j); }
+};
+
 // Work tile w: query tile t (heaviest first) of head pair p of sequence b.
 struct PfWork {
-    int b, h0, g, t;
+    int b, h0, g, t, s;    // s: the split of the cached keys (cache mode)
 };
 
 __device__ __forceinline__ PfWork work_of(const PrefillArgs &a, int w) {
     const int pairs = a.hq / 2;
-    const int per_t = a.batch_pairs;
+    const int per_t = a.batch_pairs * a.kv_splits;
     PfWork wk;
     wk.t = a.n_qtiles - 1 - w / per_t;
-    const int bp = w % per_t;
+    const int bp = (w % per_t) / a.kv_splits;
+    wk.s = w % a.kv_splits;
     wk.b = bp / pairs;
     wk.h0 = (bp % pairs) * 2;
     wk.g = wk.h0 / (a.hq / a.hkv);
     return wk;
 }
 
+template <bool kCache>
+__device__ __forceinline__ PfKeys pf_keys(const PrefillArgs &a, const PfWork &wk) {
+    PfKeys k{};
+    const int kind = a.kind[wk.g];
+    if (!kCache) {
+        k.sink = a.seq_len != nullptr ? max(0, a.sink - a.seq_len[wk.b]) : a.sink;
+        k.tl = tile_list(kind, wk.t, a.L, k.sink, a.recent, a.window);
+        return k;
+    }
+    k.n = max(a.seq_len[wk.b], 0);
+    int tiles;
+    if (kind == kKindFull) {
+        k.n = min(k.n, a.capacity);                    // a full head's rows end at the capacity
+        tiles = (k.n + kPfN - 1) / kPfN;
+        if (wk.s > 0 || tiles > a.split_tiles) {
+            // split s: tiles [s * split_tiles, ...); empty past the head's rows
+            // (split 0 of an empty cache keeps its one masked tile)
+            const int lo = wk.s * a.split_tiles, hi = min(tiles, lo + a.split_tiles);
+            k.tl = TileList{0, lo, hi - 1};
+            if (hi <= lo) k.tl = TileList{0, 0, wk.s == 0 ? 0 : -1};
+            return k;
+        }
+    } else {
+        // R = a.recent (the window on a sliding layer, whose sink is 0)
+        k.ns = min(k.n, a.sink);
+        k.cnt = min(max(k.n - a.sink, 0), a.recent);
+        k.rh = a.ring_head[wk.b];
+        // rows i >= R - 1 of the block see no ring slot, only the sink
+        const bool ring_seen = k.cnt > 0 && wk.t * kPfM < a.recent - 1;
+        tiles = ring_seen ? (a.sink + a.recent + kPfN - 1) / kPfN : (k.ns + kPfN - 1) / kPfN;
+        if (wk.s > 0) tiles = -1;                      // ring heads: split 0 only
+    }
+    k.tl = TileList{0, 0, tiles < 0 ? -1 : max(tiles, 1) - 1};
+    return k;
+}
+
+// Cache mode: the attended columns of key tile c0 for block row i, as 128 bits
+// (w[0] columns 0-31 ... w[3] columns 96-127).  A full head sees its cached rows;
+// a ring head its sink slots holding a token and the ring slots holding one of
+// positions n - 1 - d > n + i - R, i.e. d < R - 1 - i (d-th to last written): a
+// cyclic run of slots ending before the ring cursor.
+__device__ __forceinline__ void cache_mask(const PrefillArgs &a, const PfKeys &k, int kind, int i, int c0,
+                                           uint32_t (&w)[4]) {
+    int lo[3] = {1, 1, 1}, hi[3] = {0, 0, 0};       // up to three ranges of columns
+    if (kind == kKindFull) {
+        lo[0] = -c0;
+        hi[0] = k.n - 1 - c0;
+    } else {
+        lo[0] = -c0;
+        hi[0] = k.ns - 1 - c0;
+        const int R = a.recent, S = a.sink;
+        const int len = min(k.cnt, R - 1 - i);
+        if (len > 0) {
+            const int r_end = (k.rh - 1 + R) % R, r_start = r_end - len + 1;
+            if (r_start >= 0) {
+                lo[1] = S + r_start - c0;
+                hi[1] = S + r_end - c0;
+            } else {
+                lo[1] = S - c0;
+                hi[1] = S + r_end - c0;
+                lo[2] = S + R + r_start - c0;
+                hi[2] = S + R - 1 - c0;
+            }
+        }
+    }
+    uint64_t m0 = 0, m1 = 0;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+        m0 |= col_range_bits(lo[q], hi[q]);
+        m1 |= col_range_bits(lo[q] - 64, hi[q] - 64);
+    }
+    w[0] = (uint32_t)m0;
+    w[1] = (uint32_t)(m0 >> 32);
+    w[2] = (uint32_t)m1;
+    w[3] = (uint32_t)(m1 >> 32);
+}
+
+// Cache mode: does key e (a full head's row, a ring head's slot) hold a token?
+// (Rows past the cache's end are zero-filled by the tensor map.)
+__device__ __forceinline__ bool cache_key_valid(const PrefillArgs &a, const PfKeys &k, int kind, int e) {
+    if (kind == kKindFull) return e < k.n || e >= a.capacity;
+    const int S = a.sink, R = a.recent;
+    if (e < S) return e < k.ns;
+    if (e >= S + R) return true;
+    const int d = ((k.rh - 1 - (e - S)) % R + R) % R;
+    return d < k.cnt;
+}
+
 // kGate: 0 no output gate, 1 one gate per (head, channel), 2 one gate per head
-template <int kGate>
+// kCache: the block's queries against the cache (see PrefillArgs), else a prompt
+template <int kGate, bool kCache>
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_constant__ PrefillArgs a) {
     extern __shared__ __align__(16) char psmem_base[];
     char *smem = psmem_base + ((1024u - (smem_u32(psmem_base) & 1023u)) & 1023u);
@@ -166,6 +284,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     char *sKV = smem + 2 * kQTileBytes;                // [stages][K 32 KB | V 32 KB]
     char *sO = sKV + kPfStages * kPfStageBytes;        // [epilogue warp][2][32 rows][16 columns] bf16
     __shared__ uint64_t q_full, q_empty, kv_full[kPfStages], kv_empty[kPfStages];
+    __shared__ uint64_t vprep[kPfStages];             // cache mode: the stage's invalid V rows are zeroed
     __shared__ uint64_t s_full[2], p_full[2], o_done[2], mma_drained;
     // a work tile's rows handed from the softmax to the epilogue warps: (running
     // max, sum) per row, double-buffered by work tile; O of a head is free again
@@ -188,6 +307,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         for (int s = 0; s < kPfStages; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
+            mbar_init(&vprep[s], 1);
         }
         for (int h = 0; h < 2; ++h) {
             mbar_init(&s_full[h], 1);
@@ -201,7 +321,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         for (int w4 = 0; w4 < 4; ++w4) mbar_arrive(&turn[0]);   // head 0 takes the first turn
         for (int sl = 0; sl < kPfSlots; ++sl) {
             mbar_init(&work_full[sl], 1);
-            mbar_init(&work_empty[sl], 13);     // the MMA issuer, 8 softmax and 4 epilogue warps
+            // the MMA issuer, 8 softmax and 4 epilogue warps (and the V preparation warp)
+            mbar_init(&work_empty[sl], kCache ? 14 : 13);
         }
         mbar_init(&mma_drained, 1);
         fence_mbar_init();
@@ -222,12 +343,22 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&a.tm_q);
-            prefetch_tmap(&a.tm_k);
-            prefetch_tmap(&a.tm_v);
             prefetch_tmap(&a.tm_o);
+            if (!kCache) {             // (in cache mode a layer may lack one kind's maps)
+                prefetch_tmap(&a.tm_k);
+                prefetch_tmap(&a.tm_v);
+            }
             int jg = 0;
             bool ok = true;
-            int w = blockIdx.x;
+            // cache mode: work tiles with no key tile (a ring head's splits past the
+            // first, a split past a full head's rows) are passed over, unpublished
+            auto claim = [&](int wn) {
+                while (kCache && wn < a.n_work && pf_keys<kCache>(a, work_of(a, wn)).count() == 0)
+                    wn = a.work_counter != nullptr ? (int)gridDim.x + atomicAdd(a.work_counter, 1)
+                                                   : wn + (int)gridDim.x;
+                return wn;
+            };
+            int w = claim(blockIdx.x);
             for (int wc = 0; ok; ++wc) {
                 // publish the work tile (an index >= n_work tells the consumers to stop)
                 const int sl = wc % kPfSlots;
@@ -238,10 +369,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                 // claim the next one now: the atomic's latency hides behind this tile's loads.
                 // Claims follow the heaviest-first order, so every CTA takes the next
                 // tile when it is free (longest-processing-time-first scheduling)
-                const int w_next = a.work_counter != nullptr ? (int)gridDim.x + atomicAdd(a.work_counter, 1)
-                                                             : w + (int)gridDim.x;
+                const int w_next = claim(a.work_counter != nullptr ? (int)gridDim.x + atomicAdd(a.work_counter, 1)
+                                                                   : w + (int)gridDim.x);
                 const PfWork wk = work_of(a, w);
-                const TileList tl = tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window);
+                const PfKeys tl = pf_keys<kCache>(a, wk);
                 // Q of the previous work tile must no longer be read by the MMA
                 if (wc > 0 && !(ok = mbar_wait(&q_empty, (wc - 1) & 1))) break;
                 mbar_expect_tx(&q_full, 2 * kQTileBytes);
@@ -259,10 +390,21 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     const int row = tl.at(j) * kPfN;
                     char *kst = sKV + st * kPfStageBytes;
                     mbar_expect_tx(&kv_full[st], kPfStageBytes);
-                    for (int half = 0; half < 2; ++half) {
-                        tma_load_4d(kst + half * kKVHalfBytes, &a.tm_k, half * 64, wk.g, row, wk.b, &kv_full[st]);
-                        tma_load_4d(kst + kKVTileBytes + half * kKVHalfBytes, &a.tm_v, half * 64, wk.g, row,
-                                    wk.b, &kv_full[st]);
+                    if (kCache) {
+                        // the head's cache: (channel, row, rank, sequence)
+                        const bool full = a.kind[wk.g] == kKindFull;
+                        const CUtensorMap *mk = full ? &a.tm_k : &a.tm_k2, *mv = full ? &a.tm_v : &a.tm_v2;
+                        for (int half = 0; half < 2; ++half) {
+                            tma_load_4d(kst + half * kKVHalfBytes, mk, half * 64, row, a.rank[wk.g], wk.b, &kv_full[st]);
+                            tma_load_4d(kst + kKVTileBytes + half * kKVHalfBytes, mv, half * 64, row, a.rank[wk.g],
+                                        wk.b, &kv_full[st]);
+                        }
+                    } else {
+                        for (int half = 0; half < 2; ++half) {
+                            tma_load_4d(kst + half * kKVHalfBytes, &a.tm_k, half * 64, wk.g, row, wk.b, &kv_full[st]);
+                            tma_load_4d(kst + kKVTileBytes + half * kKVHalfBytes, &a.tm_v, half * 64, wk.g, row,
+                                        wk.b, &kv_full[st]);
+                        }
                     }
                 }
                 w = w_next;
@@ -305,7 +447,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             };
             auto kv_count = [&](int w) {
                 const PfWork wk = work_of(a, w);
-                return tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window).count();
+                return pf_keys<kCache>(a, wk).count();
             };
             int jg = 0, wc = 0, w = 0;
             bool ok = fetch(0, &w);
@@ -339,6 +481,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                         // the first PV of a work tile overwrites O: the epilogue of the
                         // previous one must have read it
                         if (j == 0 && wc > 0 && !(ok = mbar_wait(&o_free[h], (wc - 1) & 1))) break;
+                        // cache mode: the V rows of keys that hold no token are zeroed first
+                        if (kCache && h == 0 && !(ok = mbar_wait(&vprep[st], (jg / kPfStages) & 1))) break;
                         tc_fence_after();
                         issue_pv(h, st, j == 0);
                         if (more) {
@@ -389,7 +533,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             if (w >= a.n_work) break;
             const PfWork wk = work_of(a, w);
             const int kind = a.kind[wk.g];
-            const TileList tl = tile_list(kind, wk.t, a.L, a.sink, a.recent, a.window);
+            const PfKeys tl = pf_keys<kCache>(a, wk);
             const int n_kv = tl.count();
             const int i = wk.t * kPfM + r;             // query position
             const int hq = wk.h0 + h;
@@ -415,7 +559,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[q4 * 32]));
                 const int c0 = tl.at(j) * kPfN;
-                if (!tile_dense(kind, wk.t * kPfM, c0, a.sink, a.recent, a.window)) {
+                if (kCache) {
+                    if (!(kind == kKindFull && c0 + kPfN <= tl.n)) {
+                        uint32_t mw[4];
+                        cache_mask(a, tl, kind, i, c0, mw);
+#pragma unroll
+                        for (int cc = 0; cc < 128; ++cc)
+                            if (!((mw[cc >> 5] >> (cc & 31)) & 1u)) sr[cc] = __float_as_uint(-INFINITY);
+                    }
+                } else if (!tile_dense(kind, wk.t * kPfM, c0, tl.sink, a.recent, a.window)) {
                     // the row's attended keys among the tile's 128 columns as two
                     // 64-bit masks built from their one or two ranges
                     const int di = i - c0;                     // the diagonal's column
@@ -425,7 +577,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                         hi0 = di;
                     } else if (kind == kKindStreaming) {
                         lo0 = 0;
-                        hi0 = min(di, a.sink - 1 - c0);
+                        hi0 = min(di, tl.sink - 1 - c0);
                         lo1 = di - a.recent + 1;
                         hi1 = di;
                     } else {
@@ -547,7 +699,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             if (lane == 0) mbar_arrive(&work_empty[sl]);
             if (w >= a.n_work) break;
             const PfWork wk = work_of(a, w);
-            jg += tile_list(a.kind[wk.g], wk.t, a.L, a.sink, a.recent, a.window).count();
+            jg += pf_keys<kCache>(a, wk).count();
             const int i = wk.t * kPfM + r;             // query position
             const int row0 = wk.t * kPfM + quarter * 32;   // first row of this warp's boxes
             for (int h = 0; h < 2 && ok; ++h) {
@@ -609,14 +761,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     fence_proxy_async_smem();              // visible to the copy engine
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_4d(&a.tm_o, stage, chunk * 16, hq, row0, wk.b);
+                        tma_store_4d(&a.tm_o, stage, chunk * 16, hq, row0, wk.s * a.batch + wk.b);
                         bulk_commit_group();
                     }
                     g0 = n0;
                     g1 = n1;
                 }
                 if (a.lse != nullptr && i < a.L)
-                    a.lse[((size_t)wk.b * a.hq + hq) * a.L + i] =
+                    a.lse[((size_t)(wk.s * a.batch + wk.b) * a.hq + hq) * a.L + i] =
                         l_exact > 0.f ? (m_run + __log2f(l_exact)) * kLn2F : -INFINITY;
                 // O of this head has been read: the next work tile's first PV may overwrite it
                 tc_fence_before();
@@ -627,8 +779,50 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
         if (lane == 0) bulk_wait_all();                    // this warp's O stores have landed
         __syncwarp();
     } else {
-        // warps 14 and 15 hold no role: they only give up their registers
+        // warps 14 and 15 give up their registers; in cache mode warp 14 zeroes,
+        // in each loaded stage, the V rows of keys that hold no token (cache memory
+        // past a sequence's tokens is never written, and 0 x NaN would reach O)
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfOtherRegs));
+        if (kCache && warp == 14) {
+            int jg = 0;
+            bool ok = true;
+            for (int wc = 0; ok; ++wc) {
+                const int sl = wc % kPfSlots;
+                const bool have = mbar_wait(&work_full[sl], (wc / kPfSlots) & 1);
+                __syncwarp();
+                if (!__all_sync(0xffffffffu, have)) break;
+                const int w = work_slot[sl];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&work_empty[sl]);
+                if (w >= a.n_work) break;
+                const PfWork wk = work_of(a, w);
+                const int kind = a.kind[wk.g];
+                const PfKeys tl = pf_keys<kCache>(a, wk);
+                const int n_kv = tl.count();
+                for (int j = 0; j < n_kv; ++j, ++jg) {
+                    const int st = jg % kPfStages;
+                    const bool got = mbar_wait(&kv_full[st], (jg / kPfStages) & 1);
+                    __syncwarp();
+                    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                    char *vt = sKV + st * kPfStageBytes + kKVTileBytes;
+                    const int c0 = tl.at(j) * kPfN;
+#pragma unroll 1
+                    for (int k = lane; k < kPfN; k += 32) {
+                        if (cache_key_valid(a, tl, kind, c0 + k)) continue;
+                        // row k of V: 128 bytes in each 64-column half (swizzled within the row)
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            reinterpret_cast<uint4 *>(vt + k * 128)[q] = make_uint4(0, 0, 0, 0);
+                            reinterpret_cast<uint4 *>(vt + kKVHalfBytes + k * 128)[q] = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    fence_proxy_async_smem();       // the zeroed rows, for the tensor core
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&vprep[st]);
+                }
+            }
+            __syncwarp();
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -684,10 +878,84 @@ inline bool make_tmap(CUtensorMap *m, const void *base, int B, int L, int H, int
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The cache as a 4-D tensor (128, rows, heads of the kind, B) loaded in
+// 64-column x 128-row boxes with the 128-byte swizzle: (channel, row, rank, b).
+inline bool make_cache_tmap(CUtensorMap *m, const void *base, int B, int heads, int64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)rows, (cuuint64_t)heads, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {256, (cuuint64_t)rows * 256, (cuuint64_t)rows * heads * 256};
+    const cuuint32_t box[4] = {64, (cuuint32_t)kPfN, 1, 1};
+    const cuuint32_t elem[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, elem,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launches prefill_fwd<kGate, kCache> for the arguments a (maps, geometry and
+// pointers set; the work list is filled in here).
+template <int kGate, bool kCache>
+inline int launch_prefill_kernel(PrefillArgs &a, int B, int32_t *work_counter, cudaStream_t stream, char *err,
+                                 size_t err_len) {
+    void (*kernel)(PrefillArgs) = prefill_fwd<kGate, kCache>;
+    // set once per device and instantiation (atomic: host threads may launch concurrently)
+    static std::atomic<bool> smem_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !smem_set[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmem) !=
+            cudaSuccess) {
+            snprintf(err, err_len, "cudaFuncSetAttribute(prefill_fwd) failed");
+            return DUO_ERR_CUDA;
+        }
+        // the warps' register split adds up to exactly the launch allocation: a
+        // build with another register count would leave a setmaxnreg.inc waiting
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.numRegs != kPfLaunchRegs) {
+            snprintf(err, err_len, "prefill_fwd was built with %d registers per thread, not %d",
+                     fa.numRegs, kPfLaunchRegs);
+            return DUO_ERR_CUDA;
+        }
+        if (dev >= 0 && dev < 64) smem_set[dev].store(true, std::memory_order_release);
+    }
+    a.batch = B;
+    if (a.kv_splits < 1) {                 // prompt mode: one split holding every key tile
+        a.kv_splits = 1;
+        a.split_tiles = INT32_MAX / 2;
+    }
+    a.batch_pairs = B * (a.hq / 2);
+    const int64_t n_work = (int64_t)a.batch_pairs * a.n_qtiles * a.kv_splits;
+    // the counter runs up to n_work + 2 * grid
+    if (n_work > INT32_MAX - 4096) {
+        snprintf(err, err_len, "too many query tiles for one prefill launch");
+        return DUO_ERR_INVALID_ARG;
+    }
+    a.n_work = (int32_t)n_work;
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const unsigned grid = (unsigned)std::min<int64_t>(n_work, sms);
+    a.work_counter = work_counter;
+    if (work_counter != nullptr && cudaMemsetAsync(work_counter, 0, sizeof(int32_t), stream) != cudaSuccess) {
+        snprintf(err, err_len, "zeroing the prefill work counter failed");
+        return DUO_ERR_CUDA;
+    }
+    kernel<<<grid, kPfThreads, kPfSmem, stream>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        snprintf(err, err_len, "prefill_fwd launch: %s", cudaGetErrorString(e));
+        return DUO_ERR_CUDA;
+    }
+    return DUO_OK;
+}
+
+// Prompt mode: q, k, v [B][L][H][128].  block_start (device, [B]) or null: the
+// position each sequence's keys start at, which shifts the sink (a block of
+// queries continuing cached tokens); the sink logit, if any, is included.
 inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_full, int sink,
                           int ring, const void *q, const void *k, const void *v, int32_t L, void *out,
                           float *lse, int32_t *work_counter, int gate_mode, const void *gate,
-                          int withhold_tile, cudaStream_t stream, char *err, size_t err_len) {
+                          int withhold_tile, cudaStream_t stream, char *err, size_t err_len,
+                          const int32_t *block_start = nullptr) {
     PrefillArgs a;
     memset(&a, 0, sizeof a);
     const int B = p->batch;
@@ -710,52 +978,63 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     a.window = sliding ? ring : 0;
     a.scale_log2 = p->softmax_scale * kLog2eF;
     a.withhold_tile = withhold_tile;
+    a.seq_len = block_start;
     for (int g = 0; g < p->num_kv_heads; ++g)
         a.kind[g] = sliding ? kKindSliding : (is_full[g] ? kKindFull : kKindStreaming);
-    void (*kernel)(PrefillArgs) = gate_mode == 1 ? prefill_fwd<1> : gate_mode == 2 ? prefill_fwd<2> : prefill_fwd<0>;
-    // set once per device and instantiation (atomic: host threads may launch concurrently)
-    static std::atomic<bool> smem_set[3][64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !smem_set[gate_mode][dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmem) !=
-            cudaSuccess) {
-            snprintf(err, err_len, "cudaFuncSetAttribute(prefill_fwd) failed");
-            return DUO_ERR_CUDA;
-        }
-        // the warps' register split adds up to exactly the launch allocation: a
-        // build with another register count would leave a setmaxnreg.inc waiting
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.numRegs != kPfLaunchRegs) {
-            snprintf(err, err_len, "prefill_fwd was built with %d registers per thread, not %d",
-                     fa.numRegs, kPfLaunchRegs);
-            return DUO_ERR_CUDA;
-        }
-        if (dev >= 0 && dev < 64) smem_set[gate_mode][dev].store(true, std::memory_order_release);
-    }
-    a.batch_pairs = B * (p->num_q_heads / 2);
-    const int64_t n_work = (int64_t)a.batch_pairs * a.n_qtiles;
-    // the counter runs up to n_work + 2 * grid
-    if (n_work > INT32_MAX - 4096) {
-        snprintf(err, err_len, "too many query tiles for one prefill launch");
-        return DUO_ERR_INVALID_ARG;
-    }
-    a.n_work = (int32_t)n_work;
-    int sms = 148;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const unsigned grid = (unsigned)std::min<int64_t>(n_work, sms);
-    a.work_counter = work_counter;
-    if (work_counter != nullptr && cudaMemsetAsync(work_counter, 0, sizeof(int32_t), stream) != cudaSuccess) {
-        snprintf(err, err_len, "zeroing the prefill work counter failed");
+    if (gate_mode == 1) return launch_prefill_kernel<1, false>(a, B, work_counter, stream, err, err_len);
+    if (gate_mode == 2) return launch_prefill_kernel<2, false>(a, B, work_counter, stream, err, err_len);
+    return launch_prefill_kernel<0, false>(a, B, work_counter, stream, err, err_len);
+}
+
+// Cache mode: the block q [B][L][Hq][128] against the cache as it stands (no
+// output gate, no sink logit: those are folded in once the block's own keys
+// are added).  full_k/v [B][n_full][capacity][128], strm_k/v [B][n_ring][slots][128].
+// A full head's cached key tiles are cut into kv_splits runs of split_tiles
+// tiles: out [kv_splits][B][L][Hq][128], lse [kv_splits][B][Hq][L] (ring heads:
+// slice 0 only).
+inline int launch_prefill_cache(const duo_params *p, bool sliding, const int8_t *is_full, const int8_t *rank,
+                                int n_full, int n_ring, int sink, int ring, int64_t capacity,
+                                const void *full_k, const void *full_v, const void *strm_k, const void *strm_v,
+                                const int32_t *seq_len, const int32_t *ring_head, const void *q, int32_t L,
+                                int kv_splits, int split_tiles, void *out, float *lse, int32_t *work_counter,
+                                int withhold_tile, cudaStream_t stream, char *err, size_t err_len) {
+    PrefillArgs a;
+    memset(&a, 0, sizeof a);
+    const int B = p->batch;
+    const int slots = (sliding ? 0 : sink) + ring;
+    // out holds one [B][L][Hq][128] slice per split: the map sees kv_splits * B sequences
+    bool okm = make_tmap(&a.tm_q, q, B, L, p->num_q_heads, kPfM) &&
+               make_out_tmap(&a.tm_o, out, B * kv_splits, L, p->num_q_heads);
+    if (n_full > 0)
+        okm = okm && make_cache_tmap(&a.tm_k, full_k, B, n_full, capacity) &&
+              make_cache_tmap(&a.tm_v, full_v, B, n_full, capacity);
+    if (n_ring > 0)
+        okm = okm && make_cache_tmap(&a.tm_k2, strm_k, B, n_ring, slots) &&
+              make_cache_tmap(&a.tm_v2, strm_v, B, n_ring, slots);
+    if (!okm) {
+        snprintf(err, err_len, "cuTensorMapEncodeTiled failed (driver entry point unavailable?)");
         return DUO_ERR_CUDA;
     }
-    kernel<<<grid, kPfThreads, kPfSmem, stream>>>(a);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) {
-        snprintf(err, err_len, "prefill_fwd launch: %s", cudaGetErrorString(e));
-        return DUO_ERR_CUDA;
+    a.lse = lse;
+    a.L = L;
+    a.hq = p->num_q_heads;
+    a.hkv = p->num_kv_heads;
+    a.n_qtiles = (L + kPfM - 1) / kPfM;
+    // ring heads: sink S and ring R (a sliding layer: no sink, R = the window)
+    a.sink = sliding ? 0 : sink;
+    a.recent = ring;
+    a.scale_log2 = p->softmax_scale * kLog2eF;
+    a.withhold_tile = withhold_tile;
+    a.seq_len = seq_len;
+    a.ring_head = ring_head;
+    a.capacity = (int32_t)std::min<int64_t>(capacity, INT32_MAX);
+    a.kv_splits = kv_splits;
+    a.split_tiles = split_tiles;
+    for (int g = 0; g < p->num_kv_heads; ++g) {
+        a.kind[g] = sliding ? kKindSliding : (is_full[g] ? kKindFull : kKindStreaming);
+        a.rank[g] = rank[g];
     }
-    return DUO_OK;
+    return launch_prefill_kernel<0, true>(a, B, work_counter, stream, err, err_len);
 }
 
 }  // namespace duo

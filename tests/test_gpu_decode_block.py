@@ -7,6 +7,8 @@ sequences that are empty, below the sink, filling the ring and past it, a
 sliding layer with sink logits, an output gate, and a 32768-token context.
 The cache must be left untouched.  Tolerances as the one-token decode.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -110,17 +112,19 @@ def test_block_decode_bench_shape_sampled(cuda_device):
     assert_close(got_o, ref_o, got_l, ref_l, "verify_b32 shape")
 
 
-def test_block_decode_rejects_long_blocks(cuda_device):
+def test_block_decode_rejects_empty_blocks(cuda_device):
     p, o = layers(1, full_mask=(1,) * 8)
     cache = random_cache(p, 64, [10], [0], seed=109)
-    q = torch.zeros((1, 9, 48, 128), dtype=torch.bfloat16, device="cuda")
-    kv = torch.zeros((1, 9, 8, 128), dtype=torch.bfloat16, device="cuda")
-    out = torch.zeros_like(q)
+    q = torch.zeros((1, 1, 48, 128), dtype=torch.bfloat16, device="cuda")
+    lib = duo.load_library()
     ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
-    with pytest.raises(duo.DuoError) as e:
-        duo.duo_attn_decode_block(p, cache, q, kv, kv, 64, out, None, ws)
-    assert e.value.code == duo.DUO_ERR_UNSUPPORTED
-    assert duo.duo_decode_block_workspace_bytes(p, 9, 64) == 0
+    pc, cc = p.as_c(), cache.as_c(p)
+    rc = lib.duo_attn_decode_block(ctypes.byref(pc), ctypes.byref(cc), q.data_ptr(), q.data_ptr(),
+                                   q.data_ptr(), 0, 64, q.data_ptr(), None, ws.data_ptr(), ws.numel(), None,
+                                   None)
+    assert rc == duo.DUO_ERR_UNSUPPORTED
+    assert duo.duo_decode_block_workspace_bytes(p, 0, 64) == 0
+    assert duo.duo_decode_block_workspace_bytes(p, 9, 64) > 0
 
 
 def test_block_decode_repeat_is_bitwise_stable(cuda_device):
@@ -153,3 +157,92 @@ def test_block_decode_repeat_is_bitwise_stable(cuda_device):
         assert duo.duo_get_device_status() == duo.DUO_OK
         assert torch.equal(out, ref_out), f"call {i}: output differs"
         assert torch.equal(lse, ref_lse), f"call {i}: lse differs"
+
+
+# ---------------------------------------------------------------- long blocks
+# q_len > 8: chunked prefill.  The two-pass path (prefill over the cached keys,
+# prefill over the block's own keys, folded by their log-sum-exps) against the
+# same oracle.
+
+@pytest.mark.parametrize("q_len", [9, 130, 300])
+def test_long_block_duo_layer(cuda_device, q_len):
+    p, o = layers(6, full_mask=(1, 0, 0, 1, 0, 1, 1, 0))
+    seq = [0, 5, 64, 200, 320, 3000]
+    rh = [0, 0, 0, 136, 0, 77]
+    cache = random_cache(p, 3000, seq, rh, seed=180 + q_len)
+    block_case(p, o, cache, q_len, seed=190 + q_len, max_seq_len=3000)
+
+
+@pytest.mark.parametrize("q_len", [200, 700])
+def test_long_block_sliding_layer_with_sink(cuda_device, q_len):
+    sig = inputs.randn_f32((48,), 200)
+    p, o = layers(3, window=512, sink_logit=sig)
+    seq = [3, 511, 9000]
+    cache = random_cache(p, 64, seq, [0, 0, 300], seed=201)
+    block_case(p, o, cache, q_len, seed=202 + q_len, max_seq_len=9000)
+
+
+@pytest.mark.parametrize("mode", ["per_element", "per_head"])
+def test_long_block_output_gate(cuda_device, mode):
+    p, o = layers(2, full_mask=(0, 1, 0, 0, 0, 0, 1, 0))
+    cache = random_cache(p, 700, [700, 33], [10, 0], seed=203)
+    shape = (2, 150, 48, 128) if mode == "per_element" else (2, 150, 48)
+    g = (inputs.randn_f32(shape, 204) * 2.0).to("cuda", torch.bfloat16)
+    gm = oracle.GATE_PER_ELEMENT if mode == "per_element" else oracle.GATE_PER_HEAD
+    block_case(p, o, cache, 150, seed=205, max_seq_len=700, gate=g, gate_mode=gm)
+
+
+def test_long_block_ignores_unwritten_cache_memory(cuda_device):
+    """Cache rows past a sequence's tokens and ring slots that hold no token are
+    filled with NaN: the long path must never let them reach an output (their V
+    rows are zeroed before the PV product, their scores masked)."""
+    p, o = layers(3, full_mask=(1, 0, 0, 0, 0, 0, 1, 0))
+    seq, rh = [0, 40, 300], [0, 0, 17]
+    cache = random_cache(p, 512, seq, rh, seed=206)
+    nan = float("nan")
+    S, R = 64, 256
+    for b, n in enumerate(seq):
+        cache.full_k[b, :, n:] = nan
+        cache.full_v[b, :, n:] = nan
+        cache.strm_k[b, :, min(n, S):S] = nan
+        cache.strm_v[b, :, min(n, S):S] = nan
+        cnt = min(max(n - S, 0), R)
+        for r in range(R):
+            if (rh[b] - 1 - r) % R >= cnt:
+                cache.strm_k[b, :, S + r] = nan
+                cache.strm_v[b, :, S + r] = nan
+    block_case(p, o, cache, 140, seed=207, max_seq_len=512)
+
+
+@pytest.mark.slow
+def test_long_block_bench_shape_sampled(cuda_device):
+    """The chunk_32k line's call: a 4096-token chunk after 28672 cached tokens,
+    prefill_16k's head mask (the full heads' cached keys cut into several
+    slices); every query head of 24 seeded chunk positions against the oracle,
+    the cache untouched, every output finite."""
+    w = inputs.workload("prefill_16k")
+    n, C = 28672, 4096
+    p, o = layers(1, full_mask=w.full_mask)
+    cache = random_cache(p, n, [n], [141], seed=210)
+    q = inputs.randn_bf16((1, C, 48, 128), 211, "cuda")
+    kn = inputs.randn_bf16((1, C, 8, 128), 212, "cuda")
+    vn = inputs.randn_bf16((1, C, 8, 128), 213, "cuda")
+    out = torch.full((1, C, 48, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((1, C, 48), float("nan"), dtype=torch.float32, device="cuda")
+    nb = duo.duo_decode_block_workspace_bytes(p, C, n)
+    ws = torch.full(((nb + 255) // 256 * 256,), 0x7f, dtype=torch.uint8, device="cuda")
+    before = (cache.seq_len.clone(), cache.ring_head.clone(), cache.full_k[0, 0, :64].clone())
+    duo.duo_attn_decode_block(p, cache, q, kn, vn, n, out, lse, ws)
+    torch.cuda.synchronize()
+    assert duo.duo_get_device_status() == duo.DUO_OK
+    assert torch.equal(before[0], cache.seq_len) and torch.equal(before[1], cache.ring_head)
+    assert torch.equal(before[2], cache.full_k[0, 0, :64])
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    snap = host_cache(o, cache)
+    pos = np.sort(np.random.default_rng(214).choice(C, size=24, replace=False))
+    pos[0], pos[-1] = 0, C - 1
+    rows = [int(t) * 48 + h for t in pos for h in range(48)]
+    ref_o, ref_l = oracle.attn_decode_block(o, snap, inputs.bits(q), inputs.bits(kn), inputs.bits(vn), rows=rows)
+    got_o = out[0, pos].reshape(-1, 128)
+    got_l = lse[0, pos].reshape(-1)
+    assert_close(got_o, ref_o, got_l, ref_l, "chunk_32k shape")

@@ -126,8 +126,9 @@ def test_prep_writes_stay_inside(cuda_device):
     assert not np.array_equal(inputs.bits(k), k_in)      # k was rewritten
 
 
-def test_verify_block_writes_stay_inside(cuda_device):
-    B, q_len = 3, 8
+@pytest.mark.parametrize("q_len", [8, 150])
+def test_verify_block_writes_stay_inside(cuda_device, q_len):
+    B = 3
     g = Guarded()
     p, o = layers(B, full_mask=MASK)
     seq = [0, 300, 2000]

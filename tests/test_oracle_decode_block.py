@@ -7,6 +7,8 @@ n..n+k-1 against the cache of the first n tokens, plus the block's own keys.
   only the softmax): full, streaming and sliding heads, with and without a
   sink logit, for n below the sink, inside the ring's fill and far past it.
 * k = 1 must equal "append the token, then one-token decode".
+* Blocks longer than the ring and the window (chunked prefill) too: their
+  later queries see none of the cached ring slots.
 """
 import numpy as np
 import pytest
@@ -28,7 +30,8 @@ def layer(B, kind, sink, recent, window, sigma):
 
 
 @pytest.mark.parametrize("kind", ["duo", "sliding"])
-@pytest.mark.parametrize("n,k", [(0, 3), (2, 4), (5, 1), (9, 6), (23, 8), (60, 5)])
+@pytest.mark.parametrize("n,k", [(0, 3), (2, 4), (5, 1), (9, 6), (23, 8), (60, 5),
+                                 (0, 20), (3, 33), (11, 17), (40, 25)])
 @pytest.mark.parametrize("with_sink", [False, True])
 def test_block_decode_equals_prefill_rows(kind, n, k, with_sink):
     B, sink, recent, window = 2, 4, 6, 7
