@@ -672,6 +672,8 @@ __global__ void __launch_bounds__(kMergeThreads) decode_block_merge(const __grid
 // (prefill_fwd's prompt mode, which also adds the sink logit).  Each part is
 // normalised by its own sum and rounded to bf16; they are folded here by their
 // sums: O = sum_p e^Lp Op / sum_p e^Lp, LSE = ln sum_p e^Lp.
+constexpr int kMaxLongSplits = 8;     // slices of a full head's cached keys in a long block
+
 struct CombineArgs {
     const __nv_bfloat16 *oa, *ob;   // [S][B][C][Hq][D], [B][C][Hq][D]
     const float *lse_a, *lse_b;     // [S][B][Hq][C], [B][Hq][C]
@@ -699,18 +701,32 @@ __global__ void __launch_bounds__(kMergeThreads) block_combine(const __grid_cons
     }
     const size_t slice_o = (size_t)a.batch * a.C * a.hq * kD, slice_l = (size_t)a.batch * a.hq * a.C;
     const size_t li = ((size_t)b * a.hq + h) * a.C + t;
-    float M = a.lse_b[li] * kLog2eF;
-    for (int s = 0; s < parts; ++s) M = fmaxf(M, a.lse_a[s * slice_l + li] * kLog2eF);
+    // every part's log-sum-exp and four outputs are loaded at once (part
+    // kMaxLongSplits is the block's own)
+    float l[kMaxLongSplits + 1];
+    uint2 ov[kMaxLongSplits + 1];
+#pragma unroll
+    for (int s = 0; s <= kMaxLongSplits; ++s) {
+        const bool own = s == kMaxLongSplits;
+        l[s] = -INFINITY;
+        ov[s] = make_uint2(0u, 0u);
+        if (own || s < parts) {
+            l[s] = (own ? a.lse_b[li] : a.lse_a[s * slice_l + li]) * kLog2eF;
+            ov[s] = *reinterpret_cast<const uint2 *>((own ? a.ob : a.oa + s * slice_o) + row * kD + c4);
+        }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s <= kMaxLongSplits; ++s) M = fmaxf(M, l[s]);
     float den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
     if (M != -INFINITY) {
-        for (int s = 0; s <= parts; ++s) {          // the cached slices, then the block's own part
-            const bool own = s == parts;
-            const float l = (own ? a.lse_b[li] : a.lse_a[s * slice_l + li]) * kLog2eF;
-            if (l == -INFINITY) continue;
-            const float wgt = ex2_approx(l - M);
+#pragma unroll
+        for (int s = 0; s <= kMaxLongSplits; ++s) {
+            if (l[s] == -INFINITY) continue;
+            const float wgt = ex2_approx(l[s] - M);
             float f[4];
-            unpack_bf16x4(*reinterpret_cast<const uint2 *>((own ? a.ob : a.oa + s * slice_o) + row * kD + c4), f);
+            unpack_bf16x4(ov[s], f);
             den += wgt;
             num.x += wgt * f[0];
             num.y += wgt * f[1];

@@ -609,9 +609,11 @@ int duo_cache_bytes(const duo_params *params, int64_t capacity, int64_t seq_len,
 
 // ------------------------------------------------------------------ block decode
 // A block longer than kMaxBlock tokens.  The full heads' cached keys are cut
-// into kv_splits runs so that the pass over the cache has enough work tiles for
-// the SMs: the count minimises the estimated makespan of the persistent CTAs
-// (a work tile costs its key tiles plus two for its fill and epilogue).
+// into kv_splits runs (at most kMaxLongSplits: block_combine reads one slice per
+// run) so that the pass over the cache has enough work tiles for the SMs: the
+// count minimises the estimated makespan of the persistent CTAs, all work spread
+// evenly plus the last work tile (a work tile costs its key tiles plus two for
+// its fill and epilogue; a ring head's about five).
 struct LongBlockPlan {
     int kv_splits, split_tiles;
     size_t o_bytes, l_bytes, total;     // one bf16 [B][q_len][Hq][D] slice, one fp32 [B][Hq][q_len] slice
@@ -627,9 +629,9 @@ LongBlockPlan long_block_plan(const duo_params *p, const Layout &L, int64_t q_le
     w.split_tiles = (int)tiles;
     if (units > 0) {
         double best = 1e300;
-        for (int64_t s = 1; s <= std::min<int64_t>(tiles, 64); ++s) {
+        for (int64_t s = 1; s <= std::min<int64_t>(tiles, duo::kMaxLongSplits); ++s) {
             const int64_t chunk = (tiles + s - 1) / s;
-            const double span = (double)((units * s + ring_units + sms - 1) / sms) * (double)(chunk + 2);
+            const double span = ((double)units * s * (chunk + 2) + 5.0 * ring_units) / sms + (double)(chunk + 2);
             if (span < best - 1e-9) {
                 best = span;
                 w.kv_splits = (int)s;
@@ -673,13 +675,16 @@ int long_block(const duo_params *params, const Layout &L, const duo_cache *cache
     float *lb = (float *)((char *)la + (size_t)pl.kv_splits * pl.l_bytes);
     int32_t *ca = (int32_t *)((char *)lb + pl.l_bytes), *cb = ca + 64;
     char err[256];
+    // both passes' work counters at once: no memset between the passes, so that the
+    // second can start on the SMs the first leaves
+    if (cudaMemsetAsync(ca, 0, 2 * 256, st) != cudaSuccess) return fail(DUO_ERR_CUDA, "zeroing the work counters failed");
     int rc = duo::launch_prefill_cache(params, L.sliding, L.heads.is_full, L.heads.rank, L.n_full, L.n_ring,
                                        L.sink, L.ring, L.n_full > 0 ? cache->capacity : 0, cache->full_k,
                                        cache->full_v, cache->strm_k, cache->strm_v, cache->seq_len, cache->ring_head,
                                        q, q_len, pl.kv_splits, pl.split_tiles, oa, la, ca, -1, st, err, sizeof err);
     if (rc) return fail(rc, "%s", err);
     rc = duo::launch_prefill(params, L.sliding, L.heads.is_full, L.sink, L.ring, q, k_new, v_new, q_len, ob, lb,
-                             cb, 0, nullptr, -1, st, err, sizeof err, cache->seq_len);
+                             cb, 0, nullptr, -1, st, err, sizeof err, cache->seq_len, false, true);
     if (rc) return fail(rc, "%s", err);
     duo::CombineArgs c;
     memset(&c, 0, sizeof c);

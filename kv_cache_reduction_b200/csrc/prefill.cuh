@@ -335,6 +335,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // cache mode: the next grid (the block's own keys) may take each SM this CTA
+    // leaves; it does not read what this grid writes
+    if (kCache) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = tmem_base;
     // each role sets its register budget first thing in its own branch, so that
     // the compiler allocates that branch's code within it
@@ -824,6 +827,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
             __syncwarp();
         }
     }
+    // launched as a programmatic dependent (the block's own keys after the pass over
+    // the cache): the grid completes only after the one before it, whose results
+    // the next kernel reads (a no-op otherwise)
+    if (!kCache) pdl_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == kPfMmaWarp) {
@@ -894,9 +901,11 @@ inline bool make_cache_tmap(CUtensorMap *m, const void *base, int B, int heads, 
 
 // Launches prefill_fwd<kGate, kCache> for the arguments a (maps, geometry and
 // pointers set; the work list is filled in here).
+// zero: zero the work counter on the stream first (else the caller has);
+// pdl: launch as a programmatic dependent of the previous kernel.
 template <int kGate, bool kCache>
 inline int launch_prefill_kernel(PrefillArgs &a, int B, int32_t *work_counter, cudaStream_t stream, char *err,
-                                 size_t err_len) {
+                                 size_t err_len, bool zero = true, bool pdl = false) {
     void (*kernel)(PrefillArgs) = prefill_fwd<kGate, kCache>;
     // set once per device and instantiation (atomic: host threads may launch concurrently)
     static std::atomic<bool> smem_set[64] = {};
@@ -935,11 +944,25 @@ inline int launch_prefill_kernel(PrefillArgs &a, int B, int32_t *work_counter, c
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const unsigned grid = (unsigned)std::min<int64_t>(n_work, sms);
     a.work_counter = work_counter;
-    if (work_counter != nullptr && cudaMemsetAsync(work_counter, 0, sizeof(int32_t), stream) != cudaSuccess) {
+    if (zero && work_counter != nullptr && cudaMemsetAsync(work_counter, 0, sizeof(int32_t), stream) != cudaSuccess) {
         snprintf(err, err_len, "zeroing the prefill work counter failed");
         return DUO_ERR_CUDA;
     }
-    kernel<<<grid, kPfThreads, kPfSmem, stream>>>(a);
+    if (pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kPfThreads);
+        cfg.dynamicSmemBytes = kPfSmem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaLaunchKernelEx(&cfg, kernel, a);
+    } else {
+        kernel<<<grid, kPfThreads, kPfSmem, stream>>>(a);
+    }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
         snprintf(err, err_len, "prefill_fwd launch: %s", cudaGetErrorString(e));
@@ -955,7 +978,7 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
                           int ring, const void *q, const void *k, const void *v, int32_t L, void *out,
                           float *lse, int32_t *work_counter, int gate_mode, const void *gate,
                           int withhold_tile, cudaStream_t stream, char *err, size_t err_len,
-                          const int32_t *block_start = nullptr) {
+                          const int32_t *block_start = nullptr, bool zero = true, bool pdl = false) {
     PrefillArgs a;
     memset(&a, 0, sizeof a);
     const int B = p->batch;
@@ -981,9 +1004,9 @@ inline int launch_prefill(const duo_params *p, bool sliding, const int8_t *is_fu
     a.seq_len = block_start;
     for (int g = 0; g < p->num_kv_heads; ++g)
         a.kind[g] = sliding ? kKindSliding : (is_full[g] ? kKindFull : kKindStreaming);
-    if (gate_mode == 1) return launch_prefill_kernel<1, false>(a, B, work_counter, stream, err, err_len);
-    if (gate_mode == 2) return launch_prefill_kernel<2, false>(a, B, work_counter, stream, err, err_len);
-    return launch_prefill_kernel<0, false>(a, B, work_counter, stream, err, err_len);
+    if (gate_mode == 1) return launch_prefill_kernel<1, false>(a, B, work_counter, stream, err, err_len, zero, pdl);
+    if (gate_mode == 2) return launch_prefill_kernel<2, false>(a, B, work_counter, stream, err, err_len, zero, pdl);
+    return launch_prefill_kernel<0, false>(a, B, work_counter, stream, err, err_len, zero, pdl);
 }
 
 // Cache mode: the block q [B][L][Hq][128] against the cache as it stands (no
@@ -1034,7 +1057,7 @@ inline int launch_prefill_cache(const duo_params *p, bool sliding, const int8_t 
         a.kind[g] = sliding ? kKindSliding : (is_full[g] ? kKindFull : kKindStreaming);
         a.rank[g] = rank[g];
     }
-    return launch_prefill_kernel<0, true>(a, B, work_counter, stream, err, err_len);
+    return launch_prefill_kernel<0, true>(a, B, work_counter, stream, err, err_len, false);   // zeroed by the caller
 }
 
 }  // namespace duo
