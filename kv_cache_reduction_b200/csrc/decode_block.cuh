@@ -685,13 +685,25 @@ struct CombineArgs {
     int8_t is_full[64];             // per KV head: its cached keys come in split slices (else one)
 };
 
-// One warp per (sequence, block token, query head), four output dimensions per thread.
-__global__ void __launch_bounds__(kMergeThreads) block_combine(const __grid_constant__ CombineArgs a) {
-    const int hh = threadIdx.x >> 5, c4 = (threadIdx.x & 31) * 4;
-    const int64_t row = (int64_t)blockIdx.x * kGroup + hh;          // (b * C + t) * Hq + h
-    const int h = (int)(row % a.hq);
-    const int64_t bt = row / a.hq;
-    const int64_t t = bt % a.C, b = bt / a.C;
+// kCombineDims output dimensions per thread, 128 / kCombineDims threads per
+// output row (sequence, block token, query head): the per-row work (indices,
+// the parts' log-sum-exps and weights) is shared by a row's threads, and every
+// part's 16-byte loads are issued at once.  Rows are (b * C + t) * Hq + h,
+// fewer than 2^31 (the host checks), so the index arithmetic stays 32-bit.
+#ifndef DUO_COMBINE_DIMS
+#define DUO_COMBINE_DIMS 8
+#endif
+constexpr int kCombineDims = DUO_COMBINE_DIMS, kCombineVec = kCombineDims / 8;
+constexpr int kCombineRowThreads = kD / kCombineDims, kCombineThreads = 256;
+constexpr int kCombineRows = kCombineThreads / kCombineRowThreads;
+
+__global__ void __launch_bounds__(kCombineThreads) block_combine(const __grid_constant__ CombineArgs a) {
+    const uint32_t rows = (uint32_t)a.batch * (uint32_t)a.C * (uint32_t)a.hq;
+    const uint32_t row = blockIdx.x * kCombineRows + threadIdx.x / kCombineRowThreads;
+    const int c16 = (threadIdx.x % kCombineRowThreads) * kCombineDims;
+    if (row >= rows) return;
+    const uint32_t h = row % (uint32_t)a.hq, bt = row / (uint32_t)a.hq;
+    const uint32_t t = bt % (uint32_t)a.C, b = bt / (uint32_t)a.C;
     // a full head's slices: as many as its cached rows fill (prefill_fwd passes
     // over the rest unwritten); split 0 always, maybe with no key
     int parts = 1;
@@ -699,45 +711,73 @@ __global__ void __launch_bounds__(kMergeThreads) block_combine(const __grid_cons
         const int tiles = (min(max(a.seq_len[b], 0), a.capacity) + 127) / 128;
         parts = min(a.kv_splits, max(1, (tiles + a.split_tiles - 1) / a.split_tiles));
     }
-    const size_t slice_o = (size_t)a.batch * a.C * a.hq * kD, slice_l = (size_t)a.batch * a.hq * a.C;
+    const size_t slice_o = (size_t)rows * kD, slice_l = rows;
     const size_t li = ((size_t)b * a.hq + h) * a.C + t;
-    // every part's log-sum-exp and four outputs are loaded at once (part
-    // kMaxLongSplits is the block's own)
+    const size_t oi = (size_t)row * kD + c16;
+    // every part's log-sum-exp and outputs (part kMaxLongSplits is the block's own)
     float l[kMaxLongSplits + 1];
-    uint2 ov[kMaxLongSplits + 1];
+    uint4 ov[kMaxLongSplits + 1][kCombineVec];
 #pragma unroll
     for (int s = 0; s <= kMaxLongSplits; ++s) {
         const bool own = s == kMaxLongSplits;
         l[s] = -INFINITY;
-        ov[s] = make_uint2(0u, 0u);
+#pragma unroll
+        for (int v = 0; v < kCombineVec; ++v) ov[s][v] = make_uint4(0u, 0u, 0u, 0u);
         if (own || s < parts) {
             l[s] = (own ? a.lse_b[li] : a.lse_a[s * slice_l + li]) * kLog2eF;
-            ov[s] = *reinterpret_cast<const uint2 *>((own ? a.ob : a.oa + s * slice_o) + row * kD + c4);
+            const uint4 *src = reinterpret_cast<const uint4 *>((own ? a.ob : a.oa + s * slice_o) + oi);
+#pragma unroll
+            for (int v = 0; v < kCombineVec; ++v) ov[s][v] = src[v];
         }
     }
     float M = -INFINITY;
 #pragma unroll
     for (int s = 0; s <= kMaxLongSplits; ++s) M = fmaxf(M, l[s]);
-    float den = 0.f;
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f, num[kCombineDims];
+#pragma unroll
+    for (int e = 0; e < kCombineDims; ++e) num[e] = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
         for (int s = 0; s <= kMaxLongSplits; ++s) {
             if (l[s] == -INFINITY) continue;
             const float wgt = ex2_approx(l[s] - M);
-            float f[4];
-            unpack_bf16x4(ov[s], f);
             den += wgt;
-            num.x += wgt * f[0];
-            num.y += wgt * f[1];
-            num.z += wgt * f[2];
-            num.w += wgt * f[3];
+#pragma unroll
+            for (int e = 0; e < kCombineDims / 2; ++e) {
+                const uint4 &q = ov[s][e >> 2];
+                const uint32_t wv = (e & 3) == 0 ? q.x : (e & 3) == 1 ? q.y : (e & 3) == 2 ? q.z : q.w;
+                num[2 * e] = fmaf(wgt, __uint_as_float(wv << 16), num[2 * e]);
+                num[2 * e + 1] = fmaf(wgt, __uint_as_float(wv & 0xffff0000u), num[2 * e + 1]);
+            }
         }
     }
-    const float g_head = a.gate_mode == 2 ? __bfloat162float(a.gate[row]) : 0.f;
-    *reinterpret_cast<uint2 *>(a.out + row * kD + c4) =
-        fold_out4(num, den, a.gate_mode, a.gate_mode == 1 ? a.gate + row * kD + c4 : nullptr, g_head);
-    if (a.lse != nullptr && c4 == 0) a.lse[row] = den > 0.f ? (M + __log2f(den)) * kLn2F : -INFINITY;
+    // O = num / den, times the sigmoid of the output gate (per channel or per head)
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int e = 0; e < kCombineDims; ++e) num[e] *= inv;
+    if (a.gate_mode == 1) {
+        const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + oi);
+#pragma unroll
+        for (int v = 0; v < kCombineVec; ++v) {
+            const uint4 g = gp[v];
+            const uint32_t gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float gx = __uint_as_float(e & 1 ? (gv[e >> 1] & 0xffff0000u) : (gv[e >> 1] << 16));
+                num[8 * v + e] = __fdividef(num[8 * v + e], 1.f + ex2_approx(-gx * kLog2eF));
+            }
+        }
+    } else if (a.gate_mode == 2) {
+        const float gs = 1.f / (1.f + ex2_approx(-__bfloat162float(a.gate[row]) * kLog2eF));
+#pragma unroll
+        for (int e = 0; e < kCombineDims; ++e) num[e] *= gs;
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(a.out + oi);
+#pragma unroll
+    for (int v = 0; v < kCombineVec; ++v)
+        dst[v] = make_uint4(pack_bf16x2(num[8 * v], num[8 * v + 1]), pack_bf16x2(num[8 * v + 2], num[8 * v + 3]),
+                            pack_bf16x2(num[8 * v + 4], num[8 * v + 5]), pack_bf16x2(num[8 * v + 6], num[8 * v + 7]));
+    if (a.lse != nullptr && c16 == 0) a.lse[row] = den > 0.f ? (M + __log2f(den)) * kLn2F : -INFINITY;
 }
 
 }  // namespace duo

@@ -668,6 +668,9 @@ int long_block(const duo_params *params, const Layout &L, const duo_cache *cache
                const void *k_new, const void *v_new, int32_t q_len, int32_t max_seq_len, void *out, float *lse,
                void *workspace, int gate_mode, const void *gate_values, int sms, cudaStream_t st) {
     const LongBlockPlan pl = long_block_plan(params, L, q_len, max_seq_len, sms);
+    if ((int64_t)params->batch * q_len * params->num_q_heads > INT32_MAX)
+        return fail(DUO_ERR_UNSUPPORTED, "batch x q_len x query heads must be below 2^31 for a block of %d tokens",
+                    q_len);
     char *w = (char *)workspace;
     void *oa = w;                                                  // [S][B][q_len][Hq][D]
     void *ob = w + (size_t)pl.kv_splits * pl.o_bytes;              // [B][q_len][Hq][D]
@@ -704,7 +707,8 @@ int long_block(const duo_params *params, const Layout &L, const duo_cache *cache
     c.capacity = L.n_full > 0 ? (int32_t)std::min<int64_t>(cache->capacity, INT32_MAX) : 0;
     c.seq_len = cache->seq_len;
     for (int g = 0; g < params->num_kv_heads; ++g) c.is_full[g] = L.heads.is_full[g];
-    duo::block_combine<<<(unsigned)((int64_t)params->batch * q_len * params->num_kv_heads), duo::kMergeThreads, 0,
+    const int64_t rows = (int64_t)params->batch * q_len * params->num_q_heads;
+    duo::block_combine<<<(unsigned)((rows + duo::kCombineRows - 1) / duo::kCombineRows), duo::kCombineThreads, 0,
                          st>>>(c);
     return launch_status("block_combine");
 }
