@@ -50,6 +50,7 @@ template <int kQ>
 struct BlockCfg {
     static constexpr int NR = kGroup * kQ;                       // query rows per item
     static constexpr int RQ = (NR + 3) / 4;                      // rows per TMEM lane quarter
+    static_assert(RQ <= 16, "an M = 64 product holds 16 rows per lane quarter");
     static constexpr int Stages = 3;
     static constexpr size_t Smem = 1024 + Stages * kDecStageBytes;
     static_assert(Smem + 2048 <= 232448, "shared memory");
@@ -301,8 +302,11 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         // as its inputs land and takes no issue slots from the softmax warp on
         // its sub-partition meanwhile.
         if (lane == 0) {
-            const uint32_t id_qk = idesc_bf16_f32(128, kTok, 0, 0);
-            const uint32_t id_pv = idesc_bf16_f32(128, kD, 0, 1);
+            // M = 64: the product's 64 rows sit in lanes 0-15 of each 32-lane
+            // quarter of tensor memory, where the item's (at most 12 per quarter)
+            // query rows are, at half the tensor work of M = 128
+            const uint32_t id_qk = idesc_bf16_f32(64, kTok, 0, 0);
+            const uint32_t id_pv = idesc_bf16_f32(64, kD, 0, 1);
             const uint32_t kv_addr = smem_u32(sKV);
             constexpr int kInfo = 8;
             __shared__ int info_w[kInfo], info_n[kInfo];   // items by fetch order: work index, tiles
