@@ -8,8 +8,9 @@
 // token's cos / sin table once (the angle p * inv_freq in double precision and
 // reduced modulo 2 pi in double, so that positions up to 2^30 keep their
 // phase), then 8 threads per head row normalise it, rotate the pairs
-// (i, i + 64) and write it back in place; key rows also go to the cache with
-// their values, with the append's survivor rule for ring heads.
+// (i, i + 64) and write it back in place; key rows also go to the cache, and
+// so do the values (loaded when the CTA starts), with the append's survivor
+// rule for ring heads.
 #pragma once
 
 #include "kv_append.cuh"
@@ -42,7 +43,7 @@ constexpr int kPrepBatch = 4;       // head rows an 8-thread group has in flight
 // channels [8j, 8j + 8) and their rotation partners [64 + 8j, 64 + 8j + 8), so
 // that the rotation needs no exchange between threads and every load and store
 // is 16 bytes wide; the sum of squares is reduced over the 8 threads.
-__global__ void __launch_bounds__(kPrepThreads) qk_prep_append(const __grid_constant__ PrepArgs a) {
+__global__ void __launch_bounds__(kPrepThreads, 4) qk_prep_append(const __grid_constant__ PrepArgs a) {
     pdl_wait();        // launched as a programmatic dependent of the previous kernel
     const AppendArgs &ap = a.app;
     const int tok = blockIdx.x;
@@ -57,6 +58,22 @@ __global__ void __launch_bounds__(kPrepThreads) qk_prep_append(const __grid_cons
         return r < a.hq ? a.q + (tok_row * a.hq + r) * kVecPerRow
                         : a.kw + (tok_row * ap.hkv + (r - a.hq)) * kVecPerRow;
     };
+    // the value rows that survive the append go straight to the cache: thread c
+    // of the first pass holds chunk c % 16 of head c / 16, loaded first so that
+    // the load overlaps the table and the rotation (heads past the first pass
+    // are copied at the end)
+    const int vc = threadIdx.x;
+    uint4 vpre = make_uint4(0, 0, 0, 0);
+    uint4 *vdst = nullptr;
+    if (vc < ap.hkv * kVecPerRow) {
+        const int g = vc / kVecPerRow;
+        bool full = false;
+        const int64_t row = append_row(ap, b, g, t, &full);
+        if (row >= 0) {
+            vpre = ap.v[(tok_row * ap.hkv + g) * kVecPerRow + vc % kVecPerRow];
+            vdst = (full ? ap.full_v : ap.strm_v) + row * kVecPerRow + vc % kVecPerRow;
+        }
+    }
     // the first batch of rows in flight before the cos / sin table is built
     uint4 xlo[kPrepBatch], xhi[kPrepBatch];
 #pragma unroll
@@ -147,17 +164,21 @@ __global__ void __launch_bounds__(kPrepThreads) qk_prep_append(const __grid_cons
                 bool full = false;
                 const int64_t row = append_row(ap, b, g, t, &full);
                 if (row >= 0) {
-                    const uint4 *vr = ap.v + (tok_row * ap.hkv + g) * kVecPerRow;
-                    const uint4 v_lo = vr[j], v_hi = vr[8 + j];
                     uint4 *kd = (full ? ap.full_k : ap.strm_k) + row * kVecPerRow;
-                    uint4 *vd = (full ? ap.full_v : ap.strm_v) + row * kVecPerRow;
                     kd[j] = out_lo;
                     kd[8 + j] = out_hi;
-                    vd[j] = v_lo;
-                    vd[8 + j] = v_hi;
                 }
             }
         }
+    }
+    if (vdst != nullptr) *vdst = vpre;
+    for (int c = vc + kPrepThreads; c < ap.hkv * kVecPerRow; c += kPrepThreads) {
+        const int g = c / kVecPerRow;
+        bool full = false;
+        const int64_t row = append_row(ap, b, g, t, &full);
+        if (row >= 0)
+            ((full ? ap.full_v : ap.strm_v) + row * kVecPerRow)[c % kVecPerRow] =
+                ap.v[(tok_row * ap.hkv + g) * kVecPerRow + c % kVecPerRow];
     }
 }
 
