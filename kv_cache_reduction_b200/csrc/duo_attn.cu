@@ -203,14 +203,17 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Items are processed by one persistent CTA per SM, round robin.  Full-head
 // caches are cut into equal chunks of whole 128-token tiles; the chunk count
 // is the one that minimises the estimated makespan (tiles of the busiest
-// CTA plus a small per-item cost).  Ring heads take one item each unless
+// CTA plus a per-item cost).  Ring heads take one item each unless
 // there are too few of them to occupy the SMs.
 DecodePlan plan_decode(const duo_params *p, const Layout &L, int64_t max_n, int sms) {
     DecodePlan d;
     const int64_t ring_units = (int64_t)p->batch * L.n_ring;
     const int64_t full_units = (int64_t)p->batch * L.n_full;
     const int64_t ring_tiles = cdiv(L.slots, duo::kTok);
-    const double item_cost = 0.5;      // pipeline fill and epilogue, in tiles
+    // pipeline fill and epilogue, in tiles: the value that fits the measured
+    // decode times over split counts (B=32 at 32768 tokens: 9, 16, 20, 32 and
+    // 12 splits rank as the model ranks them)
+    const double item_cost = 1.5;
     if (ring_units > 0) {
         int64_t want = 1;
         if (full_units == 0 || max_n <= 4 * L.slots)
