@@ -692,7 +692,7 @@ class ChunkPrefill:
         self.launches_per_step = 3      # prefill_fwd twice (cached keys, own keys) + block_combine
         self.unit = "TFLOP/s"
         self.kernel = "prefill_fwd (cache mode) + prefill_fwd + block_combine (one duo_attn_decode_block call)"
-        self.traffic_key = ("prefill_fwd", "chunk_32k")
+        self.traffic_key = ("prefill_fwd+block_combine", "chunk_32k")
 
     def step(self):
         duo.duo_attn_decode_block(self.params, self.cache, self.q, self.kb, self.vb, self.CACHED,
@@ -1008,7 +1008,9 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
 KERNEL_SOURCES = {"decode_split": ("decode.cuh", "ptx.cuh", "kv_append.cuh"),
                   "prefill_fwd": ("prefill.cuh", "ptx.cuh"),
                   "decode_block_split": ("decode_block.cuh", "decode.cuh", "ptx.cuh", "kv_append.cuh"),
-                  "qk_prep_append": ("qk_prep.cuh", "kv_append.cuh", "ptx.cuh")}
+                  "qk_prep_append": ("qk_prep.cuh", "kv_append.cuh", "ptx.cuh"),
+                  # the chunked-prefill step: both prefill_fwd passes and block_combine
+                  "prefill_fwd+block_combine": ("prefill.cuh", "decode_block.cuh", "ptx.cuh")}
 
 
 def sources_digest(kernel: str) -> str:

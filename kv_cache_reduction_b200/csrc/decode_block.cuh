@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(BlockCfg<kQ>::Threads, 1) decode_block_split(c
         if (lane == 0) {
             // M = 64: the product's 64 rows sit in lanes 0-15 of each 32-lane
             // quarter of tensor memory, where the item's (at most 12 per quarter)
-            // query rows are, at half the tensor work of M = 128
+            // query rows are: half the multiply-adds of M = 128
             const uint32_t id_qk = idesc_bf16_f32(64, kTok, 0, 0);
             const uint32_t id_pv = idesc_bf16_f32(64, kD, 0, 1);
             const uint32_t kv_addr = smem_u32(sKV);
