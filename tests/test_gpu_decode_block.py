@@ -173,6 +173,38 @@ def test_long_block_duo_layer(cuda_device, q_len):
     block_case(p, o, cache, q_len, seed=190 + q_len, max_seq_len=3000)
 
 
+def test_long_block_repeat_is_bitwise_stable(cuda_device):
+    """The two passes of a long block share the SMs (the pass over the block's
+    own keys is a programmatic dependent launch of the pass over the cached
+    keys) and the fold reads both: 30 calls on the same inputs give identical
+    bytes, the first one matching the oracle.  A fold that read a slice before
+    its pass had written it shows up as a call that differs."""
+    p, o = layers(4, full_mask=(1, 0, 0, 1, 0, 1, 1, 0))
+    seq, rh = [0, 320, 1500, 3000], [0, 0, 99, 77]
+    cache = random_cache(p, 3000, seq, rh, seed=214)
+    q_len = 300
+    block_case(p, o, cache, q_len, seed=215, max_seq_len=3000)     # inputs from seeds 215, 216, 217
+    B = p.batch
+    q = inputs.randn_bf16((B, q_len, 48, 128), 215, "cuda")
+    kn = inputs.randn_bf16((B, q_len, 8, 128), 216, "cuda")
+    vn = inputs.randn_bf16((B, q_len, 8, 128), 217, "cuda")
+    n = duo.duo_decode_block_workspace_bytes(p, q_len, 3000)
+    ws = torch.empty(((n + 255) // 256 * 256,), dtype=torch.uint8, device="cuda")
+    ref_out = torch.empty((B, q_len, 48, 128), dtype=torch.bfloat16, device="cuda")
+    ref_lse = torch.empty((B, q_len, 48), dtype=torch.float32, device="cuda")
+    duo.duo_attn_decode_block(p, cache, q, kn, vn, 3000, ref_out, ref_lse, ws)
+    torch.cuda.synchronize()
+    assert duo.duo_get_device_status() == duo.DUO_OK
+    out = torch.empty_like(ref_out)
+    lse = torch.empty_like(ref_lse)
+    for i in range(30):
+        duo.duo_attn_decode_block(p, cache, q, kn, vn, 3000, out, lse, ws)
+        torch.cuda.synchronize()
+        assert duo.duo_get_device_status() == duo.DUO_OK
+        assert torch.equal(out, ref_out), f"call {i}: output differs"
+        assert torch.equal(lse, ref_lse), f"call {i}: lse differs"
+
+
 @pytest.mark.parametrize("q_len", [200, 700])
 def test_long_block_sliding_layer_with_sink(cuda_device, q_len):
     sig = inputs.randn_f32((48,), 200)
