@@ -590,9 +590,19 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_fwd(const __grid_consta
                     const uint64_t m0 = col_range_bits(lo0, hi0) | col_range_bits(lo1, hi1);
                     const uint64_t m1 = col_range_bits(lo0 - 64, hi0 - 64) | col_range_bits(lo1 - 64, hi1 - 64);
                     const uint32_t mw[4] = {(uint32_t)m0, (uint32_t)(m0 >> 32), (uint32_t)m1, (uint32_t)(m1 >> 32)};
+                    // a warp's 32 consecutive rows have their range ends within 32
+                    // columns of one another: a 16-column chunk that every row keeps
+                    // (or none does) is passed over (or cleared) whole, and only the
+                    // few chunks in between are masked column by column
 #pragma unroll
-                    for (int cc = 0; cc < 128; ++cc)
-                        if (!((mw[cc >> 5] >> (cc & 31)) & 1u)) sr[cc] = __float_as_uint(-INFINITY);
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t bits = (mw[k >> 1] >> (16 * (k & 1))) & 0xffffu;
+                        if (!__all_sync(0xffffffffu, bits == 0xffffu)) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                if (!((bits >> e) & 1u)) sr[16 * k + e] = __float_as_uint(-INFINITY);
+                        }
+                    }
                 }
                 // the row max over the tile, eight independent chains of 3-input max
                 float mx8[8];
