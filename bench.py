@@ -828,8 +828,8 @@ class DecodeSmall:
         self.lse = torch.empty((S, 1, 48), dtype=torch.float32, device="cuda")
         self.flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")   # 2 x L2
         self.unit = "us/step"
-        self.kernel = "kv_append_scatter + kv_append_commit + decode_split + decode_merge"
-        self.launches_per_step = 4
+        self.kernel = "kv_append_small + decode_split + decode_merge"
+        self.launches_per_step = 3
         self.graph = None
         if product:
             self.ws_p = torch.empty(duo.duo_prefill_workspace_bytes(), dtype=torch.uint8, device="cuda")

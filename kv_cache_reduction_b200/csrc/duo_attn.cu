@@ -399,6 +399,13 @@ int duo_kv_append(const duo_params *params, const duo_cache *cache, const void *
     int rc = append_args(params, cache, k, v, n_new, &L, &a);
     if (rc || n_new == 0) return rc;
     cudaStream_t st = (cudaStream_t)stream;
+    if ((int64_t)n_new * params->num_kv_heads * duo::kVecPerRow <= duo::kAppendSmallMaxVecs) {
+        // a short append: copy and commit in one launch, one CTA per sequence
+        if (launch_pdl(duo::kv_append_small, dim3((unsigned)params->batch), dim3(duo::kAppendSmallThreads), 0, st,
+                       a) != cudaSuccess)
+            return launch_status("kv_append_small");
+        return launch_status("kv_append_small");
+    }
     const int64_t vecs = (int64_t)params->batch * n_new * params->num_kv_heads * duo::kVecPerRow;
     const int64_t blocks = (vecs + 255) / 256;
     if (blocks > INT32_MAX) return fail(DUO_ERR_INVALID_ARG, "append too large for one launch");

@@ -24,8 +24,8 @@ struct AppendArgs {
     const uint4 *v;
     uint4 *full_k, *full_v;   // [B][n_full][capacity][D]
     uint4 *strm_k, *strm_v;   // [B][n_ring][slots][D]
-    const int32_t *seq_len;
-    const int32_t *ring_head;
+    int32_t *seq_len;     // read by the copies, moved forward by the commit
+    int32_t *ring_head;
     int64_t capacity;
     int32_t batch, n_new, hkv, n_full, n_ring;
     int32_t sink, ring, slots;    // ring = recent (Duo) or window (sliding)
@@ -90,19 +90,54 @@ __global__ void __launch_bounds__(256) kv_append_scatter(AppendArgs a) {
     dv[vec] = a.v[idx];
 }
 
-// Moves seq_len and ring_head forward once the scatter has read them (to the
-// append's end, which stops at the capacity as append_end says).
-__global__ void kv_append_commit(int32_t *seq_len, int32_t *ring_head, int32_t batch, int32_t n_new,
-                                 int32_t sink, int32_t ring, int32_t n_full, int64_t capacity) {
-    pdl_wait();        // the scatter has read seq_len and ring_head
-    const int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= batch) return;
+// Moves sequence b's seq_len and ring_head forward (to the append's end, which
+// stops at the capacity as append_end says); every read of them is done.
+__device__ __forceinline__ void commit_sequence(int32_t *seq_len, int32_t *ring_head, int b, int32_t n_new,
+                                                int32_t sink, int32_t ring, int32_t n_full, int64_t capacity) {
     const int64_t n_old = seq_len[b];
     const int64_t n_end = append_end(n_old, n_new, n_full, capacity);
     const int64_t first = n_old > sink ? n_old : sink;
     const int64_t ring_writes = n_end > first ? n_end - first : 0;
     ring_head[b] = (int32_t)(((int64_t)ring_head[b] + ring_writes) % ring);
     seq_len[b] = (int32_t)n_end;
+}
+
+// Moves seq_len and ring_head forward once the scatter has read them.
+__global__ void kv_append_commit(int32_t *seq_len, int32_t *ring_head, int32_t batch, int32_t n_new,
+                                 int32_t sink, int32_t ring, int32_t n_full, int64_t capacity) {
+    pdl_wait();        // the scatter has read seq_len and ring_head
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= batch) return;
+    commit_sequence(seq_len, ring_head, b, n_new, sink, ring, n_full, capacity);
+}
+
+// A short append (a decode step, a verify block) in one launch: one CTA per
+// sequence copies that sequence's n_new x Hkv rows (16-byte vectors in input
+// order, as the scatter does) and then moves its seq_len and ring_head
+// forward itself: no other CTA reads them, so the commit needs no second
+// kernel.
+constexpr int kAppendSmallThreads = 256;
+constexpr int kAppendSmallMaxVecs = 4096;     // n_new x Hkv x 16 vectors of a sequence, at most
+
+__global__ void __launch_bounds__(kAppendSmallThreads) kv_append_small(AppendArgs a) {
+    pdl_wait();        // launched as a programmatic dependent of the previous kernel
+    const int b = blockIdx.x;
+    const int per_seq = a.n_new * a.hkv * kVecPerRow;
+    const int64_t base = (int64_t)b * per_seq;
+    for (int i = threadIdx.x; i < per_seq; i += kAppendSmallThreads) {
+        const int vec = i % kVecPerRow;
+        const int row = i / kVecPerRow;            // t * Hkv + g
+        const int g = row % a.hkv;
+        const int64_t t = row / a.hkv;
+        bool full = false;
+        const int64_t r = append_row(a, b, g, t, &full);
+        if (r < 0) continue;
+        (full ? a.full_k : a.strm_k)[r * kVecPerRow + vec] = a.k[base + i];
+        (full ? a.full_v : a.strm_v)[r * kVecPerRow + vec] = a.v[base + i];
+    }
+    __syncthreads();   // this CTA's reads of seq_len[b] and ring_head[b] are done
+    if (threadIdx.x == 0)
+        commit_sequence(a.seq_len, a.ring_head, b, a.n_new, a.sink, a.ring, a.n_full, a.capacity);
 }
 
 }  // namespace duo
