@@ -28,7 +28,10 @@ def run_and_compare(params, o_layer, cache, chunks, seed):
         assert np.array_equal(getattr(got, name), getattr(ref, name)), name
 
 
-@pytest.mark.parametrize("chunks", [[1] * 20, [1000], [64, 300, 1, 1, 700], [65], [320, 1], [3, 5000]])
+# 32 tokens x 8 KV heads is the longest append done in one launch (kv_append_small),
+# 33 the shortest done by the scatter and the commit
+@pytest.mark.parametrize("chunks", [[1] * 20, [1000], [64, 300, 1, 1, 700], [65], [320, 1], [3, 5000],
+                                    [32, 33, 32, 1]])
 def test_append_duo_layer(cuda_device, chunks):
     p, o = layers(2, full_mask=(1, 0, 0, 1, 0, 1, 1, 0))
     cache = random_cache(p, 6200, [0, 0], [0, 0], seed=7)
