@@ -466,6 +466,7 @@ int duo_kv_append_prep(const duo_params *params, const duo_cache *cache, const d
     cudaStream_t st = (cudaStream_t)stream;
     if (launch_pdl(duo::qk_prep_append, dim3((unsigned)blocks), dim3(duo::kPrepThreads), 0, st, a) != cudaSuccess)
         return launch_status("qk_prep_append");
+    if (n_new == 1) return launch_status("qk_prep_append");     // it committed the one token itself
     if (launch_pdl(duo::kv_append_commit, dim3((params->batch + 127) / 128), dim3(128), 0, st, cache->seq_len,
                    cache->ring_head, params->batch, n_new, L.sink, L.ring, L.n_full, a.app.capacity) != cudaSuccess)
         return launch_status("kv_append_commit");

@@ -10,7 +10,7 @@
 // phase), then 8 threads per head row normalise it, rotate the pairs
 // (i, i + 64) and write it back in place; key rows also go to the cache, and
 // so do the values (loaded when the CTA starts), with the append's survivor
-// rule for ring heads.
+// rule for ring heads.  A one-token append is committed by its CTA.
 #pragma once
 
 #include "kv_append.cuh"
@@ -179,6 +179,12 @@ __global__ void __launch_bounds__(kPrepThreads, 4) qk_prep_append(const __grid_c
         if (row >= 0)
             ((full ? ap.full_v : ap.strm_v) + row * kVecPerRow)[c % kVecPerRow] =
                 ap.v[(tok_row * ap.hkv + g) * kVecPerRow + c % kVecPerRow];
+    }
+    // a one-token append (a decode step): this CTA is its sequence's only one, so
+    // it moves seq_len and ring_head forward itself once all its reads are done
+    if (ap.n_new == 1) {
+        __syncthreads();
+        if (threadIdx.x == 0) commit_sequence(ap.seq_len, ap.ring_head, b, 1, ap.sink, ap.ring, ap.n_full, ap.capacity);
     }
 }
 
