@@ -468,49 +468,48 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_split(const __grid_cons
     }
 }
 
-// The split fold of one output element: M = max(M, m_s) over the splits, then
-// den = sum_s 2^(m_s - M) l_s and num = sum_s 2^(m_s - M) acc_s in split order
-// (splits with m_s = -inf skipped).  m_s, l_s, acc_s sit at floats m_off,
-// l_off, a_off of split s's record of `stride` floats.  The partials were
-// written by the previous grid and sit in L2: the loads go out kFoldBatch
-// splits at a time (only real records are read), so a fold costs about two L2
-// round trips per batch instead of two per split.
+// The split fold of one output element in one pass: with M entering as the
+// sink logit (log2 units) or -inf and den = num = 0, it leaves
+// M = max(M, m_s) over the splits, den = sum_s 2^(m_s - M) l_s and
+// num = sum_s 2^(m_s - M) acc_s (splits with m_s = -inf skipped).  m_s, l_s,
+// acc_s sit at floats m_off, l_off, a_off of split s's record of `stride`
+// floats.  The partials were written by the previous grid and sit in L2: the
+// loads go out kFoldBatch splits at a time (only real records are read), the
+// running max rises batch by batch and the sums so far are rescaled when it
+// does, so a fold costs one L2 round trip per batch.
 template <int kFoldBatch>
 __device__ __forceinline__ void fold_splits(const float *part, int stride, int splits, int m_off, int l_off,
                                             int a_off, float *M_io, float *den_io, float *num_io) {
-    float M = *M_io;
+    float M = *M_io, den = 0.f, num = 0.f;
     for (int s0 = 0; s0 < splits; s0 += kFoldBatch) {
-        float mv[kFoldBatch];
+        float mv[kFoldBatch], lv[kFoldBatch], av[kFoldBatch];
 #pragma unroll
         for (int i = 0; i < kFoldBatch; ++i) {
             mv[i] = -INFINITY;
-            if (s0 + i < splits) mv[i] = part[(s0 + i) * stride + m_off];
+            lv[i] = av[i] = 0.f;
+            if (s0 + i < splits) {
+                const float *ps = part + (s0 + i) * stride;
+                mv[i] = ps[m_off];
+                lv[i] = ps[l_off];
+                av[i] = ps[a_off];
+            }
+        }
+        float Mb = M;
+#pragma unroll
+        for (int i = 0; i < kFoldBatch; ++i) Mb = fmaxf(Mb, mv[i]);
+        if (Mb == -INFINITY) continue;
+        if (Mb > M) {
+            const float r = ex2_approx(M - Mb);       // 0 while M is -inf (the sums are 0 then)
+            den *= r;
+            num *= r;
+            M = Mb;
         }
 #pragma unroll
-        for (int i = 0; i < kFoldBatch; ++i) M = fmaxf(M, mv[i]);
-    }
-    float den = 0.f, num = 0.f;
-    if (M != -INFINITY) {
-        for (int s0 = 0; s0 < splits; s0 += kFoldBatch) {
-            float mv[kFoldBatch], lv[kFoldBatch], av[kFoldBatch];
-#pragma unroll
-            for (int i = 0; i < kFoldBatch; ++i) {
-                mv[i] = -INFINITY;
-                lv[i] = av[i] = 0.f;
-                if (s0 + i < splits) {
-                    const float *ps = part + (s0 + i) * stride;
-                    mv[i] = ps[m_off];
-                    lv[i] = ps[l_off];
-                    av[i] = ps[a_off];
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < kFoldBatch; ++i) {
-                if (mv[i] == -INFINITY) continue;
-                const float f = ex2_approx(mv[i] - M);
-                den += f * lv[i];
-                num += f * av[i];
-            }
+        for (int i = 0; i < kFoldBatch; ++i) {
+            if (mv[i] == -INFINITY) continue;
+            const float f = ex2_approx(mv[i] - M);
+            den += f * lv[i];
+            num += f * av[i];
         }
     }
     *M_io = M;
@@ -518,55 +517,49 @@ __device__ __forceinline__ void fold_splits(const float *part, int stride, int s
     *num_io = num;
 }
 
-// The split fold of four consecutive output elements: M = max(M, m_s) over
-// the splits, then den = sum_s 2^(m_s - M) l_s and num = sum_s 2^(m_s - M)
-// acc_s in split order (splits with m_s = -inf skipped).  m_s, l_s sit at
-// floats m_off, l_off of split s's record of `stride` floats, the four acc_s at
-// a_off (16-byte aligned).  The partials were written by the previous grid and
-// sit in L2: the loads go out kFoldBatch splits at a time (only real records
-// are read), so a fold costs about two L2 round trips per batch.
+// fold_splits for four consecutive output elements (acc_s a float4 at a_off).
 template <int kFoldBatch>
 __device__ __forceinline__ void fold_splits4(const float *part, int stride, int splits, int m_off, int l_off,
                                              int a_off, float *M_io, float *den_io, float4 *num_io) {
-    float M = *M_io;
+    float M = *M_io, den = 0.f;
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = 0; s0 < splits; s0 += kFoldBatch) {
-        float mv[kFoldBatch];
+        float mv[kFoldBatch], lv[kFoldBatch];
+        float4 av[kFoldBatch];
 #pragma unroll
         for (int i = 0; i < kFoldBatch; ++i) {
             mv[i] = -INFINITY;
-            if (s0 + i < splits) mv[i] = part[(s0 + i) * stride + m_off];
+            lv[i] = 0.f;
+            av[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s0 + i < splits) {
+                const float *ps = part + (s0 + i) * stride;
+                mv[i] = ps[m_off];
+                lv[i] = ps[l_off];
+                av[i] = *reinterpret_cast<const float4 *>(ps + a_off);
+            }
+        }
+        float Mb = M;
+#pragma unroll
+        for (int i = 0; i < kFoldBatch; ++i) Mb = fmaxf(Mb, mv[i]);
+        if (Mb == -INFINITY) continue;
+        if (Mb > M) {
+            const float r = ex2_approx(M - Mb);
+            den *= r;
+            num.x *= r;
+            num.y *= r;
+            num.z *= r;
+            num.w *= r;
+            M = Mb;
         }
 #pragma unroll
-        for (int i = 0; i < kFoldBatch; ++i) M = fmaxf(M, mv[i]);
-    }
-    float den = 0.f;
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-        for (int s0 = 0; s0 < splits; s0 += kFoldBatch) {
-            float mv[kFoldBatch], lv[kFoldBatch];
-            float4 av[kFoldBatch];
-#pragma unroll
-            for (int i = 0; i < kFoldBatch; ++i) {
-                mv[i] = -INFINITY;
-                lv[i] = 0.f;
-                av[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (s0 + i < splits) {
-                    const float *ps = part + (s0 + i) * stride;
-                    mv[i] = ps[m_off];
-                    lv[i] = ps[l_off];
-                    av[i] = *reinterpret_cast<const float4 *>(ps + a_off);
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < kFoldBatch; ++i) {
-                if (mv[i] == -INFINITY) continue;
-                const float f = ex2_approx(mv[i] - M);
-                den += f * lv[i];
-                num.x += f * av[i].x;
-                num.y += f * av[i].y;
-                num.z += f * av[i].z;
-                num.w += f * av[i].w;
-            }
+        for (int i = 0; i < kFoldBatch; ++i) {
+            if (mv[i] == -INFINITY) continue;
+            const float f = ex2_approx(mv[i] - M);
+            den += f * lv[i];
+            num.x += f * av[i].x;
+            num.y += f * av[i].y;
+            num.z += f * av[i].z;
+            num.w += f * av[i].w;
         }
     }
     *M_io = M;
